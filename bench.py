@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step on one node (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config opt13b]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+A step is one decode round of the whole hot path for one batch of running
+sequences, through the library's decode-step runtime (``pkv_decode_step``):
+host block-table update with copy-on-write, one table upload, block copy,
+append of the new K/V rows, paged decode attention and the split-context
+merge.  The metric is KV GB/s: sum over the batch of context_len x 2 x H_kv x d
+x bytes (the bytes attention must read), per second, in 10^9 B/s.
+
+Inputs: the workload's shapes (``workloads.CONFIGS``), K/V histories drawn on
+the GPU from a seeded torch generator and written through ``kv_append``.  The
+pool holds ``--replicas`` independent batches of the workload; step k runs
+batch k mod replicas, so contexts grow by only steps/replicas tokens during
+the run and every step streams the whole batch's KV from HBM (far more than
+the 126 MB L2).  Multi-GPU: each rank runs its own pool and batches (weak
+scaling, no collective on the data path); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode KV GB/s (% of B200 HBM peak); attended tokens/sec at 1 GPU"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=600)
+    ap.add_argument("--warmup", type=int, default=12)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="opt13b", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--variant", default="b", choices=["a", "b"])
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=0, help="default: steps // 3")
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--kernel", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def config_of(args) -> wl.Config:
+    cfg = wl.CONFIGS[args.config]
+    if args.block_size:
+        cfg = cfg.with_block_size(args.block_size)
+    return cfg
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, polled)
+# ---------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(torch_device)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((sm, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_sm, "reasons": [], "samples": 0}
+        sms = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        return {"sm_mhz": float(statistics.median(sms)), "sm_max_mhz": int(self.max_sm),
+                "reasons": [n for b, n in REASONS.items() if bits & b and b != 0x1],
+                "samples": len(sms)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg: wl.Config, target_bytes: float, seed: int = 0):
+    """The first sequences of the workload whose KV bytes reach target_bytes,
+    admitted into a fresh oracle (set-up, not timed)."""
+    from oracle.engine import DecodeOracle
+    lens = wl.history_lengths(cfg, seed, "b")
+    per = cfg.samples_per_prompt
+    seqs, tot = [], 0
+    for i in range(cfg.batch):
+        n = int(lens[i // per]) if per > 1 else int(lens[i])
+        seqs.append(i)
+        tot += (n + 1) * cfg.kv_bytes_per_token
+        if tot >= target_bytes:
+            break
+    nb = sum(-(-(int(lens[i // per] if per > 1 else lens[i]) + 64) // cfg.block_size) + 2
+             for i in seqs)
+    ks = vs = 1.0
+    if cfg.kv_dtype == "fp8":
+        ks, vs = wl.fp8_scales_for(cfg, seed, [lens[i] for i in seqs], steps=1)
+    orc = DecodeOracle(nb, cfg.block_size, cfg.n_kv_heads, cfg.head_dim, cfg.kv_dtype, ks, vs,
+                       order=wl.free_order(nb, seed, cfg.permute))
+    for i in seqs:
+        src = i // per if per > 1 else i
+        n = int(lens[src])
+        k, v = wl.history_kv(cfg, seed, src, n)
+        orc.admit(i, wl.round_to(k, cfg.q_dtype), wl.round_to(v, cfg.q_dtype), cfg.q_dtype)
+    return orc, seqs
+
+
+def oracle_step(orc, cfg, seqs, step):
+    q, k, v = [], [], []
+    for s in seqs:
+        a, b, c = wl.step_qkv(cfg, 0, s, step)
+        q.append(a), k.append(b), v.append(c)
+    q = wl.round_to(np.stack(q), cfg.q_dtype)
+    k = wl.round_to(np.stack(k), cfg.q_dtype)
+    v = wl.round_to(np.stack(v), cfg.q_dtype)
+    t0 = time.perf_counter()
+    orc.step(seqs, q, k, v, cfg.q_dtype, cfg.scale)
+    dt = time.perf_counter() - t0
+    nbytes = sum(orc.bm.lengths[s] for s in seqs) * cfg.kv_bytes_per_token
+    return dt, nbytes
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(cfg: wl.Config, budget_s: float) -> dict:
+    """The oracle as it stands on a bounded sample of the workload: one warm-up
+    step, then oracle decode steps (append then attend) until the budget is
+    spent; GB/s over the same byte definition."""
+    orc, seqs = oracle_sample(cfg, target_bytes=64e6)
+    oracle_step(orc, cfg, seqs, 0)
+    times, nbytes = [], []
+    t_end = time.perf_counter() + budget_s
+    step = 1
+    while time.perf_counter() < t_end and step < 200:
+        dt, nb = oracle_step(orc, cfg, seqs, step)
+        times.append(dt)
+        nbytes.append(nb)
+        step += 1
+    gbs = sum(nbytes) / sum(times) / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(seqs)} of {cfg.batch} sequences of the workload, {len(times)} "
+                      f"decode steps (append + fp64 attention), median step "
+                      f"{statistics.median(times) * 1e3:.1f} ms"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = config_of(args)
+    # per step a bounded sample sized so that the whole run stays within minutes
+    orc, seqs = oracle_sample(cfg, target_bytes=24e6)
+    for s in range(args.warmup):
+        oracle_step(orc, cfg, seqs, s)
+    times, nbytes = [], []
+    for s in range(args.steps):
+        dt, nb = oracle_step(orc, cfg, seqs, args.warmup + s)
+        times.append(dt)
+        nbytes.append(nb)
+    tot = sum(times)
+    gbs = sum(nbytes) / tot / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.description, "sample_sequences": len(seqs)},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{len(seqs)} of {cfg.batch} sequences per step"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def build_batches(cfg: wl.Config, pk, torch, replicas: int, growth: int, seed: int):
+    """One pool holding `replicas` independent batches of the workload.
+    Returns (pool, [seq ids per batch], [context lengths per batch])."""
+    B = cfg.batch
+    per = cfg.samples_per_prompt
+    lens = [wl.history_lengths(cfg, seed + r, "b") for r in range(replicas)]
+    if per > 1:
+        nb = sum(int(sum(-(-int(n) // cfg.block_size) for n in l)) + B * (growth // cfg.block_size + 3)
+                 for l in lens)
+    else:
+        nb = sum(wl.pool_blocks(cfg, l, growth) for l in lens)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[cfg.q_dtype]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed * 7919 + 17)
+    # draw every history first (the FP8 scale is amax / 448 over all of it)
+    hist = []
+    for r in range(replicas):
+        n_rows = int(sum(lens[r]))
+        k = torch.randn((n_rows, cfg.n_kv_heads, cfg.head_dim), generator=gen, device="cuda",
+                        dtype=torch.float32).to(dt)
+        v = torch.randn((n_rows, cfg.n_kv_heads, cfg.head_dim), generator=gen, device="cuda",
+                        dtype=torch.float32).to(dt)
+        hist.append((k, v))
+    ks = vs = 1.0
+    if cfg.kv_dtype == "fp8":
+        ks = wl.fp8_scale(max(float(k.abs().max()) for k, _ in hist) * 1.05)
+        vs = wl.fp8_scale(max(float(v.abs().max()) for _, v in hist) * 1.05)
+    pool = pk.kv_pool_create(nb, cfg.block_size, cfg.n_kv_heads, cfg.head_dim, cfg.kv_dtype, ks, vs)
+    pk.bt_reset(pool, wl.free_order(nb, seed, cfg.permute))
+    groups, ctx = [], []
+    for r in range(replicas):
+        k, v = hist[r]
+        ids = []
+        slots = []
+        row = 0
+        if per > 1:
+            for p_i, n in enumerate(lens[r]):
+                sid = r * B + p_i * per
+                slots.append(pk.bt_alloc(pool, sid, int(n)))
+                rows = np.arange(row, row + int(n))
+                row += int(n)
+                ids.append(sid)
+                for c in range(1, per):
+                    pk.bt_fork(pool, sid, sid + c)
+                    ids.append(sid + c)
+            c_r = np.repeat(lens[r], per).astype(np.int64)
+        else:
+            for i, n in enumerate(lens[r]):
+                sid = r * B + i
+                slots.append(pk.bt_alloc(pool, sid, int(n)))
+                ids.append(sid)
+            c_r = lens[r].astype(np.int64).copy()
+        s = torch.from_numpy(np.concatenate(slots)).cuda()
+        pk.kv_append(pool, s, k, v)
+        groups.append(np.asarray(sorted(ids), dtype=np.int64))
+        ctx.append(c_r)
+    del hist
+    torch.cuda.synchronize()
+    assert pk.pkv_device_error(pool) == 0
+    return pool, groups, ctx
+
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import pagedattention_decode_02_b200 as pk
+
+    cfg = config_of(args)
+    K, W = args.steps, args.warmup
+    E = args.e2e_steps or max(K // 3, 3)
+    R = max(1, args.replicas)
+    growth = -(-(K + W + E) // R) + 2
+    pool, groups, ctx = build_batches(cfg, pk, torch, R, growth, seed=1000 * rank)
+    B = cfg.batch
+    max_ctx = max(int(c.max()) for c in ctx) + growth
+    max_blocks = -(-max_ctx // cfg.block_size) + 2
+    step = pk.Step(pool, B, max_blocks, cfg.n_q_heads, cfg.q_dtype, args.partition, args.kernel)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[cfg.q_dtype]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4242 + rank)
+    n_sets = 16
+    q = torch.randn((n_sets, B, cfg.n_q_heads, cfg.head_dim), generator=gen, device="cuda").to(dt)
+    kn = torch.randn((n_sets, B, cfg.n_kv_heads, cfg.head_dim), generator=gen, device="cuda").to(dt)
+    vn = torch.randn((n_sets, B, cfg.n_kv_heads, cfg.head_dim), generator=gen, device="cuda").to(dt)
+    out = torch.empty((B, cfg.n_q_heads, cfg.head_dim), dtype=dt, device="cuda")
+    b_tok = cfg.kv_bytes_per_token
+    scale = cfg.scale
+
+    def run_step(k):
+        r = k % R
+        ctx[r] += 1
+        pk.pkv_decode_step(step, groups[r], q[k % n_sets], kn[k % n_sets], vn[k % n_sets], scale, out)
+        return int(ctx[r].sum()), step.last_launches
+
+    for k in range(W):
+        run_step(k)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    pk.pkv_step_profile(step, K)
+    clocks = ClockSampler(local)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    torch.cuda.synchronize()
+    ev0.record()
+    tokens = 0
+    launches = 0
+    step_bytes = []
+    for k in range(W, W + K):
+        t, nl = run_step(k)
+        tokens += t
+        launches += nl
+        step_bytes.append(t * b_tok)
+    ev1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    dec_ms, merge_ms = pk.pkv_step_profile_read(step, K)
+    pk.pkv_step_profile(step, 0)
+
+    # end to end through the public API with host buffers: per round the new
+    # q/k/v arrive from pinned host memory and the output goes back to the host
+    # (a serving loop needs it before the next round)
+    hq = q[0].cpu().pin_memory()
+    hk = kn[0].cpu().pin_memory()
+    hv = vn[0].cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=dt).pin_memory()
+    dq, dk, dv = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e2e_bytes = 0
+    e0.record()
+    for k in range(W + K, W + K + E):
+        r = k % R
+        ctx[r] += 1
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        pk.pkv_decode_step(step, groups[r], dq, dk, dv, scale, out)
+        hout.copy_(out, non_blocking=True)
+        stream.synchronize()
+        e2e_bytes += int(ctx[r].sum()) * b_tok
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
+    d2h = hout.numel() * hout.element_size()
+
+    bits = pk.pkv_device_error(pool)
+    if bits:
+        raise SystemExit(f"device error bits {bits:#x}")
+
+    total_bytes = tokens * b_tok
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+        s = torch.tensor([total_bytes, tokens, e2e_bytes, launches], device="cuda", dtype=torch.float64)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+        total_bytes, tokens_all, e2e_all, launches_all = (float(x) for x in s)
+    else:
+        tokens_all, e2e_all, launches_all = tokens, e2e_bytes, launches
+
+    if rank == 0:
+        value = total_bytes / (elapsed_ms / 1e3) / 1e9
+        peak, peak_kind = peaks()
+        dec_total_ms = float(np.sum(dec_ms))
+        achieved = float(np.sum(step_bytes)) / (dec_total_ms / 1e3) / 1e9
+        traffic = None
+        tr_path = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
+        if os.path.exists(tr_path):
+            try:
+                with open(tr_path) as f:
+                    traffic = json.load(f).get("bytes_per_launch")
+            except Exception:
+                traffic = None
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": W,
+            "ms_per_step": round(elapsed_ms / K, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": cfg.kv_dtype,
+            "data": "synthetic (seeded torch.randn K/V/q; lengths from workloads.py)",
+            "config": {
+                "workload": cfg.description,
+                "batch": cfg.batch, "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads,
+                "head_dim": cfg.head_dim, "block_size": cfg.block_size,
+                "mean_context": round(tokens / K / cfg.batch, 1),
+                "replica_batches_in_pool": R,
+                "pool_blocks": pool.num_blocks,
+                "l2": "no flush: every step reads its whole batch's KV "
+                      f"({np.mean(step_bytes) / 1e6:.0f} MB) from HBM, > 126 MB L2",
+                "parallelism": f"dp{world}",
+            },
+            "attended_tokens_per_s": round(tokens_all / (elapsed_ms / 1e3), 1),
+            "seq_tokens_heads_per_s": round(tokens_all * cfg.n_q_heads / (elapsed_ms / 1e3), 1),
+            "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS / world, 2),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "paged_decode (decode kernel; merge reported separately)",
+                "achieved": round(achieved, 2),
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": int(np.mean(step_bytes)),
+                "decode_ms_mean": round(dec_total_ms / K, 5),
+                "merge_ms_mean": round(float(np.mean(merge_ms)), 5),
+            },
+            "e2e": {
+                "value": round(e2e_all / (e2e_ms / 1e3) / 1e9, 2),
+                "unit": "GB/s",
+                "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h),
+                "steps": E,
+                "ms_per_step": round(e2e_ms / E, 5),
+            },
+            "gpu_launches": int(launches_all),
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    step.close()
+    pool.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,338 @@
+/*
+ * pagedkv.h - C ABI of the paged KV cache and its decode-step kernels (sm_100a).
+ *
+ * What the library does, and where each call comes from
+ * ------------------------------------------------------
+ * Pages cited (by title and section):
+ *   [F55]   "KV 缓存与分页注意力" (world.lapla.si, exhibit F55)
+ *   [TOPIC] "KV 缓存" topic page (aiinfact.com), levels 1-3
+ *   [IPLEX] "读懂PagedAttention：vLLM的KV缓存与GPU显存管理" (iplexlaw.co.kr)
+ *
+ * The KV pool is one region of device memory cut into equal physical blocks
+ * ([F55] §像内存分页): no external fragmentation.  Each sequence owns a block
+ * table: logical block -> physical block id, plus the fill count of the last
+ * block ([F55] §块表).  A block is taken only when the last one is full
+ * ([F55] §块表), shared blocks carry a reference count and are copied on write
+ * ([F55] FAQ 08 共用，写时复制; [IPLEX] §同一提示生成两个回答的假想例子), and a finished
+ * sequence's blocks are returned ([F55] §块表).  Each decode round stores the
+ * new token's key and value and then attends over the whole history, reading
+ * it block by block through the table ([F55] §一次写一个词元, §块表; [TOPIC]
+ * level 3, cached generation).
+ *
+ * Layouts (all row-major, no padding):
+ *   pool K, pool V     [num_blocks][n_kv_heads][block_size][head_dim]  (pool dtype)
+ *   q, out             [B][n_q_heads][head_dim]                        (q dtype)
+ *   new k, new v       [n_tokens][n_kv_heads][head_dim]                (input dtype)
+ *   block_tables       [B][max_blocks] int32, unused entries -1
+ *   context_lens       [B] int32, tokens per sequence *including* the new one
+ *   slot_mapping       [n_tokens] int32, slot = physical_block * block_size + offset
+ * Query head h reads KV head floor(h / (n_q_heads / n_kv_heads)).
+ *
+ * Conventions
+ *   - Nothing throws or aborts across this ABI; every call returns a status.
+ *   - Host calls (kv_pool_*, bt_*) are all-or-nothing: on any error the state
+ *     is exactly as before the call.
+ *   - Device calls are asynchronous on the given stream (a cudaStream_t passed
+ *     as void*, NULL = legacy default stream).  Argument errors visible on the
+ *     host return PKV_ERR_INVALID_ARG before anything is launched; errors only
+ *     visible on the device (a context length or block id out of range, a
+ *     bounded wait that gave up) set bits in the pool's device error word,
+ *     which pkv_device_error() reads and clears.  Kernels never trap.
+ *   - Ownership: the caller owns every pointer it passes (q, out, k, v,
+ *     tables, lengths, slot mapping, workspace).  The pool owns its host
+ *     bookkeeping, its device error word and - when it allocated them - its
+ *     K/V buffers.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,  /* bad argument; nothing done */
+    PKV_ERR_NO_BLOCKS = 2,    /* not enough free blocks; nothing done */
+    PKV_ERR_UNKNOWN_SEQ = 3,  /* sequence id not in the pool */
+    PKV_ERR_SEQ_EXISTS = 4,   /* sequence id already in the pool */
+    PKV_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+    PKV_ERR_DEVICE = 6        /* the device error word was set (see pkv_device_error) */
+} pkv_status;
+
+typedef enum {
+    PKV_F32 = 0,
+    PKV_F16 = 1,
+    PKV_BF16 = 2,
+    PKV_FP8_E4M3 = 3          /* OCP FP8 E4M3, per-tensor scale ([F55] §后来的做法) */
+} pkv_dtype;
+
+/* bits of the device error word */
+#define PKV_DEVERR_CONTEXT_LEN 0x1u  /* context_len < 1 or > max_blocks * block_size */
+#define PKV_DEVERR_BLOCK_ID    0x2u  /* block id outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT        0x4u  /* slot outside [0, num_blocks * block_size) */
+#define PKV_DEVERR_TIMEOUT     0x8u  /* a bounded wait on a copy gave up */
+
+/* kv_pool_create flags */
+#define PKV_POOL_HOST_ONLY 0x1u      /* bookkeeping only: no device memory, device calls refused */
+
+typedef struct pkv_pool pkv_pool;
+
+typedef struct {
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t free_blocks;
+    int32_t used_blocks;      /* blocks with refcount > 0 */
+    int32_t num_seqs;
+    int32_t pad_;
+    int64_t stored_slots;     /* filled slots over used blocks (a shared block counts once) */
+    int64_t logical_tokens;   /* sum of sequence lengths (a shared token counts per sequence) */
+    int64_t table_slots;      /* sum over sequences of |table| * block_size */
+    int64_t cow_count;        /* copy-on-write events since the last bt_reset */
+} pkv_stats;
+
+typedef struct {
+    int32_t num_blocks, block_size, n_kv_heads, head_dim;
+    int32_t dtype;            /* pkv_dtype */
+    int32_t host_only;
+    float k_scale, v_scale;
+    void* k_buf;              /* device pointers (NULL for host-only pools) */
+    void* v_buf;
+    size_t bytes_per_buffer;  /* num_blocks * n_kv_heads * block_size * head_dim * elem bytes */
+    uint32_t* error_word;     /* device pointer */
+} pkv_pool_info;
+
+/* ---------------------------------------------------------------------------
+ * Pool
+ * ------------------------------------------------------------------------- */
+
+/* kv_pool_create - the KV pool of equal physical blocks ([F55] §像内存分页).
+ *   num_blocks >= 1, block_size >= 1, n_kv_heads >= 1, head_dim in {32, 64, 128}.
+ *   dtype: storage type.  k_scale, v_scale: FP8 dequantisation scales (stored
+ *   value = code * scale); must be finite and > 0 for PKV_FP8_E4M3, ignored
+ *   otherwise.
+ *   k_buf, v_buf: both NULL -> the pool allocates both buffers itself (and
+ *   frees them in kv_pool_destroy); both non-NULL -> caller-owned device
+ *   buffers of at least *bytes_needed_out bytes each, 16-byte aligned.
+ *   flags: PKV_POOL_HOST_ONLY for a bookkeeping-only pool (k_buf/v_buf ignored).
+ *   bytes_needed_out (may be NULL): receives the size of one buffer.
+ *   out: receives the pool; if NULL, only *bytes_needed_out is computed.
+ *   The free queue starts in identity order (see bt_reset).
+ *   Errors: INVALID_ARG, CUDA (allocation failed; nothing leaked). */
+pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim,
+                          pkv_dtype dtype, float k_scale, float v_scale,
+                          void* k_buf, void* v_buf, unsigned flags,
+                          size_t* bytes_needed_out, pkv_pool** out);
+
+/* kv_pool_destroy - frees the bookkeeping, the error word and self-allocated
+ *   buffers.  NULL is accepted.  The caller must make sure no kernel using the
+ *   pool is still running. */
+void kv_pool_destroy(pkv_pool* pool);
+
+/* kv_pool_get_info - fills *info (device pointers, sizes, scales). */
+pkv_status kv_pool_get_info(const pkv_pool* pool, pkv_pool_info* info);
+
+/* ---------------------------------------------------------------------------
+ * Block tables (host; [F55] §块表, FAQ 08; [IPLEX] §分离逻辑顺序与实际存储位置,
+ * §同一提示生成两个回答的假想例子).  Free-queue policy: FIFO; a block is taken from
+ * the front and returned to the back when its refcount reaches zero.
+ * ------------------------------------------------------------------------- */
+
+/* bt_reset - drops every sequence and refills the free queue in the given
+ *   order (free_order: host array of num_blocks distinct ids; NULL = identity).
+ *   Resets cow_count.  Errors: INVALID_ARG (not a permutation). */
+pkv_status bt_reset(pkv_pool* pool, const int32_t* free_order);
+
+/* bt_alloc - admits a new sequence with n_tokens >= 0 prompt tokens: takes
+ *   ceil(n_tokens / block_size) blocks and writes the n_tokens slots, in token
+ *   order, to slot_mapping_out (host, n_tokens entries; may be NULL when
+ *   n_tokens == 0).  Errors: INVALID_ARG, SEQ_EXISTS, NO_BLOCKS. */
+pkv_status bt_alloc(pkv_pool* pool, int64_t seq_id, int n_tokens, int32_t* slot_mapping_out);
+
+/* bt_append - reserves the slot of one new token of seq_id: the next slot of
+ *   the last block; a fresh block if the last is full (or there is none); if
+ *   the last block is partially filled and shared (refcount > 1), a fresh
+ *   block receives a copy first: *cow_src_out / *cow_dst_out get the pair
+ *   (else -1), the old block's count drops by one, and the caller must run
+ *   block_copy(src -> dst) before kv_append writes the slot.
+ *   Errors: UNKNOWN_SEQ, NO_BLOCKS. */
+pkv_status bt_append(pkv_pool* pool, int64_t seq_id, int32_t* slot_out,
+                     int32_t* cow_src_out, int32_t* cow_dst_out);
+
+/* bt_append_batch - bt_append for seq_ids[0..n) in that order, all-or-nothing.
+ *   slots_out: host [n]; cow_src_out, cow_dst_out: host arrays of capacity n,
+ *   *n_cow_out receives the number of copy pairs written (in the order made).
+ *   Errors: INVALID_ARG, UNKNOWN_SEQ, NO_BLOCKS (state unchanged). */
+pkv_status bt_append_batch(pkv_pool* pool, const int64_t* seq_ids, int n, int32_t* slots_out,
+                           int32_t* cow_src_out, int32_t* cow_dst_out, int* n_cow_out);
+
+/* bt_fork - child_id gets parent_id's table; every block's refcount + 1
+ *   ([IPLEX]: two samples of one prompt point at the same input blocks).
+ *   Errors: UNKNOWN_SEQ (parent), SEQ_EXISTS (child). */
+pkv_status bt_fork(pkv_pool* pool, int64_t parent_id, int64_t child_id);
+
+/* bt_free - a finished sequence releases its blocks in logical order; blocks
+ *   whose count reaches zero return to the free queue.  Errors: UNKNOWN_SEQ. */
+pkv_status bt_free(pkv_pool* pool, int64_t seq_id);
+
+/* bt_export - block tables and lengths of seq_ids[0..n) for the kernels:
+ *   block_tables_out host [n][max_blocks] (entries past a table's end = -1),
+ *   context_lens_out host [n], fill_of_last_out host [n] (may be NULL; 0 for a
+ *   sequence without blocks).  Errors: INVALID_ARG (a table longer than
+ *   max_blocks), UNKNOWN_SEQ. */
+pkv_status bt_export(pkv_pool* pool, const int64_t* seq_ids, int n, int max_blocks,
+                     int32_t* block_tables_out, int32_t* context_lens_out,
+                     int32_t* fill_of_last_out);
+
+/* bt_num_blocks - number of blocks in seq_id's table. */
+pkv_status bt_num_blocks(const pkv_pool* pool, int64_t seq_id, int32_t* n_out);
+
+/* bt_refcount - refcount of one physical block. */
+pkv_status bt_refcount(const pkv_pool* pool, int32_t block_id, int32_t* refcount_out);
+
+/* bt_free_queue - copies the free queue front-to-back into out (capacity cap);
+ *   *n_out receives its length.  INVALID_ARG if cap is too small. */
+pkv_status bt_free_queue(const pkv_pool* pool, int32_t* out, int cap, int* n_out);
+
+/* bt_stats - pool counters; utilisation = logical_tokens / table_slots
+ *   ([F55] §块表: blocks actually storing tokens). */
+pkv_status bt_stats(const pkv_pool* pool, pkv_stats* out);
+
+/* ---------------------------------------------------------------------------
+ * Device calls
+ * ------------------------------------------------------------------------- */
+
+/* kv_append - stores new keys and values into their slots ([F55] §一次写一个词元;
+ *   [IPLEX] §分离逻辑顺序与实际存储位置: later tokens go into the free slots of the
+ *   last block).  pool K[slot / bs][h][slot % bs][:] = d_k[t][h][:], same for V.
+ *   d_slot_mapping: device int32 [n_tokens]; slot < 0 skips the token.
+ *   d_k, d_v: device [n_tokens][n_kv_heads][head_dim] in in_dtype.
+ *   in_dtype must equal the pool dtype, except for FP8 pools, which take
+ *   F32/F16/BF16 rows and store e4m3(round-to-nearest-even, saturating) of
+ *   (x / scale) with the quotient formed in float32.
+ *   A slot >= num_blocks * block_size sets PKV_DEVERR_SLOT and is skipped.
+ *   n_tokens == 0 is a no-op.  Errors: INVALID_ARG, CUDA. */
+pkv_status kv_append(pkv_pool* pool, const int32_t* d_slot_mapping, int n_tokens,
+                     const void* d_k, const void* d_v, pkv_dtype in_dtype, void* stream);
+
+/* block_copy - copy-on-write: copies whole physical blocks (all KV heads, K
+ *   and V) d_src[i] -> d_dst[i] ([F55] FAQ 08: copy the block, then write the
+ *   copy).  d_src, d_dst: device int32 [n_pairs]; destinations must be
+ *   distinct and no destination may be a source.  Ids out of range set
+ *   PKV_DEVERR_BLOCK_ID and the pair is skipped.  Errors: INVALID_ARG, CUDA. */
+pkv_status block_copy(pkv_pool* pool, const int32_t* d_src, const int32_t* d_dst, int n_pairs,
+                      void* stream);
+
+/* paged_decode_attention - one decode step's attention ([F55] §块表: the kernel
+ *   fetches K and V block by block following the table; blocks need not be
+ *   adjacent).  For sequence i and query head h, with g = floor(h / G):
+ *     out[i][h] = sum_j softmax_j(scale * <q[i][h], K_i[g][j]>) V_i[g][j],  j < c_i
+ *   where K_i[g][j] lives in block d_block_tables[i][j / bs], slot j % bs.
+ *   d_q: device [B][n_q_heads][head_dim] in q_dtype; q_dtype = pool dtype for
+ *   F32/F16/BF16 pools, F16 or BF16 for FP8 pools.  d_out: same shape/dtype.
+ *   d_block_tables: device int32 [B][max_blocks]; d_context_lens: device [B].
+ *   n_q_heads must be a multiple of n_kv_heads.
+ *   Long contexts are split into partitions whose partial softmax states are
+ *   merged by log-sum-exp in a second kernel; that needs d_workspace (device,
+ *   ws_bytes >= paged_decode_workspace_bytes(...), 16-byte aligned, caller
+ *   owned, contents scratch).  Without enough workspace the call returns
+ *   INVALID_ARG.  A context length outside [1, max_blocks * bs] sets
+ *   PKV_DEVERR_CONTEXT_LEN and that sequence's output is zero; a table entry
+ *   outside [0, num_blocks) sets PKV_DEVERR_BLOCK_ID and the output of the
+ *   affected partition is zero.  B == 0 is a no-op.  Errors: INVALID_ARG, CUDA. */
+pkv_status paged_decode_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
+                                  const int32_t* d_block_tables, int max_blocks,
+                                  const int32_t* d_context_lens, int B, int n_q_heads,
+                                  float scale, void* d_out, void* d_workspace, size_t ws_bytes,
+                                  void* stream);
+
+/* paged_decode_workspace_bytes - workspace paged_decode_attention needs for
+ *   this batch shape (max_blocks as passed to it). */
+size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, int max_blocks);
+
+/* Kernel selection for paged_decode_attention_ex. */
+#define PKV_KERNEL_AUTO 0
+#define PKV_KERNEL_SIMT 1          /* CUDA-core dot products (any head grouping, any dtype) */
+#define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads (F16/BF16, G > 1) */
+
+/* paged_decode_attention_ex - paged_decode_attention with explicit choices:
+ *   partition_tokens: 0 = automatic, > 0 = tokens per partition (a multiple
+ *   of 16), -1 = never split; kernel: PKV_KERNEL_*.  The workspace needed for
+ *   the same choices is paged_decode_workspace_bytes_ex(). */
+pkv_status paged_decode_attention_ex(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
+                                     const int32_t* d_block_tables, int max_blocks,
+                                     const int32_t* d_context_lens, int B, int n_q_heads,
+                                     float scale, void* d_out, void* d_workspace, size_t ws_bytes,
+                                     int partition_tokens, int kernel, void* stream);
+size_t paged_decode_workspace_bytes_ex(const pkv_pool* pool, int B, int n_q_heads, int max_blocks,
+                                       int partition_tokens);
+
+/* ---------------------------------------------------------------------------
+ * Decode-step runtime: one call per generation round for a batch of running
+ * sequences ([F55] §一次写一个词元: each round every running sequence stores its
+ * new token's key and value and attends over its history).
+ * ------------------------------------------------------------------------- */
+typedef struct pkv_step pkv_step;
+
+/* pkv_step_create - per-batch runtime state for a pool: pinned host staging
+ *   and device buffers for up to max_batch sequences of up to max_blocks
+ *   blocks each, and the attention workspace for that shape.  All memory is
+ *   allocated here, none in pkv_decode_step.  q_dtype: dtype of q, of the new
+ *   K/V rows and of the output.  partition_tokens / kernel as in
+ *   paged_decode_attention_ex.  Errors: INVALID_ARG, CUDA. */
+pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_q_heads,
+                           pkv_dtype q_dtype, int partition_tokens, int kernel, pkv_step** out);
+
+/* pkv_step_destroy - synchronises on the runtime's outstanding copies and
+ *   frees its buffers.  NULL is accepted. */
+void pkv_step_destroy(pkv_step* step);
+
+/* pkv_decode_step - one decode round for seq_ids[0..B), B <= max_batch:
+ *   1. host: bt_append_batch (slots, copy-on-write pairs; all-or-nothing -
+ *      on error nothing is launched and the tables are unchanged);
+ *   2. host: the batch's block tables and context lengths into pinned staging,
+ *      one asynchronous host-to-device copy on `stream`;
+ *   3. device: block_copy of the copy-on-write pairs, then kv_append of the B
+ *      new rows, then paged decode attention into d_out.
+ *   d_q: device [B][n_q_heads][head_dim]; d_k_new, d_v_new: device
+ *   [B][n_kv_heads][head_dim]; d_out: device [B][n_q_heads][head_dim]; all in
+ *   q_dtype.  Returns INVALID_ARG if a table would exceed max_blocks (nothing
+ *   changed).  The host returns once the work is queued; staging slots are
+ *   reused only after their copies completed. */
+pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const void* d_q,
+                           const void* d_k_new, const void* d_v_new, float scale, void* d_out,
+                           void* stream);
+
+/* pkv_step_last_launches - number of kernels the last pkv_decode_step call
+ *   launched (copy-on-write copy, append, decode, merge). */
+int pkv_step_last_launches(const pkv_step* step);
+
+/* pkv_step_profile - n > 0: later pkv_decode_step calls record CUDA events on
+ *   their stream right before the decode kernel, between it and the partition
+ *   merge, and after the merge, into a ring of n entries; n == 0 turns this
+ *   off.  Errors: INVALID_ARG, CUDA. */
+pkv_status pkv_step_profile(pkv_step* step, int n);
+
+/* pkv_step_profile_read - milliseconds of the decode kernel and of the merge
+ *   for the most recent min(calls, n) recorded calls, oldest first, into
+ *   decode_ms[] and merge_ms[] (capacity cap); *n_out receives the count.
+ *   Waits for those events.  Errors: INVALID_ARG (cap too small), CUDA. */
+pkv_status pkv_step_profile_read(pkv_step* step, float* decode_ms, float* merge_ms, int cap,
+                                 int* n_out);
+
+/* pkv_device_error - synchronises the stream, returns the device error word's
+ *   bits in *bits_out (may be NULL) and clears it.  Returns PKV_ERR_DEVICE if
+ *   any bit was set, PKV_OK otherwise. */
+pkv_status pkv_device_error(pkv_pool* pool, void* stream, uint32_t* bits_out);
+
+/* pkv_status_str - a static, human-readable name of a status. */
+const char* pkv_status_str(pkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -56,15 +56,24 @@ def decode_attention(q: np.ndarray, k_hist: np.ndarray, v_hist: np.ndarray, scal
     the new token included).  Returns out [H_q][d] in float64.
     """
     q = np.asarray(q, dtype=np.float64)
+    k_hist = np.asarray(k_hist, dtype=np.float64)
+    v_hist = np.asarray(v_hist, dtype=np.float64)
     h_q = q.shape[0]
     h_kv = k_hist.shape[1]
     if h_q % h_kv:
         raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    if k_hist.shape[0] == 0:
+        raise ValueError("attention over an empty history is undefined")
     group = h_q // h_kv
     out = np.empty_like(q)
-    for h in range(h_q):
-        g = h // group
-        out[h] = attend_head(q[h], k_hist[:, g, :], v_hist[:, g, :], scale)
+    for g in range(h_kv):
+        # the query heads of KV head g, all at once: S = scale * Q K^T [G][c]
+        qg = q[g * group:(g + 1) * group]
+        s = scale * (qg @ k_hist[:, g, :].T)
+        s = s - s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        p = e / e.sum(axis=1, keepdims=True)
+        out[g * group:(g + 1) * group] = p @ v_hist[:, g, :]
     return out
 
 

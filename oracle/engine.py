@@ -22,7 +22,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 from .allocator import BlockManager
-from .attention import decode_attention
+from .attention import attend_head, decode_attention
 from .numerics import e4m3_decode, e4m3_quantize_for_pool, to_f64
 
 _STORE_NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16, "fp8": np.uint8}
@@ -108,12 +108,9 @@ class DecodeOracle:
                 outs.append(decode_attention(qd[i], kd, vd, scale))
             else:
                 group = qd.shape[1] // self.n_kv_heads
-                sel = np.stack([qd[i][h] for h in heads])
-                o = np.empty_like(sel)
-                for j, h in enumerate(heads):
-                    g = h // group
-                    o[j] = decode_attention(sel[j:j + 1], kd[:, g:g + 1, :], vd[:, g:g + 1, :], scale)[0]
-                outs.append(o)
+                outs.append(np.stack([
+                    attend_head(qd[i][h], kd[:, h // group, :], vd[:, h // group, :], scale)
+                    for h in heads]))
         return np.stack(outs)
 
     def step(self, seqs: Sequence[int], q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,

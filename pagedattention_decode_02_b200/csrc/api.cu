@@ -1,0 +1,593 @@
+// The C ABI declared in include/pagedkv.h: pool lifetime, block-table calls
+// (forwarded to the host BlockManager), argument validation and kernel
+// dispatch for the device calls.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "block_manager.h"
+#include "decode_launch.h"
+#include "pagedkv.h"
+#include "pool.h"
+
+using pkv::BlockManager;
+
+namespace {
+
+int elem_bytes(int dt) {
+    switch (dt) {
+        case PKV_F32: return 4;
+        case PKV_F16: return 2;
+        case PKV_BF16: return 2;
+        case PKV_FP8_E4M3: return 1;
+        default: return 0;
+    }
+}
+
+bool valid_dtype(int dt) { return dt >= PKV_F32 && dt <= PKV_FP8_E4M3; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool same_device(const pkv_pool* pool) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    return dev == pool->device;
+}
+
+// Tokens per partition when the caller leaves it to the library.  Contexts up
+// to kNoSplitTokens run as one partition per (sequence, head group); longer
+// ones are cut into kAutoPartition-token partitions so that long and short
+// sequences give CTAs of similar size and the grid fills all SMs.
+constexpr int kNoSplitTokens = 512;
+constexpr int kAutoPartition = 512;
+
+int resolve_partition(const pkv_pool* pool, int max_blocks, int requested) {
+    const long long max_ctx = (long long)max_blocks * pool->block_size;
+    const int whole = (int)(((max_ctx + 15) / 16) * 16);
+    if (requested < 0) return whole < 16 ? 16 : whole;
+    if (requested > 0) return requested;
+    if (max_ctx <= kNoSplitTokens) return whole < 16 ? 16 : whole;
+    return kAutoPartition;
+}
+
+int parts_for(const pkv_pool* pool, int max_blocks, int part_tokens) {
+    const long long max_ctx = (long long)max_blocks * pool->block_size;
+    return (int)((max_ctx + part_tokens - 1) / part_tokens);
+}
+
+size_t workspace_for(const pkv_pool* pool, int B, int n_q_heads, int max_parts) {
+    if (max_parts <= 1) return 0;
+    const size_t rows = (size_t)B * n_q_heads * max_parts;
+    const size_t ml = ((rows * 2 * sizeof(float)) + 255) & ~(size_t)255;
+    return ml + rows * pool->head_dim * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_str(pkv_status s) {
+    switch (s) {
+        case PKV_OK: return "OK";
+        case PKV_ERR_INVALID_ARG: return "INVALID_ARG";
+        case PKV_ERR_NO_BLOCKS: return "NO_BLOCKS";
+        case PKV_ERR_UNKNOWN_SEQ: return "UNKNOWN_SEQ";
+        case PKV_ERR_SEQ_EXISTS: return "SEQ_EXISTS";
+        case PKV_ERR_CUDA: return "CUDA";
+        case PKV_ERR_DEVICE: return "DEVICE";
+        default: return "UNKNOWN_STATUS";
+    }
+}
+
+pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int head_dim,
+                          pkv_dtype dtype, float k_scale, float v_scale, void* k_buf, void* v_buf,
+                          unsigned flags, size_t* bytes_needed_out, pkv_pool** out) {
+    if (num_blocks < 1 || block_size < 1 || n_kv_heads < 1) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128) return PKV_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype)) return PKV_ERR_INVALID_ARG;
+    if ((flags & ~PKV_POOL_HOST_ONLY) != 0) return PKV_ERR_INVALID_ARG;
+    if (dtype == PKV_FP8_E4M3 &&
+        !(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+        return PKV_ERR_INVALID_ARG;
+    // slots are int32: num_blocks * block_size must fit
+    if ((long long)num_blocks * block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)num_blocks * n_kv_heads * block_size * head_dim * elem_bytes(dtype);
+    if (bytes_needed_out) *bytes_needed_out = bytes;
+    if (!out) return PKV_OK;
+    const bool host_only = flags & PKV_POOL_HOST_ONLY;
+    if (!host_only && ((k_buf == nullptr) != (v_buf == nullptr))) return PKV_ERR_INVALID_ARG;
+    if (!host_only && k_buf && (!aligned16(k_buf) || !aligned16(v_buf))) return PKV_ERR_INVALID_ARG;
+
+    pkv_pool* p = new (std::nothrow) pkv_pool(num_blocks, block_size);
+    if (!p) return PKV_ERR_INVALID_ARG;
+    p->num_blocks = num_blocks;
+    p->block_size = block_size;
+    p->n_kv_heads = n_kv_heads;
+    p->head_dim = head_dim;
+    p->dtype = dtype;
+    p->k_scale = dtype == PKV_FP8_E4M3 ? k_scale : 1.f;
+    p->v_scale = dtype == PKV_FP8_E4M3 ? v_scale : 1.f;
+    p->host_only = host_only;
+    p->bytes = bytes;
+    if (!host_only) {
+        if (cudaGetDevice(&p->device) != cudaSuccess) {
+            delete p;
+            return PKV_ERR_CUDA;
+        }
+        if (k_buf) {
+            p->k = static_cast<uint8_t*>(k_buf);
+            p->v = static_cast<uint8_t*>(v_buf);
+            p->owns_buffers = false;
+        } else {
+            if (cudaMalloc(&p->k, bytes) != cudaSuccess) {
+                delete p;
+                return PKV_ERR_CUDA;
+            }
+            if (cudaMalloc(&p->v, bytes) != cudaSuccess) {
+                cudaFree(p->k);
+                delete p;
+                return PKV_ERR_CUDA;
+            }
+            p->owns_buffers = true;
+        }
+        if (cudaMalloc(&p->d_err, sizeof(uint32_t)) != cudaSuccess ||
+            cudaMemset(p->d_err, 0, sizeof(uint32_t)) != cudaSuccess) {
+            if (p->owns_buffers) {
+                cudaFree(p->k);
+                cudaFree(p->v);
+            }
+            if (p->d_err) cudaFree(p->d_err);
+            delete p;
+            return PKV_ERR_CUDA;
+        }
+        pkv::pool_init_device_extras(p);
+    }
+    *out = p;
+    return PKV_OK;
+}
+
+void kv_pool_destroy(pkv_pool* p) {
+    if (!p) return;
+    if (!p->host_only) {
+        if (p->owns_buffers) {
+            cudaFree(p->k);
+            cudaFree(p->v);
+        }
+        cudaFree(p->d_err);
+    }
+    delete p;
+}
+
+pkv_status kv_pool_get_info(const pkv_pool* p, pkv_pool_info* info) {
+    if (!p || !info) return PKV_ERR_INVALID_ARG;
+    info->num_blocks = p->num_blocks;
+    info->block_size = p->block_size;
+    info->n_kv_heads = p->n_kv_heads;
+    info->head_dim = p->head_dim;
+    info->dtype = p->dtype;
+    info->host_only = p->host_only;
+    info->k_scale = p->k_scale;
+    info->v_scale = p->v_scale;
+    info->k_buf = p->k;
+    info->v_buf = p->v;
+    info->bytes_per_buffer = p->bytes;
+    info->error_word = p->d_err;
+    return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// block tables
+// ---------------------------------------------------------------------------
+pkv_status bt_reset(pkv_pool* p, const int32_t* order) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.reset(order);
+}
+pkv_status bt_alloc(pkv_pool* p, int64_t seq, int n_tokens, int32_t* slots) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.alloc(seq, n_tokens, slots);
+}
+pkv_status bt_append(pkv_pool* p, int64_t seq, int32_t* slot, int32_t* src, int32_t* dst) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.append(seq, slot, src, dst);
+}
+pkv_status bt_append_batch(pkv_pool* p, const int64_t* seqs, int n, int32_t* slots, int32_t* src,
+                           int32_t* dst, int* n_cow) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.append_batch(seqs, n, slots, src, dst, n_cow);
+}
+pkv_status bt_fork(pkv_pool* p, int64_t parent, int64_t child) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.fork(parent, child);
+}
+pkv_status bt_free(pkv_pool* p, int64_t seq) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.release(seq);
+}
+pkv_status bt_export(pkv_pool* p, const int64_t* seqs, int n, int max_blocks, int32_t* tables,
+                     int32_t* lens, int32_t* fills) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.export_tables(seqs, n, max_blocks, tables, lens, fills);
+}
+pkv_status bt_num_blocks(const pkv_pool* p, int64_t seq, int32_t* n) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.num_blocks_of(seq, n);
+}
+pkv_status bt_refcount(const pkv_pool* p, int32_t block, int32_t* r) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.refcount_of(block, r);
+}
+pkv_status bt_free_queue(const pkv_pool* p, int32_t* out, int cap, int* n) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.free_queue(out, cap, n);
+}
+pkv_status bt_stats(const pkv_pool* p, pkv_stats* out) {
+    if (!p || !out) return PKV_ERR_INVALID_ARG;
+    p->bm.stats(out);
+    return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// device calls
+// ---------------------------------------------------------------------------
+pkv_status kv_append(pkv_pool* p, const int32_t* slots, int n_tokens, const void* k, const void* v,
+                     pkv_dtype in_dtype, void* stream) {
+    if (!p || p->host_only || n_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype)) return PKV_ERR_INVALID_ARG;
+    if (p->dtype == PKV_FP8_E4M3 ? in_dtype == PKV_FP8_E4M3 : in_dtype != p->dtype)
+        return PKV_ERR_INVALID_ARG;
+    if (n_tokens == 0) return PKV_OK;
+    if (!slots || !k || !v || !aligned16(k) || !aligned16(v)) return PKV_ERR_INVALID_ARG;
+    if (!same_device(p)) return PKV_ERR_INVALID_ARG;
+    cudaError_t e = pkv::launch_kv_append(p->k, p->v, slots, n_tokens, k, v, in_dtype, p->dtype,
+                                          p->n_kv_heads, p->head_dim, p->block_size, p->num_blocks,
+                                          p->k_scale, p->v_scale, p->d_err,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status block_copy(pkv_pool* p, const int32_t* src, const int32_t* dst, int n_pairs,
+                      void* stream) {
+    if (!p || p->host_only || n_pairs < 0) return PKV_ERR_INVALID_ARG;
+    if (n_pairs == 0) return PKV_OK;
+    if (!src || !dst) return PKV_ERR_INVALID_ARG;
+    if (!same_device(p)) return PKV_ERR_INVALID_ARG;
+    const long long block_bytes = (long long)p->n_kv_heads * p->block_size * p->head_dim *
+                                  elem_bytes(p->dtype);
+    cudaError_t e = pkv::launch_block_copy(p->k, p->v, src, dst, n_pairs, block_bytes,
+                                           p->num_blocks, p->d_err,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+size_t paged_decode_workspace_bytes_ex(const pkv_pool* p, int B, int n_q_heads, int max_blocks,
+                                       int partition_tokens) {
+    if (!p || B <= 0 || n_q_heads <= 0 || max_blocks <= 0) return 0;
+    const int P = resolve_partition(p, max_blocks, partition_tokens);
+    if (P <= 0 || P % 16) return 0;
+    return workspace_for(p, B, n_q_heads, parts_for(p, max_blocks, P));
+}
+
+size_t paged_decode_workspace_bytes(const pkv_pool* p, int B, int n_q_heads, int max_blocks) {
+    return paged_decode_workspace_bytes_ex(p, B, n_q_heads, max_blocks, 0);
+}
+
+}  // extern "C"
+
+namespace {
+// paged_decode_attention_ex with optional events recorded on the stream right
+// before the decode kernel (ev_begin), between it and the merge (ev_mid) and
+// after the last launch (ev_end).
+pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                 const int32_t* tables, int max_blocks, const int32_t* lens, int B,
+                                 int n_q_heads, float scale, void* out, void* ws, size_t ws_bytes,
+                                 int partition_tokens, int kernel, void* stream,
+                                 cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end) {
+    if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
+    if (B == 0) return PKV_OK;
+    if (!q || !out || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
+    if (n_q_heads < p->n_kv_heads || n_q_heads % p->n_kv_heads) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (p->dtype == PKV_FP8_E4M3) {
+        if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+    } else if (q_dtype != p->dtype) {
+        return PKV_ERR_INVALID_ARG;
+    }
+    if (partition_tokens != 0 && partition_tokens != -1 &&
+        (partition_tokens < 16 || partition_tokens % 16))
+        return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_TENSOR) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_blocks * p->block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+    if (!same_device(p)) return PKV_ERR_INVALID_ARG;
+
+    const int G = n_q_heads / p->n_kv_heads;
+    const int P = resolve_partition(p, max_blocks, partition_tokens);
+    const int max_parts = parts_for(p, max_blocks, P);
+    const size_t need = workspace_for(p, B, n_q_heads, max_parts);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_parts > 0x7fffffffLL || B > 65535) return PKV_ERR_INVALID_ARG;
+
+    const bool tc_ok = pkv::tensor_path_supported(p->dtype, q_dtype, p->head_dim, G, p->block_size);
+    int use = kernel;
+    if (use == PKV_KERNEL_AUTO) use = tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT;
+    if (use == PKV_KERNEL_TENSOR && !tc_ok) return PKV_ERR_INVALID_ARG;
+
+    pkv::DecodeParams dp{};
+    dp.q = q;
+    dp.out = out;
+    dp.k_pool = p->k;
+    dp.v_pool = p->v;
+    dp.tables = tables;
+    dp.lens = lens;
+    dp.err = p->d_err;
+    dp.B = B;
+    dp.H_q = n_q_heads;
+    dp.H_kv = p->n_kv_heads;
+    dp.G = G;
+    dp.max_blocks = max_blocks;
+    dp.block_size = p->block_size;
+    dp.num_blocks = p->num_blocks;
+    dp.part_tokens = P;
+    dp.max_parts = max_parts;
+    const size_t rows = (size_t)B * n_q_heads * max_parts;
+    dp.ws_ml = need ? static_cast<float*>(ws) : nullptr;
+    dp.ws_acc = need ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                                ((rows * 2 * sizeof(float) + 255) & ~(size_t)255))
+                     : nullptr;
+    const float log2e = 1.4426950408889634f;
+    dp.q_scale = scale * log2e * p->k_scale;
+    dp.v_scale = p->v_scale;
+    dp.head_stride = (long long)p->block_size * p->head_dim * elem_bytes(p->dtype);
+    dp.block_stride = dp.head_stride * p->n_kv_heads;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = ev_begin ? cudaEventRecord(ev_begin, st) : cudaSuccess;
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+    if (use == PKV_KERNEL_TENSOR) {
+        e = pkv::launch_decode_tensor(dp, p->tmap_k, p->tmap_v, p->dtype, p->head_dim, st, ev_mid);
+    } else {
+        e = pkv::launch_decode_simt(dp, p->dtype, q_dtype, p->head_dim, pkv::simt_heads_per_cta(G),
+                                    st, ev_mid);
+    }
+    if (e == cudaSuccess && ev_end) e = cudaEventRecord(ev_end, st);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status paged_decode_attention_ex(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                     const int32_t* tables, int max_blocks, const int32_t* lens,
+                                     int B, int n_q_heads, float scale, void* out, void* ws,
+                                     size_t ws_bytes, int partition_tokens, int kernel,
+                                     void* stream) {
+    return decode_attention_impl(p, q, q_dtype, tables, max_blocks, lens, B, n_q_heads, scale, out,
+                                 ws, ws_bytes, partition_tokens, kernel, stream, nullptr, nullptr,
+                                 nullptr);
+}
+
+pkv_status paged_decode_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                  const int32_t* tables, int max_blocks, const int32_t* lens, int B,
+                                  int n_q_heads, float scale, void* out, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    return paged_decode_attention_ex(p, q, q_dtype, tables, max_blocks, lens, B, n_q_heads, scale,
+                                     out, ws, ws_bytes, 0, PKV_KERNEL_AUTO, stream);
+}
+
+pkv_status pkv_device_error(pkv_pool* p, void* stream, uint32_t* bits_out) {
+    if (!p || p->host_only) return PKV_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t bits = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemcpy(&bits, p->d_err, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (bits && cudaMemset(p->d_err, 0, sizeof(uint32_t)) != cudaSuccess) return PKV_ERR_CUDA;
+    if (bits_out) *bits_out = bits;
+    return bits ? PKV_ERR_DEVICE : PKV_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// decode-step runtime
+// ---------------------------------------------------------------------------
+struct pkv_step {
+    static constexpr int kRing = 3;   // pinned staging slots in flight
+    pkv_pool* pool = nullptr;
+    int max_batch = 0, max_blocks = 0, n_q_heads = 0;
+    pkv_dtype q_dtype = PKV_F16;
+    int partition_tokens = 0, kernel = PKV_KERNEL_AUTO;
+    size_t stage_ints = 0;            // slots | cow src | cow dst | lens | tables
+    int32_t* h_stage[kRing] = {};
+    cudaEvent_t ev[kRing] = {};
+    bool pending[kRing] = {};
+    int ring = 0;
+    int32_t* d_stage = nullptr;
+    void* d_ws = nullptr;
+    size_t ws_bytes = 0;
+    int max_parts = 1;
+    int last_launches = 0;
+    // profiling: event triples (before decode, between decode and merge,
+    // after merge) in a ring of prof_n entries
+    int prof_n = 0;
+    long long prof_count = 0;
+    cudaEvent_t* prof_ev = nullptr;
+};
+
+namespace {
+void prof_free(pkv_step* s) {
+    if (s->prof_ev) {
+        for (int i = 0; i < 3 * s->prof_n; ++i)
+            if (s->prof_ev[i]) cudaEventDestroy(s->prof_ev[i]);
+        delete[] s->prof_ev;
+    }
+    s->prof_ev = nullptr;
+    s->prof_n = 0;
+    s->prof_count = 0;
+}
+
+void step_free(pkv_step* s) {
+    prof_free(s);
+    for (int i = 0; i < pkv_step::kRing; ++i) {
+        if (s->ev[i]) {
+            cudaEventSynchronize(s->ev[i]);
+            cudaEventDestroy(s->ev[i]);
+        }
+        if (s->h_stage[i]) cudaFreeHost(s->h_stage[i]);
+    }
+    if (s->d_stage) cudaFree(s->d_stage);
+    if (s->d_ws) cudaFree(s->d_ws);
+    delete s;
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_q_heads,
+                           pkv_dtype q_dtype, int partition_tokens, int kernel, pkv_step** out) {
+    if (!pool || pool->host_only || !out || max_batch < 1 || max_batch > 65535 || max_blocks < 1)
+        return PKV_ERR_INVALID_ARG;
+    if (n_q_heads < pool->n_kv_heads || n_q_heads % pool->n_kv_heads) return PKV_ERR_INVALID_ARG;
+    if (pool->dtype == PKV_FP8_E4M3 ? (q_dtype != PKV_F16 && q_dtype != PKV_BF16)
+                                    : q_dtype != pool->dtype)
+        return PKV_ERR_INVALID_ARG;
+    if (partition_tokens != 0 && partition_tokens != -1 &&
+        (partition_tokens < 16 || partition_tokens % 16))
+        return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_TENSOR) return PKV_ERR_INVALID_ARG;
+    if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
+    pkv_step* s = new (std::nothrow) pkv_step();
+    if (!s) return PKV_ERR_INVALID_ARG;
+    s->pool = pool;
+    s->max_batch = max_batch;
+    s->max_blocks = max_blocks;
+    s->n_q_heads = n_q_heads;
+    s->q_dtype = q_dtype;
+    s->partition_tokens = partition_tokens;
+    s->kernel = kernel;
+    s->stage_ints = (size_t)4 * max_batch + (size_t)max_batch * max_blocks;
+    const size_t bytes = s->stage_ints * sizeof(int32_t);
+    bool ok = true;
+    for (int i = 0; i < pkv_step::kRing && ok; ++i) {
+        ok &= cudaMallocHost(&s->h_stage[i], bytes) == cudaSuccess;
+        ok &= ok && cudaEventCreateWithFlags(&s->ev[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    ok &= ok && cudaMalloc(&s->d_stage, bytes) == cudaSuccess;
+    const int P = resolve_partition(pool, max_blocks, partition_tokens);
+    s->max_parts = parts_for(pool, max_blocks, P);
+    s->ws_bytes = workspace_for(pool, max_batch, n_q_heads, s->max_parts);
+    if (ok && s->ws_bytes) ok &= cudaMalloc(&s->d_ws, s->ws_bytes) == cudaSuccess;
+    if (!ok) {
+        step_free(s);
+        return PKV_ERR_CUDA;
+    }
+    *out = s;
+    return PKV_OK;
+}
+
+void pkv_step_destroy(pkv_step* s) {
+    if (s) step_free(s);
+}
+
+int pkv_step_last_launches(const pkv_step* s) { return s ? s->last_launches : 0; }
+
+pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const void* q,
+                           const void* k_new, const void* v_new, float scale, void* out,
+                           void* stream) {
+    if (!s || B < 0 || B > s->max_batch) return PKV_ERR_INVALID_ARG;
+    s->last_launches = 0;
+    if (B == 0) return PKV_OK;
+    if (!seq_ids || !q || !k_new || !v_new || !out) return PKV_ERR_INVALID_ARG;
+    pkv_pool* pool = s->pool;
+    if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
+    // every table must still fit after the append: checked before anything changes
+    for (int i = 0; i < B; ++i) {
+        int32_t nb = 0;
+        pkv_status st = pool->bm.blocks_after_append(seq_ids[i], &nb);
+        if (st != PKV_OK) return st;
+        if (nb > s->max_blocks) return PKV_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int r = s->ring;
+    if (s->pending[r] && cudaEventSynchronize(s->ev[r]) != cudaSuccess) return PKV_ERR_CUDA;
+    s->pending[r] = false;
+    int32_t* h = s->h_stage[r];
+    const int mb = s->max_batch;
+    int n_cow = 0;
+    pkv_status ps = pool->bm.append_batch(seq_ids, B, h, h + mb, h + 2 * mb, &n_cow);
+    if (ps != PKV_OK) return ps;
+    ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, h + 4 * mb, h + 3 * mb, nullptr);
+    if (ps != PKV_OK) return ps;   // cannot happen after the checks above
+    const size_t ints = (size_t)4 * mb + (size_t)B * s->max_blocks;
+    if (cudaMemcpyAsync(s->d_stage, h, ints * sizeof(int32_t), cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaEventRecord(s->ev[r], st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    s->pending[r] = true;
+    s->ring = (r + 1) % pkv_step::kRing;
+    int launches = 0;
+    if (n_cow > 0) {
+        ps = block_copy(pool, s->d_stage + mb, s->d_stage + 2 * mb, n_cow, stream);
+        if (ps != PKV_OK) return ps;
+        ++launches;
+    }
+    ps = kv_append(pool, s->d_stage, B, k_new, v_new, s->q_dtype, stream);
+    if (ps != PKV_OK) return ps;
+    ++launches;
+    cudaEvent_t e0 = nullptr, e1 = nullptr, e2 = nullptr;
+    if (s->prof_n > 0) {
+        const int i = (int)(s->prof_count % s->prof_n);
+        e0 = s->prof_ev[3 * i];
+        e1 = s->prof_ev[3 * i + 1];
+        e2 = s->prof_ev[3 * i + 2];
+    }
+    ps = decode_attention_impl(pool, q, s->q_dtype, s->d_stage + 4 * mb, s->max_blocks,
+                               s->d_stage + 3 * mb, B, s->n_q_heads, scale, out, s->d_ws,
+                               s->ws_bytes, s->partition_tokens, s->kernel, stream, e0, e1, e2);
+    if (ps != PKV_OK) return ps;
+    if (s->prof_n > 0) ++s->prof_count;
+    launches += 1 + (s->max_parts > 1 ? 1 : 0);
+    s->last_launches = launches;
+    return PKV_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+pkv_status pkv_step_profile(pkv_step* s, int n) {
+    if (!s || n < 0) return PKV_ERR_INVALID_ARG;
+    prof_free(s);
+    if (n == 0) return PKV_OK;
+    s->prof_ev = new (std::nothrow) cudaEvent_t[3 * (size_t)n]();
+    if (!s->prof_ev) return PKV_ERR_INVALID_ARG;
+    s->prof_n = n;
+    for (int i = 0; i < 3 * n; ++i)
+        if (cudaEventCreate(&s->prof_ev[i]) != cudaSuccess) {
+            prof_free(s);
+            return PKV_ERR_CUDA;
+        }
+    return PKV_OK;
+}
+
+pkv_status pkv_step_profile_read(pkv_step* s, float* decode_ms, float* merge_ms, int cap,
+                                 int* n_out) {
+    if (!s || !n_out || cap < 0) return PKV_ERR_INVALID_ARG;
+    const int have = (int)(s->prof_count < s->prof_n ? s->prof_count : s->prof_n);
+    if (cap < have || (have > 0 && (!decode_ms || !merge_ms))) return PKV_ERR_INVALID_ARG;
+    const long long first = s->prof_count - have;
+    for (int j = 0; j < have; ++j) {
+        const int i = (int)((first + j) % s->prof_n);
+        if (cudaEventSynchronize(s->prof_ev[3 * i + 2]) != cudaSuccess) return PKV_ERR_CUDA;
+        float a = 0.f, b = 0.f;
+        if (cudaEventElapsedTime(&a, s->prof_ev[3 * i], s->prof_ev[3 * i + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&b, s->prof_ev[3 * i + 1], s->prof_ev[3 * i + 2]) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        decode_ms[j] = a;
+        merge_ms[j] = b;
+    }
+    *n_out = have;
+    return PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Host-side block manager of the paged KV pool.
+//
+// Implements the block-table rules of "KV 缓存与分页注意力" §块表 (one table per
+// sequence: physical block per logical block, fill count of the last block; a
+// new block only when the last one is full; blocks returned when a sequence
+// finishes), the copy-on-write rule of its FAQ 08 and of "读懂PagedAttention"
+// §同一提示生成两个回答的假想例子 (a partially filled last block that is still
+// shared is copied before the write; full shared blocks stay shared), with a
+// FIFO free queue.  Not thread-safe: calls on one pool must be serialised.
+#pragma once
+
+#include <cstdint>
+#include <unordered_map>
+#include <vector>
+
+#include "pagedkv.h"
+
+namespace pkv {
+
+struct Sequence {
+    std::vector<int32_t> blocks;  // logical block i -> physical block id
+    int64_t length = 0;           // tokens stored (the fill count is derived)
+};
+
+class BlockManager {
+  public:
+    BlockManager(int num_blocks, int block_size);
+
+    pkv_status reset(const int32_t* free_order);
+    pkv_status alloc(int64_t seq, int n_tokens, int32_t* slots);
+    pkv_status append(int64_t seq, int32_t* slot, int32_t* cow_src, int32_t* cow_dst);
+    pkv_status append_batch(const int64_t* seqs, int n, int32_t* slots, int32_t* cow_src,
+                            int32_t* cow_dst, int* n_cow);
+    pkv_status fork(int64_t parent, int64_t child);
+    pkv_status release(int64_t seq);
+    pkv_status export_tables(const int64_t* seqs, int n, int max_blocks, int32_t* tables,
+                             int32_t* lens, int32_t* fills) const;
+    pkv_status num_blocks_of(int64_t seq, int32_t* out) const;
+    // table length after one more append (the last block full -> one more)
+    pkv_status blocks_after_append(int64_t seq, int32_t* out) const;
+    pkv_status refcount_of(int32_t block, int32_t* out) const;
+    pkv_status free_queue(int32_t* out, int cap, int* n_out) const;
+    void stats(pkv_stats* out) const;
+
+    int num_blocks() const { return num_blocks_; }
+    int block_size() const { return block_size_; }
+
+  private:
+    // one undo record per successful append inside a batch
+    struct Undo {
+        int64_t seq;
+        int kind;        // 0 = in place, 1 = fresh block pushed, 2 = copy-on-write
+        int32_t old_block;
+    };
+
+    int fill_of_last(const Sequence& s) const;
+    int32_t pop_front();
+    void unpop_front(int32_t b);
+    void push_back(int32_t b);
+    pkv_status append_one(int64_t seq, int32_t* slot, int32_t* src, int32_t* dst, Undo* undo);
+    void undo_one(const Undo& u);
+
+    int num_blocks_;
+    int block_size_;
+    std::vector<int32_t> ring_;   // FIFO free queue as a ring of capacity num_blocks
+    int head_ = 0;
+    int count_ = 0;
+    std::vector<int32_t> ref_;
+    std::unordered_map<int64_t, Sequence> seqs_;
+    int64_t cow_count_ = 0;
+};
+
+}  // namespace pkv

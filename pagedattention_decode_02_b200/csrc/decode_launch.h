@@ -1,0 +1,34 @@
+// Host-side launchers of the decode-path kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "kernels_common.cuh"
+
+namespace pkv {
+
+// CUDA-core decode (any grouping, any storage type) + partition merge.
+int simt_heads_per_cta(int group);
+// mid (may be null) is recorded on st after the decode kernel, before the merge.
+cudaError_t launch_decode_simt(const DecodeParams& p, int kv_dtype, int q_dtype, int head_dim,
+                               int heads_per_cta, cudaStream_t st, cudaEvent_t mid = nullptr);
+
+// Tensor-core decode of grouped heads (F16/BF16 pools, G > 1) + partition merge.
+bool tensor_path_supported(int kv_dtype, int q_dtype, int head_dim, int group, int block_size);
+cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
+                                 int kv_dtype, int head_dim, cudaStream_t st,
+                                 cudaEvent_t mid = nullptr);
+
+// Store new rows into their slots (FP8 pools quantise).
+cudaError_t launch_kv_append(uint8_t* k_pool, uint8_t* v_pool, const int32_t* slots, int n_tokens,
+                             const void* k, const void* v, int in_dtype, int kv_dtype,
+                             int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                             float k_scale, float v_scale, uint32_t* err, cudaStream_t st);
+
+// Whole-block copies src[i] -> dst[i] of K and V.
+cudaError_t launch_block_copy(uint8_t* k_pool, uint8_t* v_pool, const int32_t* src,
+                              const int32_t* dst, int n_pairs, long long block_bytes,
+                              int num_blocks, uint32_t* err, cudaStream_t st);
+
+}  // namespace pkv

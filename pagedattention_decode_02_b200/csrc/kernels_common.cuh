@@ -1,0 +1,251 @@
+// Device helpers shared by the paged-KV kernels (sm_100a).
+//
+// - mbarrier + 1-D bulk copies (cp.async.bulk, no multicast, this GPU's own
+//   memory only) for staging K/V rows into shared memory;
+// - bounded waits: every wait on a copy gives up after a fixed wall-clock
+//   budget, sets a bit in the pool's device error word and lets the kernel
+//   finish instead of hanging;
+// - element conversions for the four storage types.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pagedkv.h"
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// element types
+// ---------------------------------------------------------------------------
+struct fp8e4m3 {
+    uint8_t x;
+};
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+    static constexpr int bytes = 4;
+    static constexpr int id = PKV_F32;
+    __device__ static float to_f(float v) { return v; }
+    __device__ static float from_f(float v) { return v; }
+};
+template <>
+struct Elem<__half> {
+    static constexpr int bytes = 2;
+    static constexpr int id = PKV_F16;
+    __device__ static float to_f(__half v) { return __half2float(v); }
+    __device__ static __half from_f(float v) { return __float2half_rn(v); }
+};
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int bytes = 2;
+    static constexpr int id = PKV_BF16;
+    __device__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    __device__ static __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+template <>
+struct Elem<fp8e4m3> {
+    static constexpr int bytes = 1;
+    static constexpr int id = PKV_FP8_E4M3;
+};
+
+// Load N consecutive elements of type T from shared/global memory as floats.
+// N * sizeof(T) is 4, 8 or 16 bytes; the address is aligned to that size.
+template <typename T, int N>
+struct VecLoad;
+
+template <int N>
+struct VecLoad<float, N> {
+    __device__ static void run(const void* p, float* out) {
+        if constexpr (N == 4) {
+            float4 v = *reinterpret_cast<const float4*>(p);
+            out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+        } else if constexpr (N == 2) {
+            float2 v = *reinterpret_cast<const float2*>(p);
+            out[0] = v.x; out[1] = v.y;
+        } else {
+            static_assert(N == 1, "");
+            out[0] = *reinterpret_cast<const float*>(p);
+        }
+    }
+};
+
+template <int N>
+struct VecLoad<__half, N> {
+    __device__ static void run(const void* p, float* out) {
+        if constexpr (N == 4) {
+            uint2 u = *reinterpret_cast<const uint2*>(p);
+            float2 a = __half22float2(*reinterpret_cast<__half2*>(&u.x));
+            float2 b = __half22float2(*reinterpret_cast<__half2*>(&u.y));
+            out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+        } else if constexpr (N == 2) {
+            uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+            float2 a = __half22float2(*reinterpret_cast<__half2*>(&u));
+            out[0] = a.x; out[1] = a.y;
+        } else {
+            static_assert(N == 1, "");
+            out[0] = __half2float(*reinterpret_cast<const __half*>(p));
+        }
+    }
+};
+
+template <int N>
+struct VecLoad<__nv_bfloat16, N> {
+    __device__ static void run(const void* p, float* out) {
+        if constexpr (N == 4) {
+            uint2 u = *reinterpret_cast<const uint2*>(p);
+            out[0] = __uint_as_float(u.x << 16); out[1] = __uint_as_float(u.x & 0xFFFF0000u);
+            out[2] = __uint_as_float(u.y << 16); out[3] = __uint_as_float(u.y & 0xFFFF0000u);
+        } else if constexpr (N == 2) {
+            uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+            out[0] = __uint_as_float(u << 16); out[1] = __uint_as_float(u & 0xFFFF0000u);
+        } else {
+            static_assert(N == 1, "");
+            uint32_t u = *reinterpret_cast<const uint16_t*>(p);
+            out[0] = __uint_as_float(u << 16);
+        }
+    }
+};
+
+// two FP8-E4M3 codes -> two floats, exact (through the hardware e4m3x2 -> f16x2 convert)
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+
+template <int N>
+struct VecLoad<fp8e4m3, N> {
+    __device__ static void run(const void* p, float* out) {
+        if constexpr (N == 4) {
+            uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+            float2 a = e4m3x2_to_float2((uint16_t)(u & 0xFFFF));
+            float2 b = e4m3x2_to_float2((uint16_t)(u >> 16));
+            out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+        } else if constexpr (N == 2) {
+            float2 a = e4m3x2_to_float2(*reinterpret_cast<const uint16_t*>(p));
+            out[0] = a.x; out[1] = a.y;
+        } else {
+            static_assert(N == 1, "");
+            uint16_t u = *reinterpret_cast<const uint8_t*>(p);
+            out[0] = e4m3x2_to_float2(u).x;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// error word
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void report_error(uint32_t* err, uint32_t bits) {
+    if (err) atomicOr(err, bits);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk copies
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// make barrier initialisation visible to the async (bulk copy) proxy
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the barrier phase with the given parity.  Gives up after
+// kWaitBudgetNs of wall-clock time and returns false.  A healthy copy of a
+// few KB completes in microseconds; the budget only ends a wait that would
+// otherwise never end.
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > kWaitBudgetNs) return false;
+    }
+}
+
+// 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned)
+// from this GPU's global memory into this CTA's shared memory; completion is
+// counted on `bar` in bytes.  The L2 policy marks the lines evict-first: the
+// KV stream is read once per step.
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src_gmem, uint32_t bytes,
+                                          uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// kernel parameter blocks
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+    const void* q;
+    void* out;
+    const uint8_t* k_pool;
+    const uint8_t* v_pool;
+    const int32_t* tables;
+    const int32_t* lens;
+    float* ws_ml;    // [B][H_q][max_parts][2]  (running max in log2 units, sum)
+    float* ws_acc;   // [B][H_q][max_parts][D]  (unnormalised accumulator)
+    uint32_t* err;
+    int B, H_q, H_kv, G;
+    int max_blocks, block_size, num_blocks;
+    int part_tokens;  // tokens per partition (multiple of 16)
+    int max_parts;    // partitions of the longest possible context
+    float q_scale;    // scale * log2(e) * k_scale: folded into q
+    float v_scale;    // FP8 V dequantisation (1 otherwise)
+    long long head_stride;   // bytes of one (block, kv head) tile: bs * D * elem
+    long long block_stride;  // bytes of one block: H_kv * head_stride
+};
+
+}  // namespace pkv

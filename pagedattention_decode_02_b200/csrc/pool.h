@@ -1,0 +1,38 @@
+// The pool object behind the opaque pkv_pool handle.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "block_manager.h"
+#include "pagedkv.h"
+
+struct pkv_pool {
+    pkv_pool(int num_blocks, int block_size) : bm(num_blocks, block_size) {}
+
+    int num_blocks = 0;
+    int block_size = 0;
+    int n_kv_heads = 0;
+    int head_dim = 0;
+    pkv_dtype dtype = PKV_F32;
+    float k_scale = 1.f;
+    float v_scale = 1.f;
+    bool host_only = false;
+    bool owns_buffers = false;
+    int device = -1;
+    uint8_t* k = nullptr;   // device [num_blocks][n_kv_heads][block_size][head_dim]
+    uint8_t* v = nullptr;
+    size_t bytes = 0;       // bytes of one of the two buffers
+    uint32_t* d_err = nullptr;
+    pkv::BlockManager bm;
+    // TMA descriptors of the K and V pools (CUtensorMap, 128 bytes each) for
+    // the tensor-core decode path; valid when has_tmaps.
+    alignas(64) unsigned char tmap_k[128] = {};
+    alignas(64) unsigned char tmap_v[128] = {};
+    bool has_tmaps = false;
+};
+
+namespace pkv {
+// device-side extras set up after the buffers exist (tensor maps)
+void pool_init_device_extras(pkv_pool* p);
+}  // namespace pkv
