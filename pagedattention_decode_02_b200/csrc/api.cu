@@ -307,7 +307,7 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
     if ((long long)max_parts > 0x7fffffffLL || B > 65535) return PKV_ERR_INVALID_ARG;
 
-    const bool tc_ok = pkv::tensor_path_supported(p->dtype, q_dtype, p->head_dim, G, p->block_size);
+    const bool tc_ok = pkv::tensor_path_supported(p, q_dtype, G);
     int use = kernel;
     if (use == PKV_KERNEL_AUTO) use = tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT;
     if (use == PKV_KERNEL_TENSOR && !tc_ok) return PKV_ERR_INVALID_ARG;

@@ -14,8 +14,15 @@ int simt_heads_per_cta(int group);
 cudaError_t launch_decode_simt(const DecodeParams& p, int kv_dtype, int q_dtype, int head_dim,
                                int heads_per_cta, cudaStream_t st, cudaEvent_t mid = nullptr);
 
-// Tensor-core decode of grouped heads (F16/BF16 pools, G > 1) + partition merge.
-bool tensor_path_supported(int kv_dtype, int q_dtype, int head_dim, int group, int block_size);
+// Log-sum-exp merge of the partitions (a no-op grid when max_parts <= 1).
+cudaError_t launch_merge(const DecodeParams& p, int q_dtype, int head_dim, cudaStream_t st);
+
+}  // namespace pkv
+struct pkv_pool;
+namespace pkv {
+// Tensor-core decode of grouped heads (F16/BF16 pools with TMA descriptors,
+// 1 < G <= 128) + partition merge.
+bool tensor_path_supported(const pkv_pool* pool, int q_dtype, int group);
 cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
                                  int kv_dtype, int head_dim, cudaStream_t st,
                                  cudaEvent_t mid = nullptr);

@@ -401,6 +401,21 @@ cudaError_t launch_simt_q(const DecodeParams& p, int D, int hpc, cudaStream_t st
 
 }  // namespace
 
+cudaError_t launch_merge(const DecodeParams& p, int q_dtype, int D, cudaStream_t st) {
+    const dim3 grid(p.H_q, p.B);
+#define PKV_MERGE(QT, DD) merge_kernel<QT, DD><<<grid, DD, 0, st>>>(p)
+    if (q_dtype == PKV_F32) {
+        if (D == 32) PKV_MERGE(float, 32); else if (D == 64) PKV_MERGE(float, 64); else PKV_MERGE(float, 128);
+    } else if (q_dtype == PKV_F16) {
+        if (D == 32) PKV_MERGE(__half, 32); else if (D == 64) PKV_MERGE(__half, 64); else PKV_MERGE(__half, 128);
+    } else {
+        if (D == 32) PKV_MERGE(__nv_bfloat16, 32); else if (D == 64) PKV_MERGE(__nv_bfloat16, 64);
+        else PKV_MERGE(__nv_bfloat16, 128);
+    }
+#undef PKV_MERGE
+    return cudaGetLastError();
+}
+
 int simt_heads_per_cta(int group) {
     for (int h : {8, 4, 2})
         if (group % h == 0) return h;

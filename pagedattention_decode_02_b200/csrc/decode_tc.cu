@@ -1,16 +1,547 @@
-// Tensor-core decode of grouped query heads (placeholder until the kernel lands).
+// Paged decode attention for grouped query heads on tensor cores.
+//
+// With G = H_q / H_kv > 1 query heads per KV head ("KV 缓存与分页注意力"
+// §后来的做法: Llama-2-70B puts 64 heads on 8 K/V groups, Falcon-7B all heads on
+// one), every K/V element read from HBM is used G times, so one KV head's
+// group is a small dense contraction per 16-token stage:
+//     S[G x 16]  = Q_group[G x d] . K_stage^T[d x 16]
+//     O[G x d]  += P[G x 16] . V_stage[16 x d]
+// done with mma.sync m16n8k16 (f16/bf16 in, fp32 accumulate).  The path stays
+// HBM-bound (8 flop/B at G = 8, 71 at G = 71); the tensor cores only remove
+// the CUDA-core FMA bound that G scalar dot products per element would hit.
+//
+// Staging: the pool is viewed by two TMA tensor maps (K and V) as a 2-D
+// tensor [num_blocks * H_kv * bs rows][d] with 128-byte swizzle; one stage is
+// a 16-row box per 64-column half (or two 8-row boxes when bs == 8), so each
+// 8 x 16-byte ldmatrix read hits 8 different bank groups.  Loads are plain
+// (no multicast) from this GPU's own memory.
+//
+// CTA = (partition, KV head, sequence).  Warps: MT m-tiles of 16 query heads
+// (MT = ceil(G / 16)) x TS token groups.  Each token group owns a ring of
+// kStages slots; lane 0 of its first warp issues the copies, every warp of the
+// group consumes every stage, and with MT > 1 an "empty" mbarrier per slot
+// (MT arrivals) tells the producer when all of them are done with it.
+// The scores' accumulator fragments are re-packed in registers as the A
+// operand of the P.V product; online softmax runs in base 2 per head row.
+#include <cuda.h>
+
+#include <cfloat>
+
 #include "decode_launch.h"
+#include "kernels_common.cuh"
 #include "pool.h"
 
 namespace pkv {
 
-void pool_init_device_extras(pkv_pool* p) { p->has_tmaps = false; }
+namespace {
 
-bool tensor_path_supported(int, int, int, int, int) { return false; }
+constexpr int kStageTokens = 16;
+constexpr int kStages = 3;
 
-cudaError_t launch_decode_tensor(const DecodeParams&, const void*, const void*, int, int,
-                                 cudaStream_t, cudaEvent_t) {
-    return cudaErrorNotSupported;
+template <typename T>
+struct MmaType;
+template <>
+struct MmaType<__half> {
+    __device__ static uint32_t pack(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+};
+template <>
+struct MmaType<__nv_bfloat16> {
+    __device__ static uint32_t pack(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// 2-D tiled TMA load of one box into shared memory, completion on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Byte offset of 16-byte chunk c (of the row's d / 8 chunks) in row r of a
+// swizzled stage tile: [d / 64 halves][16 rows][128 B], chunk index XOR (r % 8).
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)((c >> 3) * (kStageTokens * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <int D>
+struct TcSmem {
+    static constexpr int kTile = kStageTokens * D * 2;   // bytes of K (or V) of one stage
+    static constexpr int kSlot = 2 * kTile;
+};
+
+template <int D, int MT, int TS>
+__host__ __device__ constexpr int tc_union_bytes() {
+    const int tiles = TS * kStages * TcSmem<D>::kSlot;
+    const int comb = MT * TS * 16 * (D + 2) * 4;
+    return ((tiles > comb ? tiles : comb) + 15) & ~15;
+}
+
+template <typename T, int D, int MT, int TS>
+__global__ void __launch_bounds__(MT * TS * 32)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+    constexpr int NW = MT * TS;
+    constexpr int NT = NW * 32;
+    constexpr int TILE = TcSmem<D>::kTile;
+    constexpr int SLOT = TcSmem<D>::kSlot;
+    constexpr int KSTEPS = D / 16;       // k-steps of S = Q K^T
+    constexpr int DTILES = D / 8;        // n-tiles of O
+    constexpr int HALVES = D / 64;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment of the swizzled tiles; the combine area reuses the
+    // tile ring once every stage has been consumed
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* tiles = smem;                                            // [TS][kStages][SLOT]
+    float* comb = reinterpret_cast<float*>(smem);                     // [NW][16][D + 2]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS>());
+    uint64_t* empty = full + TS * kStages;
+
+    const int part = blockIdx.x;
+    const int g = blockIdx.y;
+    const int seq = blockIdx.z;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int mt = warp % MT;       // m-tile of this warp
+    const int ts = warp / MT;       // token group of this warp
+    const int G = p.G;
+    const int bs = p.block_size;
+    const int P = p.part_tokens;
+    const int h_base = g * G;       // first query head of the group
+
+    const int c = p.lens[seq];
+    if (c < 1 || c > p.max_blocks * bs) {
+        if (part == 0) {
+            if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
+            T* out = reinterpret_cast<T*>(p.out);
+            for (int i = tid; i < G * D; i += NT)
+                out[((size_t)seq * p.H_q + h_base + i / D) * D + i % D] = Elem<T>::from_f(0.f);
+        }
+        return;
+    }
+    const int nparts = (c + P - 1) / P;
+    if (part >= nparts) return;
+    const int t_begin = part * P;
+    const int t_end = min(c, t_begin + P);
+    const int32_t* table = p.tables + (size_t)seq * p.max_blocks;
+
+    bool bad = false;
+    for (int lb = t_begin / bs + tid; lb <= (t_end - 1) / bs; lb += NT) {
+        const int32_t b = table[lb];
+        bad |= (b < 0 || b >= p.num_blocks);
+    }
+    if (tid == 0) {
+        for (int i = 0; i < TS * kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], MT);
+        }
+        fence_mbar_init();
+    }
+    const bool split = nparts > 1;
+    if (__syncthreads_or(bad)) {
+        if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
+        for (int i = tid; i < G * D; i += NT) {
+            const int h = h_base + i / D, d = i % D;
+            const size_t row = ((size_t)seq * p.H_q + h) * p.max_parts + part;
+            if (split) {
+                p.ws_acc[row * D + d] = 0.f;
+                if (d == 0) { p.ws_ml[row * 2] = -INFINITY; p.ws_ml[row * 2 + 1] = 0.f; }
+            } else {
+                reinterpret_cast<T*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<T>::from_f(0.f);
+            }
+        }
+        return;
+    }
+
+    const int n_stages = (t_end - t_begin + kStageTokens - 1) / kStageTokens;
+    const int my_n = n_stages > ts ? (n_stages - ts + TS - 1) / TS : 0;
+    uint8_t* ring = tiles + ts * kStages * SLOT;
+    uint64_t* my_full = full + ts * kStages;
+    uint64_t* my_empty = empty + ts * kStages;
+    const bool producer = (mt == 0);
+    const uint64_t policy = l2_evict_first_policy();
+    const int rows_per_box = bs < kStageTokens ? bs : kStageTokens;   // 8 or 16
+
+    // issue stage k_local (this group's k-th) into `slot`; called by the
+    // producer warp (all lanes)
+    auto issue = [&](int k_local, int slot) {
+        const int a = t_begin + (ts + k_local * TS) * kStageTokens;
+        const int n = min(kStageTokens, t_end - a);
+        const int n_boxes = (n + rows_per_box - 1) / rows_per_box;   // boxes per half
+        uint8_t* kd = ring + slot * SLOT;
+        uint8_t* vd = kd + TILE;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&my_full[slot], (uint32_t)(2 * HALVES * n_boxes * rows_per_box * 128));
+            for (int bx = 0; bx < n_boxes; ++bx) {
+                const int t0 = a + bx * rows_per_box;
+                const int lb = t0 / bs;
+                const int y = (table[lb] * p.H_kv + g) * bs + (t0 - lb * bs);
+#pragma unroll
+                for (int hf = 0; hf < HALVES; ++hf) {
+                    const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
+                    tma_load_2d(kd + off, &tmap_k, hf * 64, y, &my_full[slot], policy);
+                    tma_load_2d(vd + off, &tmap_v, hf * 64, y, &my_full[slot], policy);
+                }
+            }
+        }
+        __syncwarp();
+    };
+
+    // Q fragments (A operand) of this warp's 16 heads, zero past the group
+    const int gq = lane >> 2;       // fragment row (and row + 8)
+    const int tq = lane & 3;        // fragment column pair
+    uint32_t qa[KSTEPS][4];
+    {
+        const T* qp = reinterpret_cast<const T*>(p.q);
+        const int r0 = mt * 16 + gq, r1 = r0 + 8;
+        const T* q0 = qp + ((size_t)seq * p.H_q + h_base + r0) * D;
+        const T* q1 = qp + ((size_t)seq * p.H_q + h_base + r1) * D;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            const int c0 = kk * 16 + 2 * tq;
+            qa[kk][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(q0 + c0) : 0u;
+            qa[kk][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(q1 + c0) : 0u;
+            qa[kk][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(q0 + c0 + 8) : 0u;
+            qa[kk][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(q1 + c0 + 8) : 0u;
+        }
+    }
+
+    float o[DTILES][4];
+#pragma unroll
+    for (int j = 0; j < DTILES; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+
+    if (producer) {
+        const int pro = min(kStages, my_n);
+        for (int k = 0; k < pro; ++k) issue(k, k);
+    }
+
+    int k = 0;
+    bool timed_out = false;
+    for (; k < my_n; ++k) {
+        const int slot = k % kStages;
+        if (!mbar_wait(&my_full[slot], (uint32_t)((k / kStages) & 1))) {
+            timed_out = true;
+            break;
+        }
+        const int a = t_begin + (ts + k * TS) * kStageTokens;
+        const int n = min(kStageTokens, t_end - a);
+        uint8_t* kt = ring + slot * SLOT;
+        uint8_t* vt = kt + TILE;
+        if (n < kStageTokens) {
+            // rows past the context hold stale bytes: zero V there so that
+            // P = 0 times them stays 0 (each warp zeroes its own view; the
+            // values are identical, so overlapping writes are harmless)
+            for (int i = lane; i < (kStageTokens - n) * (D / 8); i += 32) {
+                const int r = n + i / (D / 8), cc = i % (D / 8);
+                *reinterpret_cast<uint4*>(vt + swz(r, cc)) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();   // before the slot can be refilled by TMA
+            __syncwarp();
+        }
+        const uint32_t kbase = smem_addr(kt);
+        const uint32_t vbase = smem_addr(vt);
+
+        // S = Q K^T : two n-tiles of 8 tokens
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int mi = lane >> 3, r = lane & 7;
+            const int tok = (mi >> 1) * 8 + r;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kbase + swz(tok, 2 * kk + (mi & 1)), b0, b1, b2, b3);
+                MmaType<T>::mma(s[0], qa[kk], b0, b1);
+                MmaType<T>::mma(s[1], qa[kk], b2, b3);
+            }
+        }
+        // online softmax over this stage's tokens, per head row (gq, gq + 8)
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = 8 * j + 2 * tq + (e & 1);
+                float v = s[j][e] * p.q_scale;
+                v = tok < n ? v : -INFINITY;
+                s[j][e] = v;
+                mx[e >> 1] = fmaxf(mx[e >> 1], v);
+            }
+        float alpha[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+            const float m_new = fmaxf(m_run[r], mx[r]);
+            alpha[r] = exp2f(m_run[r] - m_new);
+            m_run[r] = m_new;
+            l_run[r] *= alpha[r];
+        }
+        uint32_t pa[4];
+        {
+            float pr[2][4];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    pr[j][e] = exp2f(s[j][e] - m_run[e >> 1]);
+                    l_run[e >> 1] += pr[j][e];
+                }
+            pa[0] = MmaType<T>::pack(pr[0][0], pr[0][1]);
+            pa[1] = MmaType<T>::pack(pr[0][2], pr[0][3]);
+            pa[2] = MmaType<T>::pack(pr[1][0], pr[1][1]);
+            pa[3] = MmaType<T>::pack(pr[1][2], pr[1][3]);
+        }
+#pragma unroll
+        for (int j = 0; j < DTILES; ++j) {
+            o[j][0] *= alpha[0];
+            o[j][1] *= alpha[0];
+            o[j][2] *= alpha[1];
+            o[j][3] *= alpha[1];
+        }
+        // O += P V : V^T fragments by transposed ldmatrix, two d-tiles per load
+        {
+            const int mi = lane >> 3, r = lane & 7;
+            const int tok = (mi & 1) * 8 + r;
+#pragma unroll
+            for (int j = 0; j < DTILES; j += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vbase + swz(tok, j + (mi >> 1)), b0, b1, b2, b3);
+                MmaType<T>::mma(o[j], pa, b0, b1);
+                MmaType<T>::mma(o[j + 1], pa, b2, b3);
+            }
+        }
+        __syncwarp();
+        if constexpr (MT > 1) {
+            if (lane == 0) mbar_arrive(&my_empty[slot]);
+        }
+        if (producer && k + kStages < my_n) {
+            if constexpr (MT > 1) {
+                if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1))) {
+                    timed_out = true;
+                    ++k;
+                    break;
+                }
+            }
+            issue(k + kStages, slot);
+        }
+    }
+    if (timed_out) {
+        if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
+        // bounded wait for copies this group may still have in flight
+        if (producer)
+            for (int j = k; j < min(my_n, k + kStages); ++j)
+                (void)mbar_wait(&my_full[j % kStages], (uint32_t)((j / kStages) & 1));
+    }
+
+    // full row sums: the four lanes of a quad hold disjoint token columns
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+    }
+    __syncthreads();   // every ring slot consumed: the combine area may be written
+    // per-warp state -> shared memory [NW][16 rows][D + 2]
+    {
+        float* cw = comb + warp * 16 * (D + 2);
+#pragma unroll
+        for (int j = 0; j < DTILES; ++j) {
+            const int col = 8 * j + 2 * tq;
+            cw[gq * (D + 2) + col] = o[j][0];
+            cw[gq * (D + 2) + col + 1] = o[j][1];
+            cw[(gq + 8) * (D + 2) + col] = o[j][2];
+            cw[(gq + 8) * (D + 2) + col + 1] = o[j][3];
+        }
+        if (tq == 0) {
+            cw[gq * (D + 2) + D] = m_run[0];
+            cw[gq * (D + 2) + D + 1] = l_run[0];
+            cw[(gq + 8) * (D + 2) + D] = m_run[1];
+            cw[(gq + 8) * (D + 2) + D + 1] = l_run[1];
+        }
+    }
+    __syncthreads();
+    // combine the token groups of each m-tile and write the G real heads
+    for (int i = tid; i < MT * 16 * D; i += NT) {
+        const int m_tile = i / (16 * D);
+        const int row = (i / D) % 16;
+        const int d = i % D;
+        const int hrow = m_tile * 16 + row;
+        if (hrow >= G) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < TS; ++t)
+            M = fmaxf(M, comb[((t * MT + m_tile) * 16 + row) * (D + 2) + D]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int t = 0; t < TS; ++t) {
+            const float* cw = comb + ((t * MT + m_tile) * 16 + row) * (D + 2);
+            const float w = M == -INFINITY ? 0.f : exp2f(cw[D] - M);
+            L = fmaf(cw[D + 1], w, L);
+            O = fmaf(cw[d], w, O);
+        }
+        const int h = h_base + hrow;
+        if (split) {
+            const size_t prow = ((size_t)seq * p.H_q + h) * p.max_parts + part;
+            p.ws_acc[prow * D + d] = O;
+            if (d == 0) {
+                p.ws_ml[prow * 2] = M;
+                p.ws_ml[prow * 2 + 1] = L;
+            }
+        } else {
+            reinterpret_cast<T*>(p.out)[((size_t)seq * p.H_q + h) * D + d] =
+                Elem<T>::from_f(L > 0.f ? O / L : 0.f);
+        }
+    }
+}
+
+template <int D, int MT, int TS>
+constexpr int tc_smem_bytes() {
+    return 1024 + tc_union_bytes<D, MT, TS>() + 2 * TS * kStages * 8;
+}
+
+template <typename T, int D, int MT, int TS>
+cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
+                        int q_dtype, cudaStream_t st, cudaEvent_t mid) {
+    constexpr int smem = tc_smem_bytes<D, MT, TS>();
+    static_assert(smem <= 227 * 1024, "shared memory budget");
+    auto kern = decode_tc_kernel<T, D, MT, TS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(p.max_parts, p.H_kv, p.B);
+    kern<<<grid, MT * TS * 32, smem, st>>>(*tk, *tv, p);
+    e = cudaGetLastError();
+    if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
+    if (e != cudaSuccess || p.max_parts <= 1) return e;
+    return launch_merge(p, q_dtype, D, st);
+}
+
+template <typename T, int D>
+cudaError_t launch_tc_d(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
+                        int q_dtype, cudaStream_t st, cudaEvent_t mid) {
+    const int mt = (p.G + 15) / 16;
+    switch (mt) {
+        case 1: return launch_tc_t<T, D, 1, 4>(p, tk, tv, q_dtype, st, mid);
+        case 2: return launch_tc_t<T, D, 2, 2>(p, tk, tv, q_dtype, st, mid);
+        case 3: return launch_tc_t<T, D, 3, 1>(p, tk, tv, q_dtype, st, mid);
+        case 4: return launch_tc_t<T, D, 4, 1>(p, tk, tv, q_dtype, st, mid);
+        case 5: return launch_tc_t<T, D, 5, 1>(p, tk, tv, q_dtype, st, mid);
+        case 6: return launch_tc_t<T, D, 6, 1>(p, tk, tv, q_dtype, st, mid);
+        case 7: return launch_tc_t<T, D, 7, 1>(p, tk, tv, q_dtype, st, mid);
+        case 8: return launch_tc_t<T, D, 8, 1>(p, tk, tv, q_dtype, st, mid);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda)
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+bool encode_pool_map(CUtensorMap* map, void* base, int dtype, int D, long long rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType t =
+        dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return fn(map, t, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+void pool_init_device_extras(pkv_pool* p) {
+    p->has_tmaps = false;
+    if ((p->dtype != PKV_F16 && p->dtype != PKV_BF16) || (p->head_dim != 64 && p->head_dim != 128))
+        return;
+    // a 16-token stage must be one 16-row box inside a block, or two 8-row boxes
+    if (p->block_size != 8 && p->block_size % 16 != 0) return;
+    const long long rows = (long long)p->num_blocks * p->n_kv_heads * p->block_size;
+    if (rows >= (1LL << 31)) return;
+    const int box_rows = p->block_size < kStageTokens ? p->block_size : kStageTokens;
+    static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+    p->has_tmaps = encode_pool_map(reinterpret_cast<CUtensorMap*>(p->tmap_k), p->k, p->dtype,
+                                   p->head_dim, rows, box_rows) &&
+                   encode_pool_map(reinterpret_cast<CUtensorMap*>(p->tmap_v), p->v, p->dtype,
+                                   p->head_dim, rows, box_rows);
+}
+
+bool tensor_path_supported(const pkv_pool* pool, int q_dtype, int group) {
+    return pool->has_tmaps && q_dtype == pool->dtype && group > 1 && group <= 128;
+}
+
+cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
+                                 int kv_dtype, int D, cudaStream_t st, cudaEvent_t mid) {
+    const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(tmap_k);
+    const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(tmap_v);
+    if (kv_dtype == PKV_F16) {
+        if (D == 64) return launch_tc_d<__half, 64>(p, tk, tv, PKV_F16, st, mid);
+        if (D == 128) return launch_tc_d<__half, 128>(p, tk, tv, PKV_F16, st, mid);
+    } else if (kv_dtype == PKV_BF16) {
+        if (D == 64) return launch_tc_d<__nv_bfloat16, 64>(p, tk, tv, PKV_BF16, st, mid);
+        if (D == 128) return launch_tc_d<__nv_bfloat16, 128>(p, tk, tv, PKV_BF16, st, mid);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace pkv

@@ -251,3 +251,40 @@ def test_fp8_full(bs):
     gpu, ref, info = decode_step(side, seqs, 0, check_heads=heads)
     compare_out(gpu, ref, "fp8", heads)
     check_pool_bytes(side, seqs[:8])
+
+
+# ---------------------------------------------------------------------------
+# tensor-core path for grouped heads, forced
+# ---------------------------------------------------------------------------
+TC_CASES = [
+    (dt, d, bs, hq, hkv, part)
+    for dt in ("f16", "bf16")
+    for d in (64, 128)
+    for bs in (8, 16, 32)
+    for (hq, hkv) in ((4, 2), (16, 2), (71, 1), (64, 8), (128, 1))
+    for part in (0, 32)
+    if not (d == 128 and hq == 128 and bs == 32)
+]
+
+
+@pytest.mark.parametrize("dt,d,bs,hq,hkv,part", TC_CASES)
+def test_tensor_path(dt, d, bs, hq, hkv, part):
+    cfg = small("llama2_70b", n_q_heads=hq, n_kv_heads=hkv, head_dim=d, kv_dtype=dt, q_dtype=dt,
+                block_size=bs, batch=3, lengths=("uniform", 1, 180))
+    side = setup_config(cfg, seed=bs + hq)
+    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0, partition_tokens=part,
+                              kernel=pk.PKV_KERNEL_TENSOR)
+    compare_out(gpu, ref, dt)
+
+
+def test_tensor_path_refuses_unsupported_shapes():
+    for dt, d, bs in (("f32", 64, 16), ("f16", 32, 16), ("f16", 64, 4), ("f16", 64, 24)):
+        pool = pk.kv_pool_create(16, bs, 1, d, dt)
+        tdt = {"f32": torch.float32, "f16": torch.float16}[dt]
+        q = torch.zeros(1, 4, d, device="cuda", dtype=tdt)
+        tables = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
+        lens = torch.ones(1, dtype=torch.int32, device="cuda")
+        with pytest.raises(pk.PagedKVError):
+            pk.paged_decode_attention(pool, q, tables, lens, 0.1, kernel=pk.PKV_KERNEL_TENSOR)
+        # the automatic choice falls back to the CUDA-core kernel
+        pk.paged_decode_attention(pool, q, tables, lens, 0.1)
