@@ -60,7 +60,9 @@ typedef enum {
     PKV_ERR_UNKNOWN_SEQ = 3,  /* sequence id not in the pool */
     PKV_ERR_SEQ_EXISTS = 4,   /* sequence id already in the pool */
     PKV_ERR_CUDA = 5,         /* a CUDA runtime call failed */
-    PKV_ERR_DEVICE = 6        /* the device error word was set (see pkv_device_error) */
+    PKV_ERR_DEVICE = 6,       /* the device error word was set (see pkv_device_error) */
+    PKV_ERR_SCRATCH_LIMIT = 7 /* the request needs more than the static scratch of
+                                 paged_decode_attention_static; nothing launched */
 } pkv_status;
 
 typedef enum {
@@ -322,6 +324,39 @@ pkv_status pkv_step_profile(pkv_step* step, int n);
  *   Waits for those events.  Errors: INVALID_ARG (cap too small), CUDA. */
 pkv_status pkv_step_profile_read(pkv_step* step, float* decode_ms, float* merge_ms, int cap,
                                  int* n_out);
+
+/* paged_decode_attention_static - paged_decode_attention for callers that
+ *   cannot allocate device memory: processes whose GPU memory is already held
+ *   by another allocator (a direct cudaMalloc would fail or fragment it), and
+ *   latency-bound loops that allow no cudaMalloc/cudaFree after warm-up
+ *   because those calls can synchronise the whole device.  The pages have no
+ *   counterpart: this is a deployment variant of the same computation.
+ *   Arguments and results as paged_decode_attention_ex with kernel = AUTO,
+ *   except that no workspace is passed: the split-context scratch is a
+ *   file-scope device array of paged_decode_static_scratch_bytes() (8 MiB),
+ *   held by every GPU that loads the library until the process exits.  This
+ *   call allocates nothing.
+ *   partition_tokens: 0 = automatic - the library's choice, or longer
+ *   partitions (less scratch) until the scratch fits, down to an unsplit pass
+ *   that needs none; > 0 (a multiple of 16) or -1 as in
+ *   paged_decode_attention_ex, and a request whose scratch exceeds the limit
+ *   returns PKV_ERR_SCRATCH_LIMIT without launching anything.
+ *   The first call on a device looks up the array's device address for that
+ *   device (cudaGetSymbolAddress, with that device current); make that first
+ *   call before any stream capture.  All calls share the one array and it
+ *   keeps the last call's contents; nothing in it needs to start at zero
+ *   (every partition's state is written before the merge reads it), but calls
+ *   whose kernels overlap on the GPU - on different streams, or from several
+ *   host threads - race on it: order them on one stream.
+ *   Errors: INVALID_ARG, SCRATCH_LIMIT, CUDA. */
+pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
+                                         const int32_t* d_block_tables, int max_blocks,
+                                         const int32_t* d_context_lens, int B, int n_q_heads,
+                                         float scale, void* d_out, int partition_tokens,
+                                         void* stream);
+
+/* paged_decode_static_scratch_bytes - size of the static scratch array. */
+size_t paged_decode_static_scratch_bytes(void);
 
 /* pkv_device_error - synchronises the stream, returns the device error word's
  *   bits in *bits_out (may be NULL) and clears it.  Returns PKV_ERR_DEVICE if

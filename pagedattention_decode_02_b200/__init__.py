@@ -31,7 +31,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 # enums and structs (mirror include/pagedkv.h)
 # ---------------------------------------------------------------------------
 PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_NO_BLOCKS, PKV_ERR_UNKNOWN_SEQ, PKV_ERR_SEQ_EXISTS, \
-    PKV_ERR_CUDA, PKV_ERR_DEVICE = range(7)
+    PKV_ERR_CUDA, PKV_ERR_DEVICE, PKV_ERR_SCRATCH_LIMIT = range(8)
 PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = range(4)
 PKV_DEVERR_CONTEXT_LEN, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 PKV_POOL_HOST_ONLY = 0x1
@@ -107,6 +107,9 @@ _sig("pkv_step_destroy", None, _P)
 _sig("pkv_decode_step", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
 _sig("pkv_step_last_launches", ctypes.c_int, _P)
 _sig("pkv_step_profile", _st, _P, ctypes.c_int)
+_sig("paged_decode_attention_static", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int,
+     ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P)
+_sig("paged_decode_static_scratch_bytes", ctypes.c_size_t)
 _sig("pkv_step_profile_read", _st, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float),
      ctypes.c_int, ctypes.POINTER(ctypes.c_int))
 
@@ -117,6 +120,7 @@ EXPORTED = [
     "paged_decode_attention_ex", "paged_decode_workspace_bytes", "paged_decode_workspace_bytes_ex",
     "pkv_device_error", "pkv_status_str", "pkv_step_create", "pkv_step_destroy", "pkv_decode_step",
     "pkv_step_last_launches", "pkv_step_profile", "pkv_step_profile_read",
+    "paged_decode_attention_static", "paged_decode_static_scratch_bytes",
 ]
 
 
@@ -465,3 +469,24 @@ def pkv_step_profile_read(step: Step, cap: int):
                                       b.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), int(cap),
                                       ctypes.byref(n)), "pkv_step_profile_read")
     return a[: n.value].copy(), b[: n.value].copy()
+
+
+def paged_decode_static_scratch_bytes() -> int:
+    return int(_lib.paged_decode_static_scratch_bytes())
+
+
+def paged_decode_attention_static(pool: Pool, q, block_tables, context_lens, scale: float,
+                                  out=None, partition_tokens: int = 0, stream=None):
+    """paged_decode_attention without a workspace: for callers that cannot
+    allocate device memory (the split scratch is the library's static device
+    array).  ``out`` should be preallocated by such callers; if None it is
+    allocated here for convenience."""
+    import torch
+    B, H_q, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.paged_decode_attention_static(
+        pool.handle, _dev_ptr(q), torch_dtype_code(q.dtype), _dev_ptr(block_tables),
+        int(block_tables.shape[1]), _dev_ptr(context_lens), B, H_q, float(scale), _dev_ptr(out),
+        int(partition_tokens), _stream_ptr(stream)), "paged_decode_attention_static")
+    return out

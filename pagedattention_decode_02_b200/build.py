@@ -30,6 +30,7 @@ SOURCES = [
     "decode_simt.cu",
     "decode_tc.cu",
     "api.cu",
+    "no_alloc.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

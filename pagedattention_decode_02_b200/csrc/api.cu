@@ -76,6 +76,7 @@ const char* pkv_status_str(pkv_status s) {
         case PKV_ERR_SEQ_EXISTS: return "SEQ_EXISTS";
         case PKV_ERR_CUDA: return "CUDA";
         case PKV_ERR_DEVICE: return "DEVICE";
+        case PKV_ERR_SCRATCH_LIMIT: return "SCRATCH_LIMIT";
         default: return "UNKNOWN_STATUS";
     }
 }
