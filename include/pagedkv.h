@@ -256,9 +256,13 @@ pkv_status paged_decode_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_d
 size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, int max_blocks);
 
 /* Kernel selection for paged_decode_attention_ex. */
-#define PKV_KERNEL_AUTO 0
-#define PKV_KERNEL_SIMT 1          /* CUDA-core dot products (any head grouping, any dtype) */
-#define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads (F16/BF16, G > 1) */
+#define PKV_KERNEL_AUTO 0          /* TENSOR when supported, else SIMT */
+#define PKV_KERNEL_SIMT 1          /* CUDA-core dot products: SIMT_TMA when supported, else SIMT_BULK */
+#define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads: F16/BF16 pools with
+                                      head_dim 64 or 128, power-of-two block size, 1 < G <= 128 */
+#define PKV_KERNEL_SIMT_BULK 3     /* CUDA-core, 1-D bulk copies per block run (any shape) */
+#define PKV_KERNEL_SIMT_TMA 4      /* CUDA-core, swizzled 2-D TMA boxes, one query head per CTA:
+                                      rows of 128/256/512 bytes, power-of-two block size */
 
 /* paged_decode_attention_ex - paged_decode_attention with explicit choices:
  *   partition_tokens: 0 = automatic, > 0 = tokens per partition (a multiple
@@ -297,8 +301,15 @@ void pkv_step_destroy(pkv_step* step);
  *      on error nothing is launched and the tables are unchanged);
  *   2. host: the batch's block tables and context lengths into pinned staging,
  *      one asynchronous host-to-device copy on `stream`;
- *   3. device: block_copy of the copy-on-write pairs, then kv_append of the B
- *      new rows, then paged decode attention into d_out.
+ *   3. device: copy-on-write of the shared blocks, append of the B new rows,
+ *      then paged decode attention into d_out.
+ *   The device keeps the batch's tables between calls; a round sends only
+ *   what changed (slots, lengths, copy pairs, new table entries) as the
+ *   parameters of one prologue kernel, falling back to a packed host-to-device
+ *   copy of the full tables when that does not fit.  With split contexts the
+ *   decode kernel merges the partitions itself (counters in the runtime's
+ *   workspace, zero between calls) when the tensor-core or swizzled-TMA
+ *   kernel runs.
  *   d_q: device [B][n_q_heads][head_dim]; d_k_new, d_v_new: device
  *   [B][n_kv_heads][head_dim]; d_out: device [B][n_q_heads][head_dim]; all in
  *   q_dtype.  Returns INVALID_ARG if a table would exceed max_blocks (nothing
@@ -312,18 +323,21 @@ pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const 
  *   launched (copy-on-write copy, append, decode, merge). */
 int pkv_step_last_launches(const pkv_step* step);
 
-/* pkv_step_profile - n > 0: later pkv_decode_step calls record CUDA events on
- *   their stream right before the decode kernel, between it and the partition
- *   merge, and after the merge, into a ring of n entries; n == 0 turns this
+/* pkv_step_profile - n > 0: every `every`-th later pkv_decode_step call (the
+ *   first one included) records CUDA events on its stream before the round's
+ *   prologue (copy/append), before the decode kernel, between it and the
+ *   partition merge kernel, and after it, into a ring of n entries; those
+ *   rounds run their kernels strictly one after the other.  n == 0 turns this
  *   off.  Errors: INVALID_ARG, CUDA. */
-pkv_status pkv_step_profile(pkv_step* step, int n);
+pkv_status pkv_step_profile(pkv_step* step, int n, int every);
 
-/* pkv_step_profile_read - milliseconds of the decode kernel and of the merge
- *   for the most recent min(calls, n) recorded calls, oldest first, into
- *   decode_ms[] and merge_ms[] (capacity cap); *n_out receives the count.
- *   Waits for those events.  Errors: INVALID_ARG (cap too small), CUDA. */
-pkv_status pkv_step_profile_read(pkv_step* step, float* decode_ms, float* merge_ms, int cap,
-                                 int* n_out);
+/* pkv_step_profile_read - milliseconds of the prologue, of the decode kernel
+ *   and of the merge (~0 when the decode kernel merged in-kernel) for the most
+ *   recent min(recorded rounds, n) rounds, oldest first (capacity cap each);
+ *   *n_out receives the count.  Waits for those events.
+ *   Errors: INVALID_ARG (cap too small), CUDA. */
+pkv_status pkv_step_profile_read(pkv_step* step, float* prologue_ms, float* decode_ms,
+                                 float* merge_ms, int cap, int* n_out);
 
 /* paged_decode_attention_static - paged_decode_attention for callers that
  *   cannot allocate device memory: processes whose GPU memory is already held

@@ -35,7 +35,7 @@ PKV_OK, PKV_ERR_INVALID_ARG, PKV_ERR_NO_BLOCKS, PKV_ERR_UNKNOWN_SEQ, PKV_ERR_SEQ
 PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = range(4)
 PKV_DEVERR_CONTEXT_LEN, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 PKV_POOL_HOST_ONLY = 0x1
-PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_TENSOR = 0, 1, 2
+PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_TENSOR, PKV_KERNEL_SIMT_BULK, PKV_KERNEL_SIMT_TMA = 0, 1, 2, 3, 4
 
 DTYPE_NAMES = {"f32": PKV_F32, "f16": PKV_F16, "bf16": PKV_BF16, "fp8": PKV_FP8_E4M3}
 ELEM_BYTES = {PKV_F32: 4, PKV_F16: 2, PKV_BF16: 2, PKV_FP8_E4M3: 1}
@@ -106,12 +106,12 @@ _sig("pkv_step_create", _st, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctype
 _sig("pkv_step_destroy", None, _P)
 _sig("pkv_decode_step", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
 _sig("pkv_step_last_launches", ctypes.c_int, _P)
-_sig("pkv_step_profile", _st, _P, ctypes.c_int)
+_sig("pkv_step_profile", _st, _P, ctypes.c_int, ctypes.c_int)
 _sig("paged_decode_attention_static", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int,
      ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P)
 _sig("paged_decode_static_scratch_bytes", ctypes.c_size_t)
 _sig("pkv_step_profile_read", _st, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float),
-     ctypes.c_int, ctypes.POINTER(ctypes.c_int))
+     ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int))
 
 EXPORTED = [
     "kv_pool_create", "kv_pool_destroy", "kv_pool_get_info", "bt_reset", "bt_alloc", "bt_append",
@@ -431,6 +431,15 @@ class Step:
     def last_launches(self) -> int:
         return int(_lib.pkv_step_last_launches(self.handle))
 
+    def run_raw(self, ids: np.ndarray, q_ptr: int, k_ptr: int, v_ptr: int, scale: float,
+                out_ptr: int, stream_ptr: int) -> None:
+        """pkv_decode_step with pre-resolved device pointers (int64 ``ids``):
+        the same C call without per-call tensor checks, for tight loops."""
+        st = _lib.pkv_decode_step(self.handle, ids.ctypes.data_as(_I64P), int(ids.size), q_ptr,
+                                  k_ptr, v_ptr, scale, out_ptr, stream_ptr)
+        if st != PKV_OK:
+            raise PagedKVError(st, "pkv_decode_step")
+
 
 def pkv_step_create(pool: Pool, max_batch: int, max_blocks: int, n_q_heads: int, q_dtype,
                     partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO) -> Step:
@@ -456,19 +465,18 @@ def pkv_step_last_launches(step: Step) -> int:
     return step.last_launches
 
 
-def pkv_step_profile(step: Step, n: int) -> None:
-    _check(_lib.pkv_step_profile(step.handle, int(n)), "pkv_step_profile")
+def pkv_step_profile(step: Step, n: int, every: int = 1) -> None:
+    _check(_lib.pkv_step_profile(step.handle, int(n), int(every)), "pkv_step_profile")
 
 
 def pkv_step_profile_read(step: Step, cap: int):
-    """-> (decode_ms [n], merge_ms [n]) numpy float32, oldest first."""
-    a = np.zeros(max(cap, 1), np.float32)
-    b = np.zeros(max(cap, 1), np.float32)
+    """-> (prologue_ms [n], decode_ms [n], merge_ms [n]) numpy float32, oldest first."""
+    bufs = [np.zeros(max(cap, 1), np.float32) for _ in range(3)]
     n = ctypes.c_int()
-    _check(_lib.pkv_step_profile_read(step.handle, a.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
-                                      b.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), int(cap),
+    fp = ctypes.POINTER(ctypes.c_float)
+    _check(_lib.pkv_step_profile_read(step.handle, *(b.ctypes.data_as(fp) for b in bufs), int(cap),
                                       ctypes.byref(n)), "pkv_step_profile_read")
-    return a[: n.value].copy(), b[: n.value].copy()
+    return tuple(b[: n.value].copy() for b in bufs)
 
 
 def paged_decode_static_scratch_bytes() -> int:

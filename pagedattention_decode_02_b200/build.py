@@ -28,6 +28,7 @@ SOURCES = [
     "block_manager.cpp",
     "append.cu",
     "decode_simt.cu",
+    "decode_simt2.cu",
     "decode_tc.cu",
     "api.cu",
     "no_alloc.cu",

@@ -5,6 +5,8 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
+#include <limits>
 
 #include "block_manager.h"
 #include "decode_launch.h"
@@ -42,13 +44,17 @@ bool same_device(const pkv_pool* pool) {
 constexpr int kNoSplitTokens = 512;
 constexpr int kAutoPartition = 512;
 
-int resolve_partition(const pkv_pool* pool, int max_blocks, int requested) {
+// With G query heads per KV head, a partition's partial state is G * (d + 2)
+// floats against partition * 2 * d * elem bytes of K/V, so the automatic
+// partition grows with G (about 1.5 % extra traffic at G = 8, d = 128, bf16).
+int resolve_partition(const pkv_pool* pool, int max_blocks, int requested, int group = 1) {
     const long long max_ctx = (long long)max_blocks * pool->block_size;
     const int whole = (int)(((max_ctx + 15) / 16) * 16);
     if (requested < 0) return whole < 16 ? 16 : whole;
     if (requested > 0) return requested;
-    if (max_ctx <= kNoSplitTokens) return whole < 16 ? 16 : whole;
-    return kAutoPartition;
+    const long long auto_p = (long long)kAutoPartition * ((group + 7) / 8);
+    if (max_ctx <= (group > 8 ? auto_p : kNoSplitTokens)) return whole < 16 ? 16 : whole;
+    return (int)(auto_p < (1 << 30) ? auto_p : (1 << 30));
 }
 
 int parts_for(const pkv_pool* pool, int max_blocks, int part_tokens) {
@@ -264,7 +270,7 @@ pkv_status block_copy(pkv_pool* p, const int32_t* src, const int32_t* dst, int n
 size_t paged_decode_workspace_bytes_ex(const pkv_pool* p, int B, int n_q_heads, int max_blocks,
                                        int partition_tokens) {
     if (!p || B <= 0 || n_q_heads <= 0 || max_blocks <= 0) return 0;
-    const int P = resolve_partition(p, max_blocks, partition_tokens);
+    const int P = resolve_partition(p, max_blocks, partition_tokens, n_q_heads / p->n_kv_heads);
     if (P <= 0 || P % 16) return 0;
     return workspace_for(p, B, n_q_heads, parts_for(p, max_blocks, P));
 }
@@ -283,7 +289,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                  const int32_t* tables, int max_blocks, const int32_t* lens, int B,
                                  int n_q_heads, float scale, void* out, void* ws, size_t ws_bytes,
                                  int partition_tokens, int kernel, void* stream,
-                                 cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end) {
+                                 cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end,
+                                 int* counters = nullptr, bool pdl = false) {
     if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
     if (B == 0) return PKV_OK;
     if (!q || !out || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
@@ -297,21 +304,24 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (partition_tokens != 0 && partition_tokens != -1 &&
         (partition_tokens < 16 || partition_tokens % 16))
         return PKV_ERR_INVALID_ARG;
-    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_TENSOR) return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_SIMT_TMA) return PKV_ERR_INVALID_ARG;
     if ((long long)max_blocks * p->block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
     if (!same_device(p)) return PKV_ERR_INVALID_ARG;
 
     const int G = n_q_heads / p->n_kv_heads;
-    const int P = resolve_partition(p, max_blocks, partition_tokens);
+    const int P = resolve_partition(p, max_blocks, partition_tokens, G);
     const int max_parts = parts_for(p, max_blocks, P);
     const size_t need = workspace_for(p, B, n_q_heads, max_parts);
     if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
     if ((long long)max_parts > 0x7fffffffLL || B > 65535) return PKV_ERR_INVALID_ARG;
 
     const bool tc_ok = pkv::tensor_path_supported(p, q_dtype, G);
+    const bool s2_ok = pkv::simt2_supported(p, G);
     int use = kernel;
     if (use == PKV_KERNEL_AUTO) use = tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT;
+    if (use == PKV_KERNEL_SIMT) use = s2_ok ? PKV_KERNEL_SIMT_TMA : PKV_KERNEL_SIMT_BULK;
     if (use == PKV_KERNEL_TENSOR && !tc_ok) return PKV_ERR_INVALID_ARG;
+    if (use == PKV_KERNEL_SIMT_TMA && !s2_ok) return PKV_ERR_INVALID_ARG;
 
     pkv::DecodeParams dp{};
     dp.q = q;
@@ -335,6 +345,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     dp.ws_acc = need ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                                 ((rows * 2 * sizeof(float) + 255) & ~(size_t)255))
                      : nullptr;
+    dp.counters = need ? counters : nullptr;
+    dp.pdl = pdl ? 1 : 0;
     const float log2e = 1.4426950408889634f;
     dp.q_scale = scale * log2e * p->k_scale;
     dp.v_scale = p->v_scale;
@@ -346,6 +358,9 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (e != cudaSuccess) return PKV_ERR_CUDA;
     if (use == PKV_KERNEL_TENSOR) {
         e = pkv::launch_decode_tensor(dp, p->tmap_k, p->tmap_v, p->dtype, p->head_dim, st, ev_mid);
+    } else if (use == PKV_KERNEL_SIMT_TMA) {
+        e = pkv::launch_decode_simt2(dp, p->tmap_k, p->tmap_v, p->dtype, q_dtype, p->head_dim,
+                                     __builtin_ctz((unsigned)p->block_size), st, ev_mid);
     } else {
         e = pkv::launch_decode_simt(dp, p->dtype, q_dtype, p->head_dim, pkv::simt_heads_per_cta(G),
                                     st, ev_mid);
@@ -408,17 +423,45 @@ struct pkv_step {
     size_t ws_bytes = 0;
     int max_parts = 1;
     int last_launches = 0;
-    // profiling: event triples (before decode, between decode and merge,
-    // after merge) in a ring of prof_n entries
+    // what the device tables (d_stage + 4 * max_batch) hold, row by row
+    std::vector<int64_t> row_seq;
+    std::vector<uint64_t> row_epoch;
+    std::vector<int32_t> row_nb;
+    std::vector<int32_t> mirror;      // [max_batch][max_blocks]
+    // host scratch of one round
+    std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_upd_idx, h_upd_val;
+    pkv::StepArgs args;
+    long long fast_rounds = 0, slow_rounds = 0;
+    int* d_counters = nullptr;        // [max_batch][n_q_heads], zero between launches
+    // profiling: every prof_every-th round records four events (before the
+    // prologue, before the decode kernel, between it and the merge, after the
+    // merge) into a ring of prof_n entries
     int prof_n = 0;
+    int prof_every = 1;
     long long prof_count = 0;
+    long long round = 0;
     cudaEvent_t* prof_ev = nullptr;
 };
 
 namespace {
+// the tensor-core and swizzled-TMA CUDA-core kernels merge split partitions
+// themselves when the step runtime hands them its zeroed counters
+bool decode_merges_in_kernel(const pkv_pool* pool, const pkv_step* s) {
+    const int G = s->n_q_heads / pool->n_kv_heads;
+    const bool tc = pkv::tensor_path_supported(pool, s->q_dtype, G);
+    const bool s2 = pkv::simt2_supported(pool, G);
+    switch (s->kernel) {
+        case PKV_KERNEL_AUTO: return tc || s2;
+        case PKV_KERNEL_SIMT: return s2;
+        case PKV_KERNEL_TENSOR: return tc;
+        case PKV_KERNEL_SIMT_TMA: return s2;
+        default: return false;
+    }
+}
+
 void prof_free(pkv_step* s) {
     if (s->prof_ev) {
-        for (int i = 0; i < 3 * s->prof_n; ++i)
+        for (int i = 0; i < 4 * s->prof_n; ++i)
             if (s->prof_ev[i]) cudaEventDestroy(s->prof_ev[i]);
         delete[] s->prof_ev;
     }
@@ -438,6 +481,7 @@ void step_free(pkv_step* s) {
     }
     if (s->d_stage) cudaFree(s->d_stage);
     if (s->d_ws) cudaFree(s->d_ws);
+    if (s->d_counters) cudaFree(s->d_counters);
     delete s;
 }
 }  // namespace
@@ -455,7 +499,7 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_
     if (partition_tokens != 0 && partition_tokens != -1 &&
         (partition_tokens < 16 || partition_tokens % 16))
         return PKV_ERR_INVALID_ARG;
-    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_TENSOR) return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_SIMT_TMA) return PKV_ERR_INVALID_ARG;
     if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
     pkv_step* s = new (std::nothrow) pkv_step();
     if (!s) return PKV_ERR_INVALID_ARG;
@@ -474,10 +518,20 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_
         ok &= ok && cudaEventCreateWithFlags(&s->ev[i], cudaEventDisableTiming) == cudaSuccess;
     }
     ok &= ok && cudaMalloc(&s->d_stage, bytes) == cudaSuccess;
-    const int P = resolve_partition(pool, max_blocks, partition_tokens);
+    s->row_seq.assign(max_batch, std::numeric_limits<int64_t>::min());
+    s->row_epoch.assign(max_batch, 0);
+    s->row_nb.assign(max_batch, 0);
+    s->mirror.assign((size_t)max_batch * max_blocks, -1);
+    const int P = resolve_partition(pool, max_blocks, partition_tokens,
+                                    n_q_heads / pool->n_kv_heads);
     s->max_parts = parts_for(pool, max_blocks, P);
     s->ws_bytes = workspace_for(pool, max_batch, n_q_heads, s->max_parts);
     if (ok && s->ws_bytes) ok &= cudaMalloc(&s->d_ws, s->ws_bytes) == cudaSuccess;
+    if (ok && s->ws_bytes) {
+        const size_t cb = (size_t)max_batch * n_q_heads * sizeof(int);
+        ok &= cudaMalloc(&s->d_counters, cb) == cudaSuccess;
+        ok &= ok && cudaMemset(s->d_counters, 0, cb) == cudaSuccess;
+    }
     if (!ok) {
         step_free(s);
         return PKV_ERR_CUDA;
@@ -499,6 +553,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     s->last_launches = 0;
     if (B == 0) return PKV_OK;
     if (!seq_ids || !q || !k_new || !v_new || !out) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_INVALID_ARG;
     pkv_pool* pool = s->pool;
     if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
     // every table must still fit after the append: checked before anything changes
@@ -509,45 +564,133 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         if (nb > s->max_blocks) return PKV_ERR_INVALID_ARG;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int r = s->ring;
-    if (s->pending[r] && cudaEventSynchronize(s->ev[r]) != cudaSuccess) return PKV_ERR_CUDA;
-    s->pending[r] = false;
-    int32_t* h = s->h_stage[r];
     const int mb = s->max_batch;
+    const int bs = pool->block_size;
     int n_cow = 0;
-    pkv_status ps = pool->bm.append_batch(seq_ids, B, h, h + mb, h + 2 * mb, &n_cow);
+    s->h_slots.resize(B);
+    s->h_src.resize(B);
+    s->h_dst.resize(B);
+    pkv_status ps = pool->bm.append_batch(seq_ids, B, s->h_slots.data(), s->h_src.data(),
+                                          s->h_dst.data(), &n_cow);
     if (ps != PKV_OK) return ps;
-    ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, h + 4 * mb, h + 3 * mb, nullptr);
-    if (ps != PKV_OK) return ps;   // cannot happen after the checks above
-    const size_t ints = (size_t)4 * mb + (size_t)B * s->max_blocks;
-    if (cudaMemcpyAsync(s->d_stage, h, ints * sizeof(int32_t), cudaMemcpyHostToDevice, st) !=
-            cudaSuccess ||
-        cudaEventRecord(s->ev[r], st) != cudaSuccess)
-        return PKV_ERR_CUDA;
-    s->pending[r] = true;
-    s->ring = (r + 1) % pkv_step::kRing;
+    // rows of each shared block to copy: the fill before the write, i.e. the
+    // offset of the slot that the copying sequence writes into the copy
+    s->h_rows.resize(n_cow);
+    for (int j = 0; j < n_cow; ++j) {
+        s->h_rows[j] = bs;
+        for (int i = 0; i < B; ++i)
+            if (s->h_slots[i] / bs == s->h_dst[j]) {
+                s->h_rows[j] = s->h_slots[i] % bs;
+                break;
+            }
+    }
+    // table entries that differ from what the device holds
+    s->h_upd_idx.clear();
+    s->h_upd_val.clear();
+    const size_t limit = (size_t)pkv::kStepArgInts;
+    bool fits = (size_t)2 * B + 3 * (size_t)n_cow <= limit;
+    for (int i = 0; i < B && fits; ++i) {
+        const pkv::Sequence* sq = pool->bm.find(seq_ids[i]);
+        const int nb = (int)sq->blocks.size();
+        const bool same = s->row_seq[i] == seq_ids[i] && s->row_epoch[i] == sq->epoch;
+        const int from = same ? (s->row_nb[i] > 0 ? s->row_nb[i] - 1 : 0) : 0;
+        const int32_t* m = s->mirror.data() + (size_t)i * s->max_blocks;
+        for (int e = from; e < nb; ++e) {
+            if (same && e < s->row_nb[i] && m[e] == sq->blocks[e]) continue;
+            s->h_upd_idx.push_back(i * s->max_blocks + e);
+            s->h_upd_val.push_back(sq->blocks[e]);
+        }
+        fits = 2 * B + 3 * (size_t)n_cow + 2 * s->h_upd_idx.size() <= limit;
+    }
     int launches = 0;
-    if (n_cow > 0) {
-        ps = block_copy(pool, s->d_stage + mb, s->d_stage + 2 * mb, n_cow, stream);
+    int32_t* d_lens = s->d_stage + 3 * mb;
+    int32_t* d_tables = s->d_stage + 4 * mb;
+    cudaEvent_t e_pre = nullptr, e0 = nullptr, e1 = nullptr, e2 = nullptr;
+    const bool profiled = s->prof_n > 0 && (s->round % s->prof_every) == 0;
+    ++s->round;
+    if (profiled) {
+        const int i = (int)(s->prof_count % s->prof_n);
+        e_pre = s->prof_ev[4 * i];
+        e0 = s->prof_ev[4 * i + 1];
+        e1 = s->prof_ev[4 * i + 2];
+        e2 = s->prof_ev[4 * i + 3];
+        if (cudaEventRecord(e_pre, st) != cudaSuccess) return PKV_ERR_CUDA;
+    }
+    if (fits) {
+        // fast path: everything of this round travels as kernel parameters
+        pkv::StepArgs& a = s->args;
+        a.B = B;
+        a.n_cow = n_cow;
+        a.n_upd = (int32_t)s->h_upd_idx.size();
+        a.table_cap = mb * s->max_blocks;
+        int32_t* d = a.data;
+        for (int i = 0; i < B; ++i) d[i] = s->h_slots[i];
+        d += B;
+        for (int i = 0; i < B; ++i) d[i] = (int32_t)pool->bm.find(seq_ids[i])->length;
+        d += B;
+        for (int j = 0; j < n_cow; ++j) d[j] = s->h_src[j];
+        d += n_cow;
+        for (int j = 0; j < n_cow; ++j) d[j] = s->h_dst[j];
+        d += n_cow;
+        for (int j = 0; j < n_cow; ++j) d[j] = s->h_rows[j];
+        d += n_cow;
+        for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_idx[u];
+        d += a.n_upd;
+        for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_val[u];
+        cudaError_t e = pkv::launch_step_prologue(
+            a, pool->k, pool->v, k_new, v_new, s->q_dtype, pool->dtype, d_tables, d_lens,
+            pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale, pool->v_scale,
+            pool->d_err, st);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
+        launches = 1;
+        for (size_t u = 0; u < s->h_upd_idx.size(); ++u) s->mirror[s->h_upd_idx[u]] = s->h_upd_val[u];
+        ++s->fast_rounds;
+    } else {
+        // large rounds: one packed upload of slots, copy pairs, lengths and the
+        // batch's full tables from pinned staging, then copy and append
+        const int r = s->ring;
+        if (s->pending[r] && cudaEventSynchronize(s->ev[r]) != cudaSuccess) return PKV_ERR_CUDA;
+        s->pending[r] = false;
+        int32_t* h = s->h_stage[r];
+        for (int i = 0; i < B; ++i) h[i] = s->h_slots[i];
+        for (int j = 0; j < n_cow; ++j) {
+            h[mb + j] = s->h_src[j];
+            h[2 * mb + j] = s->h_dst[j];
+        }
+        ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, h + 4 * mb, h + 3 * mb, nullptr);
+        if (ps != PKV_OK) return ps;   // cannot happen after the checks above
+        const size_t ints = (size_t)4 * mb + (size_t)B * s->max_blocks;
+        if (cudaMemcpyAsync(s->d_stage, h, ints * sizeof(int32_t), cudaMemcpyHostToDevice, st) !=
+                cudaSuccess ||
+            cudaEventRecord(s->ev[r], st) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        s->pending[r] = true;
+        s->ring = (r + 1) % pkv_step::kRing;
+        if (n_cow > 0) {
+            ps = block_copy(pool, s->d_stage + mb, s->d_stage + 2 * mb, n_cow, stream);
+            if (ps != PKV_OK) return ps;
+            ++launches;
+        }
+        ps = kv_append(pool, s->d_stage, B, k_new, v_new, s->q_dtype, stream);
         if (ps != PKV_OK) return ps;
         ++launches;
+        std::copy(h + 4 * mb, h + 4 * mb + (size_t)B * s->max_blocks, s->mirror.begin());
+        ++s->slow_rounds;
     }
-    ps = kv_append(pool, s->d_stage, B, k_new, v_new, s->q_dtype, stream);
-    if (ps != PKV_OK) return ps;
-    ++launches;
-    cudaEvent_t e0 = nullptr, e1 = nullptr, e2 = nullptr;
-    if (s->prof_n > 0) {
-        const int i = (int)(s->prof_count % s->prof_n);
-        e0 = s->prof_ev[3 * i];
-        e1 = s->prof_ev[3 * i + 1];
-        e2 = s->prof_ev[3 * i + 2];
+    for (int i = 0; i < B; ++i) {
+        const pkv::Sequence* sq = pool->bm.find(seq_ids[i]);
+        s->row_seq[i] = seq_ids[i];
+        s->row_epoch[i] = sq->epoch;
+        s->row_nb[i] = (int32_t)sq->blocks.size();
     }
-    ps = decode_attention_impl(pool, q, s->q_dtype, s->d_stage + 4 * mb, s->max_blocks,
-                               s->d_stage + 3 * mb, B, s->n_q_heads, scale, out, s->d_ws,
-                               s->ws_bytes, s->partition_tokens, s->kernel, stream, e0, e1, e2);
+    // the decode kernel starts its launch while the prologue runs (programmatic
+    // dependent launch), except in profiled rounds whose events sit between
+    ps = decode_attention_impl(pool, q, s->q_dtype, d_tables, s->max_blocks, d_lens, B,
+                               s->n_q_heads, scale, out, s->d_ws, s->ws_bytes, s->partition_tokens,
+                               s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled);
     if (ps != PKV_OK) return ps;
-    if (s->prof_n > 0) ++s->prof_count;
-    launches += 1 + (s->max_parts > 1 ? 1 : 0);
+    if (profiled) ++s->prof_count;
+    launches += 1 + (s->max_parts > 1 && !decode_merges_in_kernel(pool, s) ? 1 : 0);
     s->last_launches = launches;
     return PKV_OK;
 }
@@ -556,14 +699,16 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
 
 extern "C" {
 
-pkv_status pkv_step_profile(pkv_step* s, int n) {
-    if (!s || n < 0) return PKV_ERR_INVALID_ARG;
+pkv_status pkv_step_profile(pkv_step* s, int n, int every) {
+    if (!s || n < 0 || every < 1) return PKV_ERR_INVALID_ARG;
     prof_free(s);
     if (n == 0) return PKV_OK;
-    s->prof_ev = new (std::nothrow) cudaEvent_t[3 * (size_t)n]();
+    s->prof_ev = new (std::nothrow) cudaEvent_t[4 * (size_t)n]();
     if (!s->prof_ev) return PKV_ERR_INVALID_ARG;
     s->prof_n = n;
-    for (int i = 0; i < 3 * n; ++i)
+    s->prof_every = every;
+    s->round = 0;
+    for (int i = 0; i < 4 * n; ++i)
         if (cudaEventCreate(&s->prof_ev[i]) != cudaSuccess) {
             prof_free(s);
             return PKV_ERR_CUDA;
@@ -571,21 +716,25 @@ pkv_status pkv_step_profile(pkv_step* s, int n) {
     return PKV_OK;
 }
 
-pkv_status pkv_step_profile_read(pkv_step* s, float* decode_ms, float* merge_ms, int cap,
-                                 int* n_out) {
+pkv_status pkv_step_profile_read(pkv_step* s, float* prologue_ms, float* decode_ms,
+                                 float* merge_ms, int cap, int* n_out) {
     if (!s || !n_out || cap < 0) return PKV_ERR_INVALID_ARG;
     const int have = (int)(s->prof_count < s->prof_n ? s->prof_count : s->prof_n);
-    if (cap < have || (have > 0 && (!decode_ms || !merge_ms))) return PKV_ERR_INVALID_ARG;
+    if (cap < have || (have > 0 && (!prologue_ms || !decode_ms || !merge_ms)))
+        return PKV_ERR_INVALID_ARG;
     const long long first = s->prof_count - have;
     for (int j = 0; j < have; ++j) {
         const int i = (int)((first + j) % s->prof_n);
-        if (cudaEventSynchronize(s->prof_ev[3 * i + 2]) != cudaSuccess) return PKV_ERR_CUDA;
-        float a = 0.f, b = 0.f;
-        if (cudaEventElapsedTime(&a, s->prof_ev[3 * i], s->prof_ev[3 * i + 1]) != cudaSuccess ||
-            cudaEventElapsedTime(&b, s->prof_ev[3 * i + 1], s->prof_ev[3 * i + 2]) != cudaSuccess)
+        cudaEvent_t* ev = s->prof_ev + 4 * i;
+        if (cudaEventSynchronize(ev[3]) != cudaSuccess) return PKV_ERR_CUDA;
+        float a = 0.f, b = 0.f, c = 0.f;
+        if (cudaEventElapsedTime(&a, ev[0], ev[1]) != cudaSuccess ||
+            cudaEventElapsedTime(&b, ev[1], ev[2]) != cudaSuccess ||
+            cudaEventElapsedTime(&c, ev[2], ev[3]) != cudaSuccess)
             return PKV_ERR_CUDA;
-        decode_ms[j] = a;
-        merge_ms[j] = b;
+        prologue_ms[j] = a;
+        decode_ms[j] = b;
+        merge_ms[j] = c;
     }
     *n_out = have;
     return PKV_OK;

@@ -31,6 +31,44 @@ __device__ __forceinline__ void load16(const IN* src, float* f) {
     }
 }
 
+// One 16-byte chunk of one destination row.  `which` 0 = K, 1 = V; `t` the
+// token, `h` the KV head, `ch` the chunk of the row.  FP8 pools: 16 input
+// values -> x / scale (IEEE division) -> e4m3, round to nearest even,
+// saturating.
+template <typename IN>
+__device__ __forceinline__ void append_chunk_fp8(uint8_t* k_pool, uint8_t* v_pool, const IN* k,
+                                                 const IN* v, int which, int t, int h, int ch,
+                                                 int slot, int H, int D, int bs, float k_scale,
+                                                 float v_scale) {
+    const IN* src = (which ? v : k) + ((long long)t * H + h) * D + ch * 16;
+    const float scale = which ? v_scale : k_scale;
+    float f[16];
+    load16<IN>(src, f);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float2 a = make_float2(__fdiv_rn(f[4 * j], scale), __fdiv_rn(f[4 * j + 1], scale));
+        float2 b = make_float2(__fdiv_rn(f[4 * j + 2], scale), __fdiv_rn(f[4 * j + 3], scale));
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
+        w[j] = (lo & 0xFFFFu) | (hi << 16);
+    }
+    const long long b = slot / bs, off = slot % bs;
+    uint8_t* dst = (which ? v_pool : k_pool) + (((b * H + h) * bs + off) * D + ch * 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void append_chunk_copy(uint8_t* k_pool, uint8_t* v_pool,
+                                                  const uint8_t* k, const uint8_t* v, int which,
+                                                  int t, int h, int ch, int slot, int H,
+                                                  int row_bytes, int bs) {
+    const uint4 val = *reinterpret_cast<const uint4*>((which ? v : k) +
+                                                      ((long long)t * H + h) * row_bytes + ch * 16);
+    const long long b = slot / bs, off = slot % bs;
+    uint8_t* dst = (which ? v_pool : k_pool) + ((b * H + h) * bs + off) * row_bytes + ch * 16;
+    *reinterpret_cast<uint4*>(dst) = val;
+}
+
 // one thread = one 16-byte chunk of one destination row (K or V)
 template <typename IN>
 __global__ void kv_append_fp8_kernel(uint8_t* k_pool, uint8_t* v_pool, const int32_t* slots,
@@ -52,22 +90,7 @@ __global__ void kv_append_fp8_kernel(uint8_t* k_pool, uint8_t* v_pool, const int
             if (which == 0 && h == 0 && ch == 0) report_error(err, PKV_DEVERR_SLOT);
             continue;
         }
-        const IN* src = (which ? v : k) + ((long long)t * H + h) * D + ch * 16;
-        const float scale = which ? v_scale : k_scale;
-        float f[16];
-        load16<IN>(src, f);
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float2 a = make_float2(__fdiv_rn(f[4 * j], scale), __fdiv_rn(f[4 * j + 1], scale));
-            float2 b = make_float2(__fdiv_rn(f[4 * j + 2], scale), __fdiv_rn(f[4 * j + 3], scale));
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
-            w[j] = (lo & 0xFFFFu) | (hi << 16);
-        }
-        const long long b = slot / bs, off = slot % bs;
-        uint8_t* dst = (which ? v_pool : k_pool) + (((b * H + h) * bs + off) * D + ch * 16);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        append_chunk_fp8<IN>(k_pool, v_pool, k, v, which, t, h, ch, slot, H, D, bs, k_scale, v_scale);
     }
 }
 
@@ -91,11 +114,82 @@ __global__ void kv_append_copy_kernel(uint8_t* k_pool, uint8_t* v_pool, const in
             if (which == 0 && h == 0 && ch == 0) report_error(err, PKV_DEVERR_SLOT);
             continue;
         }
-        const uint4 val = *reinterpret_cast<const uint4*>((which ? v : k) +
-                                                          ((long long)t * H + h) * row_bytes + ch * 16);
-        const long long b = slot / bs, off = slot % bs;
-        uint8_t* dst = (which ? v_pool : k_pool) + ((b * H + h) * bs + off) * row_bytes + ch * 16;
-        *reinterpret_cast<uint4*>(dst) = val;
+        append_chunk_copy(k_pool, v_pool, k, v, which, t, h, ch, slot, H, row_bytes, bs);
+    }
+}
+
+// The decode round's prologue (see StepArgs).  blockIdx.y == 0: lengths,
+// table updates and the appends; blockIdx.y == 1 + j: copy-on-write pair j,
+// rows [0, cow_rows[j]) of every KV head's tile, K and V.  The copied rows
+// and the appended row (row cow_rows[j] of the new block) are disjoint, and
+// no append writes a row below the fill of a shared block, so the two kinds
+// of work need no ordering inside the launch.
+template <typename IN, bool FP8>
+__global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t* k_pool,
+                                     uint8_t* v_pool, const IN* k, const IN* v, int32_t* tables,
+                                     int32_t* lens, int H, int D, int bs, int num_blocks,
+                                     float k_scale, float v_scale, uint32_t* err) {
+    allow_dependent_launch();   // the decode kernel may start its launch now
+    const int B = a.B;
+    const int32_t* slots = a.data;
+    const int32_t* lens_in = a.data + B;
+    const int32_t* cow_src = a.data + 2 * B;
+    const int32_t* cow_dst = cow_src + a.n_cow;
+    const int32_t* cow_rows = cow_dst + a.n_cow;
+    const int32_t* upd_idx = cow_rows + a.n_cow;
+    const int32_t* upd_val = upd_idx + a.n_upd;
+    const int eb = FP8 ? 1 : (int)sizeof(IN);
+    const int row_bytes = D * eb;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long first = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (blockIdx.y == 0) {
+        for (long long i = first; i < B; i += stride) lens[i] = lens_in[i];
+        for (long long u = first; u < a.n_upd; u += stride) {
+            const int idx = upd_idx[u];
+            if (idx >= 0 && idx < a.table_cap) tables[idx] = upd_val[u];
+        }
+        const int chunks = FP8 ? D / 16 : row_bytes / 16;
+        const long long per_tok = (long long)H * chunks;
+        const long long total = 2LL * B * per_tok;
+        for (long long i = first; i < total; i += stride) {
+            const int which = (int)(i / (B * per_tok));
+            const long long r = i - which * (B * per_tok);
+            const int t = (int)(r / per_tok);
+            const int h = (int)((r / chunks) % H);
+            const int ch = (int)(r % chunks);
+            const int slot = slots[t];
+            if (slot < 0) continue;
+            if ((long long)slot >= (long long)num_blocks * bs) {
+                if (which == 0 && h == 0 && ch == 0) report_error(err, PKV_DEVERR_SLOT);
+                continue;
+            }
+            if constexpr (FP8)
+                append_chunk_fp8<IN>(k_pool, v_pool, k, v, which, t, h, ch, slot, H, D, bs,
+                                     k_scale, v_scale);
+            else
+                append_chunk_copy(k_pool, v_pool, reinterpret_cast<const uint8_t*>(k),
+                                  reinterpret_cast<const uint8_t*>(v), which, t, h, ch, slot, H,
+                                  row_bytes, bs);
+        }
+        return;
+    }
+    const int j = blockIdx.y - 1;
+    const int s = cow_src[j], d = cow_dst[j], rows = cow_rows[j];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || rows < 0 || rows > bs) {
+        if (first == 0) report_error(err, PKV_DEVERR_BLOCK_ID);
+        return;
+    }
+    const long long tile = (long long)bs * row_bytes;           // one (block, head) tile
+    const long long per_head = (long long)rows * row_bytes / 16; // chunks copied per tile
+    const long long total = 2LL * H * per_head;
+    for (long long i = first; i < total; i += stride) {
+        const int which = (int)(i / (H * per_head));
+        const long long r = i - which * (H * per_head);
+        const int h = (int)(r / per_head);
+        const long long c = r % per_head;
+        uint8_t* pool = which ? v_pool : k_pool;
+        const uint4 val = reinterpret_cast<const uint4*>(pool + ((long long)s * H + h) * tile)[c];
+        reinterpret_cast<uint4*>(pool + ((long long)d * H + h) * tile)[c] = val;
     }
 }
 
@@ -177,6 +271,57 @@ cudaError_t launch_block_copy(uint8_t* k_pool, uint8_t* v_pool, const int32_t* s
     if (gy > 65535) gy = 65535;
     block_copy_kernel<<<dim3(n_pairs, (unsigned)gy), kThreads, 0, st>>>(k_pool, v_pool, src, dst,
                                                                         block_bytes, num_blocks, err);
+    return cudaGetLastError();
+}
+
+}  // namespace pkv
+
+namespace pkv {
+
+cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
+                                 const void* k, const void* v, int in_dtype, int kv_dtype,
+                                 int32_t* tables, int32_t* lens, int H, int D, int bs,
+                                 int num_blocks, float k_scale, float v_scale, uint32_t* err,
+                                 cudaStream_t st) {
+    constexpr int kThreads = 256;
+    const int eb = kv_dtype == PKV_F32 ? 4 : kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
+    const int chunks_per_row = kv_dtype == PKV_FP8_E4M3 ? D / 16 : D * eb / 16;
+    const long long append_items = 2LL * a.B * H * chunks_per_row;
+    const long long copy_items = 2LL * H * bs * D * eb / 16;
+    long long items = append_items > copy_items ? append_items : copy_items;
+    long long gx = (items + kThreads - 1) / kThreads;
+    if (gx > 148 * 4) gx = 148 * 4;
+    if (gx < 1) gx = 1;
+    const dim3 grid((unsigned)gx, 1 + a.n_cow);
+    if (kv_dtype == PKV_FP8_E4M3) {
+        switch (in_dtype) {
+            case PKV_F32:
+                step_prologue_kernel<float, true><<<grid, kThreads, 0, st>>>(
+                    a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, H, D, bs,
+                    num_blocks, k_scale, v_scale, err);
+                break;
+            case PKV_F16:
+                step_prologue_kernel<__half, true><<<grid, kThreads, 0, st>>>(
+                    a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, H, D, bs,
+                    num_blocks, k_scale, v_scale, err);
+                break;
+            case PKV_BF16:
+                step_prologue_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, st>>>(
+                    a, k_pool, v_pool, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, tables,
+                    lens, H, D, bs, num_blocks, k_scale, v_scale, err);
+                break;
+            default:
+                return cudaErrorInvalidValue;
+        }
+    } else if (kv_dtype == PKV_F32) {
+        step_prologue_kernel<float, false><<<grid, kThreads, 0, st>>>(
+            a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, H, D, bs,
+            num_blocks, k_scale, v_scale, err);
+    } else {
+        step_prologue_kernel<__half, false><<<grid, kThreads, 0, st>>>(
+            a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, H, D, bs,
+            num_blocks, k_scale, v_scale, err);
+    }
     return cudaGetLastError();
 }
 

@@ -63,6 +63,7 @@ pkv_status BlockManager::alloc(int64_t seq, int n_tokens, int32_t* slots) {
     s.blocks.reserve((size_t)need);
     for (int64_t i = 0; i < need; ++i) s.blocks.push_back(pop_front());
     s.length = n_tokens;
+    s.epoch = next_epoch_++;
     for (int t = 0; t < n_tokens; ++t)
         slots[t] = s.blocks[t / block_size_] * block_size_ + t % block_size_;
     seqs_.emplace(seq, std::move(s));
@@ -156,6 +157,7 @@ pkv_status BlockManager::fork(int64_t parent, int64_t child) {
     if (it == seqs_.end()) return PKV_ERR_UNKNOWN_SEQ;
     if (seqs_.count(child)) return PKV_ERR_SEQ_EXISTS;
     Sequence c = it->second;  // copy of the table and the length
+    c.epoch = next_epoch_++;
     for (int32_t b : c.blocks) ++ref_[b];
     seqs_.emplace(child, std::move(c));
     return PKV_OK;

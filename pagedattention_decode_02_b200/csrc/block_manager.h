@@ -20,6 +20,8 @@ namespace pkv {
 struct Sequence {
     std::vector<int32_t> blocks;  // logical block i -> physical block id
     int64_t length = 0;           // tokens stored (the fill count is derived)
+    uint64_t epoch = 0;           // unique per admission / fork: between two appends
+                                  // of the same epoch only the last entry changes
 };
 
 class BlockManager {
@@ -41,6 +43,10 @@ class BlockManager {
     pkv_status refcount_of(int32_t block, int32_t* out) const;
     pkv_status free_queue(int32_t* out, int cap, int* n_out) const;
     void stats(pkv_stats* out) const;
+    const Sequence* find(int64_t seq) const {
+        auto it = seqs_.find(seq);
+        return it == seqs_.end() ? nullptr : &it->second;
+    }
 
     int num_blocks() const { return num_blocks_; }
     int block_size() const { return block_size_; }
@@ -68,6 +74,7 @@ class BlockManager {
     std::vector<int32_t> ref_;
     std::unordered_map<int64_t, Sequence> seqs_;
     int64_t cow_count_ = 0;
+    uint64_t next_epoch_ = 1;
 };
 
 }  // namespace pkv

@@ -23,9 +23,38 @@ namespace pkv {
 // Tensor-core decode of grouped heads (F16/BF16 pools with TMA descriptors,
 // 1 < G <= 128) + partition merge.
 bool tensor_path_supported(const pkv_pool* pool, int q_dtype, int group);
+bool pool_has_row_maps(const pkv_pool* pool);
+
+// CUDA-core decode with swizzled TMA staging, one query head per CTA (pools
+// with row tensor maps) + partition merge.
+bool simt2_supported(const pkv_pool* pool, int group);
+cudaError_t launch_decode_simt2(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
+                                int kv_dtype, int q_dtype, int head_dim, int bs_shift,
+                                cudaStream_t st, cudaEvent_t mid = nullptr);
 cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
                                  int kv_dtype, int head_dim, cudaStream_t st,
                                  cudaEvent_t mid = nullptr);
+
+// One decode round's small host-side results, passed by value as kernel
+// parameters (no separate host-to-device copy):
+//   data = slots[B] | lens[B] | cow_src[n_cow] | cow_dst[n_cow] | cow_rows[n_cow]
+//          | upd_idx[n_upd] | upd_val[n_upd]
+// cow_rows[j] = rows of the shared block to copy (the fill before the write);
+// upd_* = changed block-table entries (flat index into [max_batch][max_blocks]).
+constexpr int kStepArgInts = 990;   // the whole parameter block stays under 4 KB
+struct StepArgs {
+    int32_t B, n_cow, n_upd, table_cap;
+    int32_t data[kStepArgInts];
+};
+
+// The round's prologue in one launch: lengths and table updates into the
+// persistent device tables, copy-on-write of the shared rows, append of the
+// B new rows (FP8 pools quantise).
+cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
+                                 const void* k, const void* v, int in_dtype, int kv_dtype,
+                                 int32_t* tables, int32_t* lens, int n_kv_heads, int head_dim,
+                                 int block_size, int num_blocks, float k_scale, float v_scale,
+                                 uint32_t* err, cudaStream_t st);
 
 // Store new rows into their slots (FP8 pools quantise).
 cudaError_t launch_kv_append(uint8_t* k_pool, uint8_t* v_pool, const int32_t* slots, int n_tokens,

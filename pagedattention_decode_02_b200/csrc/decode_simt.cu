@@ -336,29 +336,69 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
     }
 }
 
-// Merge the partitions of one (sequence, head): blockDim.x == D.
+// Merge the partitions of one (sequence, head) per warp, 8 heads per CTA:
+// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.  Lane
+// l holds D/32 consecutive columns; the partitions' (m, l) pairs are read 32
+// at a time, one per lane, and broadcast by shuffles.
+constexpr int kMergeWarps = 8;
+
 template <typename QT, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kMergeWarps * 32)
 merge_kernel(const DecodeParams p) {
-    const int h = blockIdx.x;
+    constexpr int VEC = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x * kMergeWarps + warp;
     const int seq = blockIdx.y;
-    const int d = threadIdx.x;
+    if (h >= p.H_q) return;
     const int c = p.lens[seq];
     if (c < 1 || c > p.max_blocks * p.block_size) return;   // zeroed by the decode kernel
     const int nparts = (c + p.part_tokens - 1) / p.part_tokens;
     if (nparts <= 1) return;                                   // written by the decode kernel
     const size_t row0 = ((size_t)seq * p.H_q + h) * p.max_parts;
     float M = -INFINITY;
-    for (int q = 0; q < nparts; ++q) M = fmaxf(M, p.ws_ml[(row0 + q) * 2]);
-    float L = 0.f, O = 0.f;
-    for (int q = 0; q < nparts && M != -INFINITY; ++q) {
-        const float w = exp2f(p.ws_ml[(row0 + q) * 2] - M);
-        L = fmaf(p.ws_ml[(row0 + q) * 2 + 1], w, L);
-        O = fmaf(p.ws_acc[(row0 + q) * D + d], w, O);
+    for (int q0 = 0; q0 < nparts; q0 += 32) {
+        const float m = q0 + lane < nparts ? p.ws_ml[(row0 + q0 + lane) * 2] : -INFINITY;
+        M = fmaxf(M, m);
     }
-    // every partition skipped (bad block ids everywhere): zero output
-    const float r = L > 0.f ? O / L : 0.f;
-    reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<QT>::from_f(r);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    float acc[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+    if (M != -INFINITY) {
+        for (int q0 = 0; q0 < nparts; q0 += 32) {
+            const int qi = q0 + lane;
+            float w = 0.f, lw = 0.f;
+            if (qi < nparts) {
+                w = exp2f(p.ws_ml[(row0 + qi) * 2] - M);
+                lw = w * p.ws_ml[(row0 + qi) * 2 + 1];
+            }
+            L += lw;
+            const int cnt = min(32, nparts - q0);
+            for (int j = 0; j < cnt; ++j) {
+                const float wj = __shfl_sync(0xffffffffu, w, j);
+                const float* a = p.ws_acc + (row0 + q0 + j) * D + lane * VEC;
+                float f[VEC];
+                if constexpr (VEC == 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(a);
+                    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+                } else if constexpr (VEC == 2) {
+                    const float2 u = *reinterpret_cast<const float2*>(a);
+                    f[0] = u.x; f[1] = u.y;
+                } else {
+                    f[0] = a[0];
+                }
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wj, f[v], acc[v]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    }
+    QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)seq * p.H_q + h) * D + lane * VEC;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) out[v] = Elem<QT>::from_f(L > 0.f ? acc[v] / L : 0.f);
 }
 
 template <typename KV, typename QT, int D, int HPC>
@@ -367,15 +407,16 @@ cudaError_t launch_simt_t(const DecodeParams& p, cudaStream_t st, cudaEvent_t mi
     const int table_entries = p.part_tokens / p.block_size + 2;
     const int smem = L::bytes(table_entries);
     auto kern = decode_simt_kernel<KV, QT, D, HPC>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static unsigned long long attr_done = 0;
+    cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
     dim3 grid(p.max_parts, p.H_q / HPC, p.B);
     kern<<<grid, kThreads, smem, st>>>(p, table_entries);
     e = cudaGetLastError();
     if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
     if (e != cudaSuccess || p.max_parts <= 1) return e;
-    merge_kernel<QT, D><<<dim3(p.H_q, p.B), D, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_merge(p, Elem<QT>::id, D, st);
 }
 
 template <typename KV, typename QT, int D>
@@ -402,8 +443,8 @@ cudaError_t launch_simt_q(const DecodeParams& p, int D, int hpc, cudaStream_t st
 }  // namespace
 
 cudaError_t launch_merge(const DecodeParams& p, int q_dtype, int D, cudaStream_t st) {
-    const dim3 grid(p.H_q, p.B);
-#define PKV_MERGE(QT, DD) merge_kernel<QT, DD><<<grid, DD, 0, st>>>(p)
+    const dim3 grid((p.H_q + kMergeWarps - 1) / kMergeWarps, p.B);
+#define PKV_MERGE(QT, DD) merge_kernel<QT, DD><<<grid, kMergeWarps * 32, 0, st>>>(p)
     if (q_dtype == PKV_F32) {
         if (D == 32) PKV_MERGE(float, 32); else if (D == 64) PKV_MERGE(float, 64); else PKV_MERGE(float, 128);
     } else if (q_dtype == PKV_F16) {

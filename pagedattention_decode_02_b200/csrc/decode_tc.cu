@@ -12,7 +12,7 @@
 //
 // Staging: the pool is viewed by two TMA tensor maps (K and V) as a 2-D
 // tensor [num_blocks * H_kv * bs rows][d] with 128-byte swizzle; one stage is
-// a 16-row box per 64-column half (or two 8-row boxes when bs == 8), so each
+// min(bs, 16)-row boxes per 64-column half (bs a power of two), so each
 // 8 x 16-byte ldmatrix read hits 8 different bank groups.  Loads are plain
 // (no multicast) from this GPU's own memory.
 //
@@ -36,7 +36,6 @@ namespace pkv {
 namespace {
 
 constexpr int kStageTokens = 16;
-constexpr int kStages = 3;
 
 template <typename T>
 struct MmaType;
@@ -108,17 +107,18 @@ struct TcSmem {
     static constexpr int kSlot = 2 * kTile;
 };
 
-template <int D, int MT, int TS>
+template <int D, int MT, int TS, int S>
 __host__ __device__ constexpr int tc_union_bytes() {
-    const int tiles = TS * kStages * TcSmem<D>::kSlot;
+    const int tiles = TS * S * TcSmem<D>::kSlot;
     const int comb = MT * TS * 16 * (D + 2) * 4;
     return ((tiles > comb ? tiles : comb) + 15) & ~15;
 }
 
-template <typename T, int D, int MT, int TS>
+template <typename T, int D, int MT, int TS, int S>
 __global__ void __launch_bounds__(MT * TS * 32)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+    constexpr int kStages = S;
     constexpr int NW = MT * TS;
     constexpr int NT = NW * 32;
     constexpr int TILE = TcSmem<D>::kTile;
@@ -134,7 +134,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;                                            // [TS][kStages][SLOT]
     float* comb = reinterpret_cast<float*>(smem);                     // [NW][16][D + 2]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS>());
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS, S>());
     uint64_t* empty = full + TS * kStages;
 
     const int part = blockIdx.x;
@@ -150,6 +150,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int P = p.part_tokens;
     const int h_base = g * G;       // first query head of the group
 
+    __shared__ int last_flag;
+    grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
     const int c = p.lens[seq];
     if (c < 1 || c > p.max_blocks * bs) {
         if (part == 0) {
@@ -191,6 +193,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 reinterpret_cast<T*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<T>::from_f(0.f);
             }
         }
+        if (split && p.counters &&
+            finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
+            merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
+                                     tc_union_bytes<D, MT, TS, S>() / 4);
         return;
     }
 
@@ -284,18 +290,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t kbase = smem_addr(kt);
         const uint32_t vbase = smem_addr(vt);
 
-        // S = Q K^T : two n-tiles of 8 tokens
+        // S = Q K^T : two n-tiles of 8 tokens; even and odd k-steps go to
+        // separate accumulators to halve the dependent mma chain
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
+            float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             const int mi = lane >> 3, r = lane & 7;
             const int tok = (mi >> 1) * 8 + r;
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + swz(tok, 2 * kk + (mi & 1)), b0, b1, b2, b3);
-                MmaType<T>::mma(s[0], qa[kk], b0, b1);
-                MmaType<T>::mma(s[1], qa[kk], b2, b3);
+                if (kk & 1) {
+                    MmaType<T>::mma(s2[0], qa[kk], b0, b1);
+                    MmaType<T>::mma(s2[1], qa[kk], b2, b3);
+                } else {
+                    MmaType<T>::mma(s[0], qa[kk], b0, b1);
+                    MmaType<T>::mma(s[1], qa[kk], b2, b3);
+                }
             }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
         }
         // online softmax over this stage's tokens, per head row (gq, gq + 8)
         float mx[2] = {-INFINITY, -INFINITY};
@@ -334,12 +351,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             pa[2] = MmaType<T>::pack(pr[1][0], pr[1][1]);
             pa[3] = MmaType<T>::pack(pr[1][2], pr[1][3]);
         }
+        // rescale the accumulator only when some row's running max moved
+        // (alpha == 1 exactly otherwise): late in a sequence it rarely does
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-        for (int j = 0; j < DTILES; ++j) {
-            o[j][0] *= alpha[0];
-            o[j][1] *= alpha[0];
-            o[j][2] *= alpha[1];
-            o[j][3] *= alpha[1];
+            for (int j = 0; j < DTILES; ++j) {
+                o[j][0] *= alpha[0];
+                o[j][1] *= alpha[0];
+                o[j][2] *= alpha[1];
+                o[j][3] *= alpha[1];
+            }
         }
         // O += P V : V^T fragments by transposed ldmatrix, two d-tiles per load
         {
@@ -434,26 +455,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 Elem<T>::from_f(L > 0.f ? O / L : 0.f);
         }
     }
+    if (split && p.counters &&
+        finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
+        merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
+                                 tc_union_bytes<D, MT, TS, S>() / 4);
 }
 
-template <int D, int MT, int TS>
+template <int D, int MT, int TS, int S>
 constexpr int tc_smem_bytes() {
-    return 1024 + tc_union_bytes<D, MT, TS>() + 2 * TS * kStages * 8;
+    return 1024 + tc_union_bytes<D, MT, TS, S>() + 2 * TS * S * 8;
 }
 
-template <typename T, int D, int MT, int TS>
+template <typename T, int D, int MT, int TS, int S = (D == 128 ? 2 : 3)>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                         int q_dtype, cudaStream_t st, cudaEvent_t mid) {
-    constexpr int smem = tc_smem_bytes<D, MT, TS>();
-    static_assert(smem <= 227 * 1024, "shared memory budget");
-    auto kern = decode_tc_kernel<T, D, MT, TS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    constexpr int smem = tc_smem_bytes<D, MT, TS, S>();
+    static_assert(smem <= 227 * 1024 - 64, "shared memory budget");
+    auto kern = decode_tc_kernel<T, D, MT, TS, S>;
+    static unsigned long long attr_done = 0;
+    cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
     const dim3 grid(p.max_parts, p.H_kv, p.B);
-    kern<<<grid, MT * TS * 32, smem, st>>>(*tk, *tv, p);
-    e = cudaGetLastError();
+    e = launch_kernel(kern, grid, dim3(MT * TS * 32), smem, st, p.pdl != 0, *tk, *tv, p);
     if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
-    if (e != cudaSuccess || p.max_parts <= 1) return e;
+    if (e != cudaSuccess || p.max_parts <= 1 || p.counters) return e;
     return launch_merge(p, q_dtype, D, st);
 }
 
@@ -462,14 +487,15 @@ cudaError_t launch_tc_d(const DecodeParams& p, const CUtensorMap* tk, const CUte
                         int q_dtype, cudaStream_t st, cudaEvent_t mid) {
     const int mt = (p.G + 15) / 16;
     switch (mt) {
+        // m-tiles of 16 heads x token groups: about 12 warps per CTA
         case 1: return launch_tc_t<T, D, 1, 4>(p, tk, tv, q_dtype, st, mid);
-        case 2: return launch_tc_t<T, D, 2, 2>(p, tk, tv, q_dtype, st, mid);
-        case 3: return launch_tc_t<T, D, 3, 1>(p, tk, tv, q_dtype, st, mid);
-        case 4: return launch_tc_t<T, D, 4, 1>(p, tk, tv, q_dtype, st, mid);
-        case 5: return launch_tc_t<T, D, 5, 1>(p, tk, tv, q_dtype, st, mid);
-        case 6: return launch_tc_t<T, D, 6, 1>(p, tk, tv, q_dtype, st, mid);
-        case 7: return launch_tc_t<T, D, 7, 1>(p, tk, tv, q_dtype, st, mid);
-        case 8: return launch_tc_t<T, D, 8, 1>(p, tk, tv, q_dtype, st, mid);
+        case 2: return launch_tc_t<T, D, 2, 4>(p, tk, tv, q_dtype, st, mid);
+        case 3: return launch_tc_t<T, D, 3, 4>(p, tk, tv, q_dtype, st, mid);
+        case 4: return launch_tc_t<T, D, 4, 3>(p, tk, tv, q_dtype, st, mid);
+        case 5: return launch_tc_t<T, D, 5, 2>(p, tk, tv, q_dtype, st, mid);
+        case 6: return launch_tc_t<T, D, 6, 2>(p, tk, tv, q_dtype, st, mid);
+        case 7: return launch_tc_t<T, D, 7, 2>(p, tk, tv, q_dtype, st, mid);
+        case 8: return launch_tc_t<T, D, 8, 2>(p, tk, tv, q_dtype, st, mid);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -497,12 +523,15 @@ EncodeTiledFn encode_fn() {
 bool encode_pool_map(CUtensorMap* map, void* base, int dtype, int D, long long rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    const int eb = dtype == PKV_F32 ? 4 : dtype == PKV_FP8_E4M3 ? 1 : 2;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * eb};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType t =
-        dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMapDataType t = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if (dtype == PKV_F32) t = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (dtype == PKV_F16) t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (dtype == PKV_BF16) t = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     return fn(map, t, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -510,12 +539,16 @@ bool encode_pool_map(CUtensorMap* map, void* base, int dtype, int D, long long r
 
 }  // namespace
 
+// Row tensor maps of the K and V pools: a 2-D view [num_blocks * H_kv * bs
+// rows][d] with 128-byte inner boxes of min(bs, 16) rows and 128-byte swizzle.
+// Made when a row is 128, 256 or 512 bytes and bs is a power of two (then a
+// 16-token stage is a whole number of boxes, none crossing a block).
 void pool_init_device_extras(pkv_pool* p) {
     p->has_tmaps = false;
-    if ((p->dtype != PKV_F16 && p->dtype != PKV_BF16) || (p->head_dim != 64 && p->head_dim != 128))
-        return;
-    // a 16-token stage must be one 16-row box inside a block, or two 8-row boxes
-    if (p->block_size != 8 && p->block_size % 16 != 0) return;
+    const int eb = p->dtype == PKV_F32 ? 4 : p->dtype == PKV_FP8_E4M3 ? 1 : 2;
+    const int row = p->head_dim * eb;
+    if (row != 128 && row != 256 && row != 512) return;
+    if (p->block_size & (p->block_size - 1)) return;
     const long long rows = (long long)p->num_blocks * p->n_kv_heads * p->block_size;
     if (rows >= (1LL << 31)) return;
     const int box_rows = p->block_size < kStageTokens ? p->block_size : kStageTokens;
@@ -526,8 +559,12 @@ void pool_init_device_extras(pkv_pool* p) {
                                    p->head_dim, rows, box_rows);
 }
 
+bool pool_has_row_maps(const pkv_pool* pool) { return pool->has_tmaps; }
+
 bool tensor_path_supported(const pkv_pool* pool, int q_dtype, int group) {
-    return pool->has_tmaps && q_dtype == pool->dtype && group > 1 && group <= 128;
+    return pool->has_tmaps && (pool->dtype == PKV_F16 || pool->dtype == PKV_BF16) &&
+           q_dtype == pool->dtype && (pool->head_dim == 64 || pool->head_dim == 128) &&
+           group > 1 && group <= 128;
 }
 
 cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,

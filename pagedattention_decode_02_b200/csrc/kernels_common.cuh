@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pagedkv.h"
 
 namespace pkv {
@@ -228,6 +230,17 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
 // ---------------------------------------------------------------------------
 // kernel parameter blocks
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: wait until the preceding kernel of the
+// stream has completed and its writes are visible (a no-op when the kernel
+// was launched without the programmatic-serialization attribute) / allow the
+// next kernel of the stream to start launching
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 struct DecodeParams {
     const void* q;
     void* out;
@@ -237,6 +250,10 @@ struct DecodeParams {
     const int32_t* lens;
     float* ws_ml;    // [B][H_q][max_parts][2]  (running max in log2 units, sum)
     float* ws_acc;   // [B][H_q][max_parts][D]  (unnormalised accumulator)
+    int pdl;         // host side: launch with programmatic stream serialization
+    int* counters;   // [B][H_q] partitions finished, or null: when set, the last
+                     // CTA of a split (sequence, head) merges in the decode
+                     // kernel itself and resets its counter to 0
     uint32_t* err;
     int B, H_q, H_kv, G;
     int max_blocks, block_size, num_blocks;
@@ -247,5 +264,135 @@ struct DecodeParams {
     long long head_stride;   // bytes of one (block, kv head) tile: bs * D * elem
     long long block_stride;  // bytes of one block: H_kv * head_stride
 };
+
+}  // namespace pkv
+
+namespace pkv {
+
+// Allow the kernel the device's whole opt-in shared memory per block (minus
+// its static shared memory), once per device and kernel; occupancy follows
+// the dynamic size given at each launch.
+template <typename Kernel>
+inline cudaError_t allow_large_smem(Kernel kern, unsigned long long* done_mask) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes);
+    if (e == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+    return e;
+}
+
+// Launch with or without programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// After every thread of the CTA wrote its partition's partial state: count
+// the partition as done; returns true in the CTA that finished last (it then
+// sees every partial and has reset the counter for the next launch).
+__device__ __forceinline__ bool finish_partition(int* counter, int nparts, int* flag_smem) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int prev = atomicAdd(counter, 1);
+        const int last = prev == nparts - 1;
+        if (last) {
+            atomicExch(counter, 0);
+            __threadfence();
+        }
+        *flag_smem = last;
+    }
+    __syncthreads();
+    return *flag_smem != 0;
+}
+
+// Merge the partitions of heads h0 .. h0 + nh - 1 of one sequence inside the
+// decode kernel (the CTA that finished last), with all partial (max, sum)
+// pairs staged in shared memory first: two rounds of global loads in total.
+// `scratch` holds at least 3 * nh * nparts + nh floats, else the heads are
+// merged one after the other.
+template <typename QT, int D>
+__device__ void merge_in_cta(const DecodeParams& p, int seq, int h, int nparts);
+
+template <typename QT, int D>
+__device__ void merge_group_in_cta(const DecodeParams& p, int seq, int h0, int nh, int nparts,
+                                   float* scratch, int scratch_floats) {
+    const int n = nh * nparts;
+    if (3 * n + nh > scratch_floats) {
+        for (int hh = 0; hh < nh; ++hh) merge_in_cta<QT, D>(p, seq, h0 + hh, nparts);
+        return;
+    }
+    float* ml = scratch;        // [nh][nparts][2]
+    float* w = scratch + 2 * n; // [nh][nparts]
+    float* linv = w + n;        // [nh]
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const size_t row = ((size_t)seq * p.H_q + h0 + i / nparts) * p.max_parts + i % nparts;
+        ml[2 * i] = __ldcg(p.ws_ml + row * 2);
+        ml[2 * i + 1] = __ldcg(p.ws_ml + row * 2 + 1);
+    }
+    __syncthreads();
+    for (int hh = threadIdx.x; hh < nh; hh += blockDim.x) {
+        float M = -INFINITY;
+        for (int q = 0; q < nparts; ++q) M = fmaxf(M, ml[2 * (hh * nparts + q)]);
+        float L = 0.f;
+        for (int q = 0; q < nparts; ++q) {
+            const int i = hh * nparts + q;
+            const float wq = M == -INFINITY ? 0.f : exp2f(ml[2 * i] - M);
+            w[i] = wq;
+            L = fmaf(wq, ml[2 * i + 1], L);
+        }
+        linv[hh] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nh * D; i += blockDim.x) {
+        const int hh = i / D, d = i % D;
+        const size_t row0 = ((size_t)seq * p.H_q + h0 + hh) * p.max_parts;
+        float O = 0.f;
+        for (int q = 0; q < nparts; ++q)
+            O = fmaf(w[hh * nparts + q], __ldcg(p.ws_acc + (row0 + q) * D + d), O);
+        reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h0 + hh) * D + d] =
+            Elem<QT>::from_f(O * linv[hh]);
+    }
+}
+
+// One head at a time (the fallback of merge_group_in_cta): threads stride
+// over the D columns.
+template <typename QT, int D>
+__device__ void merge_in_cta(const DecodeParams& p, int seq, int h, int nparts) {
+    const size_t row0 = ((size_t)seq * p.H_q + h) * p.max_parts;
+    float M = -INFINITY;
+    for (int q = 0; q < nparts; ++q) M = fmaxf(M, __ldcg(p.ws_ml + (row0 + q) * 2));
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float L = 0.f, O = 0.f;
+        for (int q = 0; q < nparts && M != -INFINITY; ++q) {
+            const float w = exp2f(__ldcg(p.ws_ml + (row0 + q) * 2) - M);
+            L = fmaf(__ldcg(p.ws_ml + (row0 + q) * 2 + 1), w, L);
+            O = fmaf(__ldcg(p.ws_acc + (row0 + q) * D + d), w, O);
+        }
+        reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h) * D + d] =
+            Elem<QT>::from_f(L > 0.f ? O / L : 0.f);
+    }
+}
 
 }  // namespace pkv

@@ -222,3 +222,29 @@ def test_config_batches_allocate_like_the_oracle():
         b = bm.append_batch(list(range(len(lens))))
         assert a[0].tolist() == b[0]
         _compare(p, bm, set(range(len(lens))))
+
+
+@pytest.mark.parametrize("bs", [1, 2, 4, 8, 16, 32, 64])
+def test_utilisation_readout_fp8_sweep(bs):
+    # bt_stats after admitting the FP8 sweep's 128 sequences and one append:
+    # logical tokens / reserved slots, exactly the closed form over the same
+    # lengths (a block is taken only when the last one is full)
+    from fractions import Fraction
+    from oracle.closed_forms import max_reservation_utilisation, utilisation
+    import workloads as wl
+    cfg = wl.CONFIGS["fp8"].with_block_size(bs)
+    lens = wl.history_lengths(cfg, 0)
+    nb = wl.pool_blocks(cfg, lens)
+    p = pk.kv_pool_create(nb, bs, cfg.n_kv_heads, cfg.head_dim, "fp8", 0.01, 0.01, host_only=True)
+    pk.bt_reset(p, wl.free_order(nb, 0, True))
+    for i, n in enumerate(lens):
+        pk.bt_alloc(p, i, int(n))
+    pk.bt_append_batch(p, list(range(len(lens))))
+    st = pk.bt_stats(p)
+    ctx = [int(n) + 1 for n in lens]
+    assert Fraction(st["logical_tokens"], st["table_slots"]) == utilisation(ctx, bs)
+    assert st["stored_slots"] == st["logical_tokens"]          # nothing shared
+    if bs == 1:
+        assert st["logical_tokens"] == st["table_slots"]
+    # reserving the maximum length (2,048 + 1) up front stores about half as much
+    assert float(max_reservation_utilisation(ctx, 2049)) < 0.55

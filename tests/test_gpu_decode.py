@@ -54,13 +54,28 @@ MHA_CASES = [
 
 
 @pytest.mark.parametrize("dt,d,bs,part", MHA_CASES)
-def test_mha_small(dt, d, bs, part):
+@pytest.mark.parametrize("kernel", [pk.PKV_KERNEL_SIMT_BULK, pk.PKV_KERNEL_SIMT])
+def test_mha_small(dt, d, bs, part, kernel):
     cfg = small("opt13b", n_q_heads=3, n_kv_heads=3, head_dim=d, kv_dtype=dt, q_dtype=dt,
                 block_size=bs, batch=5, lengths=("uniform", 1, 150), min_pool_blocks=0)
     side = setup_config(cfg, seed=d + bs)
-    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0, partition_tokens=part)
+    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0, partition_tokens=part, kernel=kernel)
     compare_out(gpu, ref, dt)
     check_pool_bytes(side)
+
+
+@pytest.mark.parametrize("dt,d", [("f32", 32), ("f32", 64), ("f32", 128), ("f16", 64), ("f16", 128),
+                                  ("bf16", 64), ("bf16", 128)])
+@pytest.mark.parametrize("bs", [1, 2, 8, 16, 32])
+def test_simt_tma_small(dt, d, bs):
+    # the swizzled-TMA CUDA-core kernel, forced, with grouped heads too
+    cfg = small("opt13b", n_q_heads=6, n_kv_heads=3, head_dim=d, kv_dtype=dt, q_dtype=dt,
+                block_size=bs, batch=5, lengths=("uniform", 1, 300), min_pool_blocks=0)
+    side = setup_config(cfg, seed=3 * d + bs, growth=3)
+    for part in (0, 16, 64):
+        gpu, ref, _ = decode_step(side, list(range(cfg.batch)), part // 16,
+                                  partition_tokens=part, kernel=pk.PKV_KERNEL_SIMT_TMA)
+        compare_out(gpu, ref, dt)
 
 
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
@@ -77,11 +92,12 @@ def test_gqa_small(dt, hq, hkv, kernel, part):
 
 @pytest.mark.parametrize("bs", [1, 2, 4, 8, 16, 32, 64])
 @pytest.mark.parametrize("qdt", ["f16", "bf16"])
-def test_fp8_small(bs, qdt):
+@pytest.mark.parametrize("kernel", [pk.PKV_KERNEL_SIMT_BULK, pk.PKV_KERNEL_AUTO])
+def test_fp8_small(bs, qdt, kernel):
     cfg = small("fp8", n_q_heads=4, n_kv_heads=4, q_dtype=qdt, block_size=bs, batch=6,
                 lengths=("uniform", 1, 130))
     side = setup_config(cfg, seed=bs)
-    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0)
+    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0, kernel=kernel)
     compare_out(gpu, ref, "fp8")
     check_pool_bytes(side)
 
@@ -264,7 +280,7 @@ TC_CASES = [
     for (hq, hkv) in ((4, 2), (16, 2), (71, 1), (64, 8), (128, 1))
     for part in (0, 32)
     if not (d == 128 and hq == 128 and bs == 32)
-]
+] + [("f16", 64, bs, 8, 1, 0) for bs in (1, 2, 4)] + [("bf16", 128, bs, 16, 2, 32) for bs in (1, 2, 4)]
 
 
 @pytest.mark.parametrize("dt,d,bs,hq,hkv,part", TC_CASES)
@@ -278,9 +294,9 @@ def test_tensor_path(dt, d, bs, hq, hkv, part):
 
 
 def test_tensor_path_refuses_unsupported_shapes():
-    for dt, d, bs in (("f32", 64, 16), ("f16", 32, 16), ("f16", 64, 4), ("f16", 64, 24)):
+    for dt, d, bs in (("f32", 64, 16), ("f16", 32, 16), ("f16", 64, 24), ("bf16", 128, 12)):
         pool = pk.kv_pool_create(16, bs, 1, d, dt)
-        tdt = {"f32": torch.float32, "f16": torch.float16}[dt]
+        tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[dt]
         q = torch.zeros(1, 4, d, device="cuda", dtype=tdt)
         tables = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
         lens = torch.ones(1, dtype=torch.int32, device="cuda")

@@ -51,7 +51,7 @@ def test_step_runtime_copy_on_write():
     side = setup_config(cfg, variant="b", growth=20)
     _, launches = run_rounds(cfg, side, 20, heads=[0, 35, 70])
     check_pool_bytes(side)
-    assert launches[0] >= 3                           # copy + append + decode (+ merge)
+    assert launches[0] >= 2                           # (copy +) append + decode
     assert pk.bt_stats(side.pool)["cow_count"] == 2 * 3
 
 
@@ -70,12 +70,28 @@ def test_step_runtime_split_and_profile():
         pk.pkv_decode_step(step, seqs, to_torch(q, "f16"), to_torch(kn, "f16"), to_torch(vn, "f16"),
                            cfg.scale, out)
         side.orc.append(list(seqs), kn, vn, "f16")
-        assert step.last_launches == 3                # append, decode, merge
+        # prologue (append) + decode; the split partitions are merged inside
+        # the decode kernel
+        assert step.last_launches == 2
     ref = side.orc.attend(list(seqs), q, "f16", cfg.scale)
     torch.cuda.synchronize()
     compare_out(to_f64(from_torch(out, "f16"), "f16"), ref, "f16")
-    dec, mer = pk.pkv_step_profile_read(step, 4)
-    assert len(dec) == 3 and np.all(dec > 0) and np.all(mer > 0)
+    pro, dec, mer = pk.pkv_step_profile_read(step, 4)
+    assert len(dec) == 3 and np.all(dec > 0) and np.all(pro > 0) and np.all(mer >= 0)
+
+
+@pytest.mark.parametrize("kernel", [pk.PKV_KERNEL_SIMT_TMA, pk.PKV_KERNEL_SIMT_BULK,
+                                    pk.PKV_KERNEL_TENSOR])
+def test_step_runtime_split_merge_every_kernel(kernel):
+    # many rounds with split contexts: the in-kernel merge counters must come
+    # back to zero after every launch (else later rounds merge too early)
+    import dataclasses
+    hkv = 2 if kernel == pk.PKV_KERNEL_TENSOR else 4
+    cfg = dataclasses.replace(wl.CONFIGS["opt13b"], n_q_heads=4, n_kv_heads=hkv, batch=5,
+                              lengths=("uniform", 100, 1200), min_pool_blocks=0)
+    side = setup_config(cfg, growth=12)
+    worst, launches = run_rounds(cfg, side, 12, partition=64, kernel=kernel)
+    assert launches[-1] == (3 if kernel == pk.PKV_KERNEL_SIMT_BULK else 2)
 
 
 def test_step_runtime_rejects_table_overflow_without_changes():
@@ -90,3 +106,31 @@ def test_step_runtime_rejects_table_overflow_without_changes():
         pk.pkv_decode_step(step, seqs, q, kv, kv, 0.1, q.clone())
     assert e.value.status == pk.PKV_ERR_INVALID_ARG
     assert pk.bt_stats(side.pool) == before
+
+
+@pytest.mark.parametrize("lengths,batch", [(("uniform", 1, 60), 6), (("uniform", 1800, 2000), 10)])
+def test_step_runtime_reordered_batches(lengths, batch):
+    # the device keeps the tables between rounds and receives only changed
+    # entries; reordering the batch (or switching to other sequences) must
+    # re-send whole rows - through the parameter block when they fit, through
+    # the packed upload when they do not
+    import dataclasses
+    cfg = dataclasses.replace(wl.CONFIGS["opt13b"], n_q_heads=2, n_kv_heads=2, batch=batch,
+                              lengths=lengths, min_pool_blocks=0)
+    side = setup_config(cfg, growth=6)
+    ids = np.asarray(side.seqs, dtype=np.int64)
+    orders = [ids, ids, ids[::-1].copy(), ids[::-1].copy(), ids[: batch // 2], ids]
+    max_blocks = max(len(side.orc.bm.tables[s]) for s in side.seqs) + 2
+    step = pk.Step(side.pool, batch, max_blocks, 2, "f16")
+    out = torch.empty((batch, 2, 128), device="cuda", dtype=torch.float16)
+    for t, seqs in enumerate(orders):
+        q, kn, vn = step_inputs(side, seqs, t)
+        o = out[: len(seqs)]
+        pk.pkv_decode_step(step, seqs, to_torch(q, "f16"), to_torch(kn, "f16"), to_torch(vn, "f16"),
+                           cfg.scale, o)
+        side.orc.append(list(seqs), kn, vn, "f16")
+        ref = side.orc.attend(list(seqs), q, "f16", cfg.scale)
+        torch.cuda.synchronize()
+        compare_out(to_f64(from_torch(o, "f16"), "f16"), ref, "f16")
+    check_pool_bytes(side)
+    assert pk.pkv_device_error(side.pool) == 0
