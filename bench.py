@@ -336,7 +336,8 @@ def run_ours(args) -> None:
     B = cfg.batch
     max_ctx = max(int(c.max()) for c in ctx) + growth
     max_blocks = -(-max_ctx // cfg.block_size) + 2
-    step = pk.Step(pool, B, max_blocks, cfg.n_q_heads, cfg.q_dtype, args.partition, args.kernel)
+    step = pk.Step(pool, B, max_blocks, cfg.n_q_heads, cfg.q_dtype, args.partition, args.kernel,
+                   max_seqs=B * R)
     dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[cfg.q_dtype]
     gen = torch.Generator(device="cuda")
     gen.manual_seed(4242 + rank)

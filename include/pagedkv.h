@@ -283,14 +283,17 @@ size_t paged_decode_workspace_bytes_ex(const pkv_pool* pool, int B, int n_q_head
  * ------------------------------------------------------------------------- */
 typedef struct pkv_step pkv_step;
 
-/* pkv_step_create - per-batch runtime state for a pool: pinned host staging
- *   and device buffers for up to max_batch sequences of up to max_blocks
- *   blocks each, and the attention workspace for that shape.  All memory is
- *   allocated here, none in pkv_decode_step.  q_dtype: dtype of q, of the new
- *   K/V rows and of the output.  partition_tokens / kernel as in
+/* pkv_step_create - runtime state for decode rounds on a pool: batches of up
+ *   to max_batch sequences whose tables hold up to max_blocks blocks, with
+ *   device-resident block tables kept for up to max_seqs distinct sequences
+ *   (max_seqs >= max_batch; a sequence not seen for the longest time gives
+ *   its row up first), pinned host staging and the attention workspace.  All
+ *   memory is allocated here, none in pkv_decode_step.  q_dtype: dtype of q,
+ *   of the new K/V rows and of the output.  partition_tokens / kernel as in
  *   paged_decode_attention_ex.  Errors: INVALID_ARG, CUDA. */
-pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_q_heads,
-                           pkv_dtype q_dtype, int partition_tokens, int kernel, pkv_step** out);
+pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_blocks,
+                           int n_q_heads, pkv_dtype q_dtype, int partition_tokens, int kernel,
+                           pkv_step** out);
 
 /* pkv_step_destroy - synchronises on the runtime's outstanding copies and
  *   frees its buffers.  NULL is accepted. */
@@ -303,10 +306,11 @@ void pkv_step_destroy(pkv_step* step);
  *      one asynchronous host-to-device copy on `stream`;
  *   3. device: copy-on-write of the shared blocks, append of the B new rows,
  *      then paged decode attention into d_out.
- *   The device keeps the batch's tables between calls; a round sends only
- *   what changed (slots, lengths, copy pairs, new table entries) as the
- *   parameters of one prologue kernel, falling back to a packed host-to-device
- *   copy of the full tables when that does not fit.  With split contexts the
+ *   The device keeps each sequence's table in a row of its own between calls;
+ *   a round sends only what changed (slots, lengths, rows, copy pairs, new
+ *   table entries) as the parameters of one prologue kernel, falling back to
+ *   a packed host-to-device copy of the batch's full tables when that does not
+ *   fit (first sight of many long sequences).  With split contexts the
  *   decode kernel merges the partitions itself (counters in the runtime's
  *   workspace, zero between calls) when the tensor-core or swizzled-TMA
  *   kernel runs.
@@ -338,6 +342,32 @@ pkv_status pkv_step_profile(pkv_step* step, int n, int every);
  *   Errors: INVALID_ARG (cap too small), CUDA. */
 pkv_status pkv_step_profile_read(pkv_step* step, float* prologue_ms, float* decode_ms,
                                  float* merge_ms, int cap, int* n_out);
+
+/* ---------------------------------------------------------------------------
+ * Swapping a sequence out to host memory and back ([F55] §放不下的时候: when
+ * blocks run out a sequence gives up all of its blocks; they can move to CPU
+ * memory and come back when its turn comes).
+ * ------------------------------------------------------------------------- */
+
+/* kv_swap_out - queues on `stream` a copy of every block of seq_id, in
+ *   logical order, into h_k and h_v (pinned host buffers, e.g. cudaHostAlloc,
+ *   layout [n_blocks][n_kv_heads][block_size][head_dim] in the pool dtype,
+ *   capacity_bytes each), then releases the sequence like bt_free.  Returns
+ *   the block and token counts.  The blocks may be handed out again at once:
+ *   device work that writes them must be queued on the same stream (after
+ *   the copy).  h_k/h_v must stay valid until the copy has run.
+ *   Errors: INVALID_ARG (not pinned, too small), UNKNOWN_SEQ, CUDA. */
+pkv_status kv_swap_out(pkv_pool* pool, int64_t seq_id, void* h_k, void* h_v,
+                       size_t capacity_bytes, int32_t* n_blocks_out, int64_t* n_tokens_out,
+                       void* stream);
+
+/* kv_swap_in - admits seq_id again with n_tokens tokens (fresh blocks, as
+ *   bt_alloc) and queues on `stream` the copy of its rows from h_k/h_v
+ *   (pinned, the layout kv_swap_out wrote, capacity_bytes each; the call reads
+ *   ceil(n_tokens / block_size) blocks' worth and refuses smaller buffers).
+ *   Errors: INVALID_ARG, SEQ_EXISTS, NO_BLOCKS (nothing changed), CUDA. */
+pkv_status kv_swap_in(pkv_pool* pool, int64_t seq_id, const void* h_k, const void* h_v,
+                      size_t capacity_bytes, int64_t n_tokens, void* stream);
 
 /* paged_decode_attention_static - paged_decode_attention for callers that
  *   cannot allocate device memory: processes whose GPU memory is already held

@@ -78,6 +78,23 @@ class DecodeOracle:
         del self.k_rows[seq]
         del self.v_rows[seq]
 
+    def swap_out(self, seq: int):
+        """"KV 缓存与分页注意力" §放不下的时候: a sequence gives up all of its
+        blocks, its keys and values moving to CPU memory.  Returns the stored
+        rows ([n][H_kv][d] each) and releases the sequence."""
+        rows = self.history(seq) if self.k_rows[seq] else (None, None)
+        self.free(seq)
+        return rows
+
+    def swap_in(self, seq: int, k_rows: np.ndarray, v_rows: np.ndarray) -> List[int]:
+        """The swapped-out rows come back into fresh blocks (an admission of
+        the same length); returns the slots."""
+        n = 0 if k_rows is None else k_rows.shape[0]
+        slots = self.bm.alloc(seq, n)
+        self.k_rows[seq] = [k_rows[t] for t in range(n)]
+        self.v_rows[seq] = [v_rows[t] for t in range(n)]
+        return slots
+
     def append(self, seqs: Sequence[int], k_new: np.ndarray, v_new: np.ndarray, in_dtype: str):
         """Store one new row per sequence (k_new, v_new [B][H_kv][d]).
         Returns (slots, cow pairs)."""

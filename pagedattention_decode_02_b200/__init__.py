@@ -102,7 +102,7 @@ _sig("paged_decode_workspace_bytes_ex", ctypes.c_size_t, _P, ctypes.c_int, ctype
 _sig("pkv_device_error", _st, _P, _P, ctypes.POINTER(ctypes.c_uint32))
 _sig("pkv_status_str", ctypes.c_char_p, ctypes.c_int)
 _sig("pkv_step_create", _st, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-     ctypes.c_int, ctypes.POINTER(_P))
+     ctypes.c_int, ctypes.c_int, ctypes.POINTER(_P))
 _sig("pkv_step_destroy", None, _P)
 _sig("pkv_decode_step", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
 _sig("pkv_step_last_launches", ctypes.c_int, _P)
@@ -110,6 +110,8 @@ _sig("pkv_step_profile", _st, _P, ctypes.c_int, ctypes.c_int)
 _sig("paged_decode_attention_static", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int,
      ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P)
 _sig("paged_decode_static_scratch_bytes", ctypes.c_size_t)
+_sig("kv_swap_out", _st, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _I32P, _I64P, _P)
+_sig("kv_swap_in", _st, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, ctypes.c_int64, _P)
 _sig("pkv_step_profile_read", _st, _P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float),
      ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int))
 
@@ -120,7 +122,7 @@ EXPORTED = [
     "paged_decode_attention_ex", "paged_decode_workspace_bytes", "paged_decode_workspace_bytes_ex",
     "pkv_device_error", "pkv_status_str", "pkv_step_create", "pkv_step_destroy", "pkv_decode_step",
     "pkv_step_last_launches", "pkv_step_profile", "pkv_step_profile_read",
-    "paged_decode_attention_static", "paged_decode_static_scratch_bytes",
+    "paged_decode_attention_static", "paged_decode_static_scratch_bytes", "kv_swap_out", "kv_swap_in",
 ]
 
 
@@ -406,10 +408,12 @@ class Step:
     """Owns a ``pkv_step*`` (staging, device tables, workspace for one batch shape)."""
 
     def __init__(self, pool: Pool, max_batch: int, max_blocks: int, n_q_heads: int, q_dtype,
-                 partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO):
+                 partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO,
+                 max_seqs: Optional[int] = None):
         qd = DTYPE_NAMES[q_dtype] if isinstance(q_dtype, str) else int(q_dtype)
         h = ctypes.c_void_p()
-        _check(_lib.pkv_step_create(pool.handle, max_batch, max_blocks, n_q_heads, qd,
+        ms = max_batch if max_seqs is None else max_seqs
+        _check(_lib.pkv_step_create(pool.handle, max_batch, ms, max_blocks, n_q_heads, qd,
                                     partition_tokens, kernel, ctypes.byref(h)), "pkv_step_create")
         self.handle = h
         self.pool = pool
@@ -442,8 +446,9 @@ class Step:
 
 
 def pkv_step_create(pool: Pool, max_batch: int, max_blocks: int, n_q_heads: int, q_dtype,
-                    partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO) -> Step:
-    return Step(pool, max_batch, max_blocks, n_q_heads, q_dtype, partition_tokens, kernel)
+                    partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO,
+                    max_seqs: Optional[int] = None) -> Step:
+    return Step(pool, max_batch, max_blocks, n_q_heads, q_dtype, partition_tokens, kernel, max_seqs)
 
 
 def pkv_step_destroy(step: Step) -> None:
@@ -498,3 +503,27 @@ def paged_decode_attention_static(pool: Pool, q, block_tables, context_lens, sca
         int(block_tables.shape[1]), _dev_ptr(context_lens), B, H_q, float(scale), _dev_ptr(out),
         int(partition_tokens), _stream_ptr(stream)), "paged_decode_attention_static")
     return out
+
+
+# ---------------------------------------------------------------------------
+# swap to host memory
+# ---------------------------------------------------------------------------
+def block_bytes(pool: Pool) -> int:
+    return pool.n_kv_heads * pool.block_size * pool.head_dim * ELEM_BYTES[pool.dtype]
+
+
+def kv_swap_out(pool: Pool, seq_id: int, h_k, h_v, stream=None):
+    """Copy seq_id's blocks into pinned host uint8 tensors h_k/h_v and release
+    the sequence.  -> (n_blocks, n_tokens)."""
+    nb = ctypes.c_int32()
+    nt = ctypes.c_int64()
+    cap = min(h_k.numel() * h_k.element_size(), h_v.numel() * h_v.element_size())
+    _check(_lib.kv_swap_out(pool.handle, int(seq_id), h_k.data_ptr(), h_v.data_ptr(), cap,
+                            ctypes.byref(nb), ctypes.byref(nt), _stream_ptr(stream)), "kv_swap_out")
+    return nb.value, nt.value
+
+
+def kv_swap_in(pool: Pool, seq_id: int, h_k, h_v, n_tokens: int, stream=None) -> None:
+    cap = min(h_k.numel() * h_k.element_size(), h_v.numel() * h_v.element_size())
+    _check(_lib.kv_swap_in(pool.handle, int(seq_id), h_k.data_ptr(), h_v.data_ptr(), cap,
+                           int(n_tokens), _stream_ptr(stream)), "kv_swap_in")

@@ -32,6 +32,7 @@ SOURCES = [
     "decode_tc.cu",
     "api.cu",
     "no_alloc.cu",
+    "swap.cu",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -7,6 +7,8 @@
 #include <new>
 #include <vector>
 #include <limits>
+#include <unordered_map>
+#include <algorithm>
 
 #include "block_manager.h"
 #include "decode_launch.h"
@@ -290,7 +292,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                  int n_q_heads, float scale, void* out, void* ws, size_t ws_bytes,
                                  int partition_tokens, int kernel, void* stream,
                                  cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end,
-                                 int* counters = nullptr, bool pdl = false) {
+                                 int* counters = nullptr, bool pdl = false,
+                                 const int32_t* table_rows = nullptr, int n_table_rows = 0) {
     if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
     if (B == 0) return PKV_OK;
     if (!q || !out || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
@@ -345,8 +348,13 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     dp.ws_acc = need ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                                 ((rows * 2 * sizeof(float) + 255) & ~(size_t)255))
                      : nullptr;
-    dp.counters = need ? counters : nullptr;
+    // the tensor-core kernel merges a split KV head's G query heads in the CTA
+    // that finishes last (one handshake per G heads); the one-head CUDA-core
+    // kernels leave it to the merge kernel, launched right behind them
+    dp.counters = (need && use == PKV_KERNEL_TENSOR) ? counters : nullptr;
     dp.pdl = pdl ? 1 : 0;
+    dp.table_rows = table_rows;
+    dp.n_table_rows = n_table_rows;
     const float log2e = 1.4426950408889634f;
     dp.q_scale = scale * log2e * p->k_scale;
     dp.v_scale = p->v_scale;
@@ -410,53 +418,51 @@ pkv_status pkv_device_error(pkv_pool* p, void* stream, uint32_t* bits_out) {
 struct pkv_step {
     static constexpr int kRing = 3;   // pinned staging slots in flight
     pkv_pool* pool = nullptr;
-    int max_batch = 0, max_blocks = 0, n_q_heads = 0;
+    int max_batch = 0, max_seqs = 0, max_blocks = 0, n_q_heads = 0;
     pkv_dtype q_dtype = PKV_F16;
     int partition_tokens = 0, kernel = PKV_KERNEL_AUTO;
-    size_t stage_ints = 0;            // slots | cow src | cow dst | lens | tables
+    // device: slots | cow src | cow dst | lens | rows  (max_batch each)
+    //         | staged tables [max_batch][max_blocks]  (fallback path)
     int32_t* h_stage[kRing] = {};
     cudaEvent_t ev[kRing] = {};
     bool pending[kRing] = {};
     int ring = 0;
     int32_t* d_stage = nullptr;
+    int32_t* d_tables = nullptr;      // persistent [max_seqs][max_blocks], one row per sequence
     void* d_ws = nullptr;
     size_t ws_bytes = 0;
+    int* d_counters = nullptr;        // [max_batch][n_q_heads], zero between launches
     int max_parts = 1;
     int last_launches = 0;
-    // what the device tables (d_stage + 4 * max_batch) hold, row by row
-    std::vector<int64_t> row_seq;
+    // host mirror of the persistent rows
+    std::vector<int64_t> row_seq;     // sequence held, or INT64_MIN
     std::vector<uint64_t> row_epoch;
-    std::vector<int32_t> row_nb;
-    std::vector<int32_t> mirror;      // [max_batch][max_blocks]
-    // host scratch of one round
-    std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_upd_idx, h_upd_val;
+    std::vector<int32_t> row_nb;      // entries the device row holds
+    std::vector<long long> row_used;  // last round that used the row
+    std::unordered_map<int64_t, int> row_of;
+    std::vector<int32_t> mirror;      // [max_seqs][max_blocks]
+    // one round's host scratch
+    std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_cow_rows, h_upd_idx, h_upd_val;
     pkv::StepArgs args;
     long long fast_rounds = 0, slow_rounds = 0;
-    int* d_counters = nullptr;        // [max_batch][n_q_heads], zero between launches
     // profiling: every prof_every-th round records four events (before the
     // prologue, before the decode kernel, between it and the merge, after the
     // merge) into a ring of prof_n entries
     int prof_n = 0;
     int prof_every = 1;
     long long prof_count = 0;
-    long long round = 0;
+    long long round = 0;              // rounds run (row recency)
+    long long prof_start = 0;         // round count when profiling was (re)armed
     cudaEvent_t* prof_ev = nullptr;
 };
 
 namespace {
-// the tensor-core and swizzled-TMA CUDA-core kernels merge split partitions
-// themselves when the step runtime hands them its zeroed counters
+// the tensor-core kernel merges split partitions itself when the step runtime
+// hands it its zeroed counters
 bool decode_merges_in_kernel(const pkv_pool* pool, const pkv_step* s) {
     const int G = s->n_q_heads / pool->n_kv_heads;
     const bool tc = pkv::tensor_path_supported(pool, s->q_dtype, G);
-    const bool s2 = pkv::simt2_supported(pool, G);
-    switch (s->kernel) {
-        case PKV_KERNEL_AUTO: return tc || s2;
-        case PKV_KERNEL_SIMT: return s2;
-        case PKV_KERNEL_TENSOR: return tc;
-        case PKV_KERNEL_SIMT_TMA: return s2;
-        default: return false;
-    }
+    return (s->kernel == PKV_KERNEL_AUTO || s->kernel == PKV_KERNEL_TENSOR) && tc;
 }
 
 void prof_free(pkv_step* s) {
@@ -480,17 +486,53 @@ void step_free(pkv_step* s) {
         if (s->h_stage[i]) cudaFreeHost(s->h_stage[i]);
     }
     if (s->d_stage) cudaFree(s->d_stage);
+    if (s->d_tables) cudaFree(s->d_tables);
     if (s->d_ws) cudaFree(s->d_ws);
     if (s->d_counters) cudaFree(s->d_counters);
     delete s;
+}
+
+// Persistent table row of `seq` for this round: its own row if it has one,
+// else a free row or the least recently used row no sequence of this round
+// holds (max_seqs >= max_batch guarantees one).  A new or evicted row holds
+// nothing (nb = 0), so the whole table is sent.
+int row_for(pkv_step* s, int64_t seq) {
+    auto it = s->row_of.find(seq);
+    int r = -1;
+    if (it != s->row_of.end()) {
+        r = it->second;
+    } else {
+        long long oldest = std::numeric_limits<long long>::max();
+        for (int i = 0; i < s->max_seqs; ++i) {
+            if (s->row_seq[i] == std::numeric_limits<int64_t>::min()) {
+                r = i;
+                break;
+            }
+            if (s->row_used[i] < s->round && s->row_used[i] < oldest) {
+                oldest = s->row_used[i];
+                r = i;
+            }
+        }
+        if (r < 0) return -1;
+        if (s->row_seq[r] != std::numeric_limits<int64_t>::min()) s->row_of.erase(s->row_seq[r]);
+        s->row_seq[r] = seq;
+        s->row_epoch[r] = 0;
+        s->row_nb[r] = 0;
+        s->row_of[seq] = r;
+    }
+    s->row_used[r] = s->round;
+    return r;
 }
 }  // namespace
 
 extern "C" {
 
-pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_q_heads,
-                           pkv_dtype q_dtype, int partition_tokens, int kernel, pkv_step** out) {
+pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_blocks,
+                           int n_q_heads, pkv_dtype q_dtype, int partition_tokens, int kernel,
+                           pkv_step** out) {
     if (!pool || pool->host_only || !out || max_batch < 1 || max_batch > 65535 || max_blocks < 1)
+        return PKV_ERR_INVALID_ARG;
+    if (max_seqs < max_batch || (long long)max_seqs * max_blocks > (1LL << 31) - 1)
         return PKV_ERR_INVALID_ARG;
     if (n_q_heads < pool->n_kv_heads || n_q_heads % pool->n_kv_heads) return PKV_ERR_INVALID_ARG;
     if (pool->dtype == PKV_FP8_E4M3 ? (q_dtype != PKV_F16 && q_dtype != PKV_BF16)
@@ -505,23 +547,26 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_blocks, int n_
     if (!s) return PKV_ERR_INVALID_ARG;
     s->pool = pool;
     s->max_batch = max_batch;
+    s->max_seqs = max_seqs;
     s->max_blocks = max_blocks;
     s->n_q_heads = n_q_heads;
     s->q_dtype = q_dtype;
     s->partition_tokens = partition_tokens;
     s->kernel = kernel;
-    s->stage_ints = (size_t)4 * max_batch + (size_t)max_batch * max_blocks;
-    const size_t bytes = s->stage_ints * sizeof(int32_t);
+    const size_t stage_ints = (size_t)5 * max_batch + (size_t)max_batch * max_blocks;
     bool ok = true;
     for (int i = 0; i < pkv_step::kRing && ok; ++i) {
-        ok &= cudaMallocHost(&s->h_stage[i], bytes) == cudaSuccess;
+        ok &= cudaMallocHost(&s->h_stage[i], stage_ints * sizeof(int32_t)) == cudaSuccess;
         ok &= ok && cudaEventCreateWithFlags(&s->ev[i], cudaEventDisableTiming) == cudaSuccess;
     }
-    ok &= ok && cudaMalloc(&s->d_stage, bytes) == cudaSuccess;
-    s->row_seq.assign(max_batch, std::numeric_limits<int64_t>::min());
-    s->row_epoch.assign(max_batch, 0);
-    s->row_nb.assign(max_batch, 0);
-    s->mirror.assign((size_t)max_batch * max_blocks, -1);
+    ok &= ok && cudaMalloc(&s->d_stage, stage_ints * sizeof(int32_t)) == cudaSuccess;
+    ok &= ok && cudaMalloc(&s->d_tables, (size_t)max_seqs * max_blocks * sizeof(int32_t)) ==
+                    cudaSuccess;
+    s->row_seq.assign(max_seqs, std::numeric_limits<int64_t>::min());
+    s->row_epoch.assign(max_seqs, 0);
+    s->row_nb.assign(max_seqs, 0);
+    s->row_used.assign(max_seqs, -1);
+    s->mirror.assign((size_t)max_seqs * max_blocks, -1);
     const int P = resolve_partition(pool, max_blocks, partition_tokens,
                                     n_q_heads / pool->n_kv_heads);
     s->max_parts = parts_for(pool, max_blocks, P);
@@ -573,41 +618,50 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     pkv_status ps = pool->bm.append_batch(seq_ids, B, s->h_slots.data(), s->h_src.data(),
                                           s->h_dst.data(), &n_cow);
     if (ps != PKV_OK) return ps;
+    ++s->round;
     // rows of each shared block to copy: the fill before the write, i.e. the
     // offset of the slot that the copying sequence writes into the copy
-    s->h_rows.resize(n_cow);
+    s->h_cow_rows.resize(n_cow);
     for (int j = 0; j < n_cow; ++j) {
-        s->h_rows[j] = bs;
+        s->h_cow_rows[j] = bs;
         for (int i = 0; i < B; ++i)
             if (s->h_slots[i] / bs == s->h_dst[j]) {
-                s->h_rows[j] = s->h_slots[i] % bs;
+                s->h_cow_rows[j] = s->h_slots[i] % bs;
                 break;
             }
     }
-    // table entries that differ from what the device holds
+    // each sequence's persistent row, and the entries of it the device lacks
+    s->h_rows.resize(B);
     s->h_upd_idx.clear();
     s->h_upd_val.clear();
+    for (int i = 0; i < B; ++i) {
+        const int r = row_for(s, seq_ids[i]);
+        if (r < 0) return PKV_ERR_INVALID_ARG;   // cannot happen: max_seqs >= max_batch
+        s->h_rows[i] = r;
+    }
     const size_t limit = (size_t)pkv::kStepArgInts;
-    bool fits = (size_t)2 * B + 3 * (size_t)n_cow <= limit;
+    const size_t fixed = (size_t)3 * B + 3 * (size_t)n_cow;
+    bool fits = fixed <= limit;
     for (int i = 0; i < B && fits; ++i) {
         const pkv::Sequence* sq = pool->bm.find(seq_ids[i]);
+        const int r = s->h_rows[i];
         const int nb = (int)sq->blocks.size();
-        const bool same = s->row_seq[i] == seq_ids[i] && s->row_epoch[i] == sq->epoch;
-        const int from = same ? (s->row_nb[i] > 0 ? s->row_nb[i] - 1 : 0) : 0;
-        const int32_t* m = s->mirror.data() + (size_t)i * s->max_blocks;
+        const bool same = s->row_epoch[r] == sq->epoch;
+        const int from = same ? (s->row_nb[r] > 0 ? s->row_nb[r] - 1 : 0) : 0;
+        const int32_t* m = s->mirror.data() + (size_t)r * s->max_blocks;
         for (int e = from; e < nb; ++e) {
-            if (same && e < s->row_nb[i] && m[e] == sq->blocks[e]) continue;
-            s->h_upd_idx.push_back(i * s->max_blocks + e);
+            if (same && e < s->row_nb[r] && m[e] == sq->blocks[e]) continue;
+            s->h_upd_idx.push_back(r * s->max_blocks + e);
             s->h_upd_val.push_back(sq->blocks[e]);
         }
-        fits = 2 * B + 3 * (size_t)n_cow + 2 * s->h_upd_idx.size() <= limit;
+        fits = fixed + 2 * s->h_upd_idx.size() <= limit;
     }
     int launches = 0;
     int32_t* d_lens = s->d_stage + 3 * mb;
-    int32_t* d_tables = s->d_stage + 4 * mb;
+    int32_t* d_rows = s->d_stage + 4 * mb;
     cudaEvent_t e_pre = nullptr, e0 = nullptr, e1 = nullptr, e2 = nullptr;
-    const bool profiled = s->prof_n > 0 && (s->round % s->prof_every) == 0;
-    ++s->round;
+    const bool profiled =
+        s->prof_n > 0 && ((s->round - 1 - s->prof_start) % s->prof_every) == 0;
     if (profiled) {
         const int i = (int)(s->prof_count % s->prof_n);
         e_pre = s->prof_ev[4 * i];
@@ -622,32 +676,35 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         a.B = B;
         a.n_cow = n_cow;
         a.n_upd = (int32_t)s->h_upd_idx.size();
-        a.table_cap = mb * s->max_blocks;
+        a.table_cap = s->max_seqs * s->max_blocks;
         int32_t* d = a.data;
         for (int i = 0; i < B; ++i) d[i] = s->h_slots[i];
         d += B;
         for (int i = 0; i < B; ++i) d[i] = (int32_t)pool->bm.find(seq_ids[i])->length;
         d += B;
+        for (int i = 0; i < B; ++i) d[i] = s->h_rows[i];
+        d += B;
         for (int j = 0; j < n_cow; ++j) d[j] = s->h_src[j];
         d += n_cow;
         for (int j = 0; j < n_cow; ++j) d[j] = s->h_dst[j];
         d += n_cow;
-        for (int j = 0; j < n_cow; ++j) d[j] = s->h_rows[j];
+        for (int j = 0; j < n_cow; ++j) d[j] = s->h_cow_rows[j];
         d += n_cow;
         for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_idx[u];
         d += a.n_upd;
         for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_val[u];
         cudaError_t e = pkv::launch_step_prologue(
-            a, pool->k, pool->v, k_new, v_new, s->q_dtype, pool->dtype, d_tables, d_lens,
-            pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale, pool->v_scale,
-            pool->d_err, st);
+            a, pool->k, pool->v, k_new, v_new, s->q_dtype, pool->dtype, s->d_tables, d_lens,
+            d_rows, pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale,
+            pool->v_scale, pool->d_err, st);
         if (e != cudaSuccess) return PKV_ERR_CUDA;
         launches = 1;
         for (size_t u = 0; u < s->h_upd_idx.size(); ++u) s->mirror[s->h_upd_idx[u]] = s->h_upd_val[u];
         ++s->fast_rounds;
     } else {
-        // large rounds: one packed upload of slots, copy pairs, lengths and the
-        // batch's full tables from pinned staging, then copy and append
+        // large rounds: one packed upload of slots, copy pairs, lengths, rows and
+        // the batch's full tables from pinned staging; the tables are scattered
+        // into their persistent rows, then the copy and the append
         const int r = s->ring;
         if (s->pending[r] && cudaEventSynchronize(s->ev[r]) != cudaSuccess) return PKV_ERR_CUDA;
         s->pending[r] = false;
@@ -657,15 +714,21 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
             h[mb + j] = s->h_src[j];
             h[2 * mb + j] = s->h_dst[j];
         }
-        ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, h + 4 * mb, h + 3 * mb, nullptr);
+        for (int i = 0; i < B; ++i) h[4 * mb + i] = s->h_rows[i];
+        int32_t* ht = h + 5 * mb;
+        ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, ht, h + 3 * mb, nullptr);
         if (ps != PKV_OK) return ps;   // cannot happen after the checks above
-        const size_t ints = (size_t)4 * mb + (size_t)B * s->max_blocks;
+        const size_t ints = (size_t)5 * mb + (size_t)B * s->max_blocks;
         if (cudaMemcpyAsync(s->d_stage, h, ints * sizeof(int32_t), cudaMemcpyHostToDevice, st) !=
                 cudaSuccess ||
             cudaEventRecord(s->ev[r], st) != cudaSuccess)
             return PKV_ERR_CUDA;
         s->pending[r] = true;
         s->ring = (r + 1) % pkv_step::kRing;
+        if (pkv::launch_scatter_rows(s->d_stage + 5 * mb, d_rows, B, s->max_blocks, s->d_tables,
+                                     st) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        ++launches;
         if (n_cow > 0) {
             ps = block_copy(pool, s->d_stage + mb, s->d_stage + 2 * mb, n_cow, stream);
             if (ps != PKV_OK) return ps;
@@ -674,20 +737,23 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         ps = kv_append(pool, s->d_stage, B, k_new, v_new, s->q_dtype, stream);
         if (ps != PKV_OK) return ps;
         ++launches;
-        std::copy(h + 4 * mb, h + 4 * mb + (size_t)B * s->max_blocks, s->mirror.begin());
+        for (int i = 0; i < B; ++i)
+            std::copy(ht + (size_t)i * s->max_blocks, ht + (size_t)(i + 1) * s->max_blocks,
+                      s->mirror.begin() + (size_t)s->h_rows[i] * s->max_blocks);
         ++s->slow_rounds;
     }
     for (int i = 0; i < B; ++i) {
         const pkv::Sequence* sq = pool->bm.find(seq_ids[i]);
-        s->row_seq[i] = seq_ids[i];
-        s->row_epoch[i] = sq->epoch;
-        s->row_nb[i] = (int32_t)sq->blocks.size();
+        const int r = s->h_rows[i];
+        s->row_epoch[r] = sq->epoch;
+        s->row_nb[r] = (int32_t)sq->blocks.size();
     }
     // the decode kernel starts its launch while the prologue runs (programmatic
     // dependent launch), except in profiled rounds whose events sit between
-    ps = decode_attention_impl(pool, q, s->q_dtype, d_tables, s->max_blocks, d_lens, B,
+    ps = decode_attention_impl(pool, q, s->q_dtype, s->d_tables, s->max_blocks, d_lens, B,
                                s->n_q_heads, scale, out, s->d_ws, s->ws_bytes, s->partition_tokens,
-                               s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled);
+                               s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled,
+                               d_rows, s->max_seqs);
     if (ps != PKV_OK) return ps;
     if (profiled) ++s->prof_count;
     launches += 1 + (s->max_parts > 1 && !decode_merges_in_kernel(pool, s) ? 1 : 0);
@@ -707,7 +773,7 @@ pkv_status pkv_step_profile(pkv_step* s, int n, int every) {
     if (!s->prof_ev) return PKV_ERR_INVALID_ARG;
     s->prof_n = n;
     s->prof_every = every;
-    s->round = 0;
+    s->prof_start = s->round;   // the next round is profiled
     for (int i = 0; i < 4 * n; ++i)
         if (cudaEventCreate(&s->prof_ev[i]) != cudaSuccess) {
             prof_free(s);

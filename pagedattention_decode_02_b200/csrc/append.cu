@@ -127,13 +127,14 @@ __global__ void kv_append_copy_kernel(uint8_t* k_pool, uint8_t* v_pool, const in
 template <typename IN, bool FP8>
 __global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t* k_pool,
                                      uint8_t* v_pool, const IN* k, const IN* v, int32_t* tables,
-                                     int32_t* lens, int H, int D, int bs, int num_blocks,
-                                     float k_scale, float v_scale, uint32_t* err) {
+                                     int32_t* lens, int32_t* rows, int H, int D, int bs,
+                                     int num_blocks, float k_scale, float v_scale, uint32_t* err) {
     allow_dependent_launch();   // the decode kernel may start its launch now
     const int B = a.B;
     const int32_t* slots = a.data;
     const int32_t* lens_in = a.data + B;
-    const int32_t* cow_src = a.data + 2 * B;
+    const int32_t* rows_in = a.data + 2 * B;
+    const int32_t* cow_src = a.data + 3 * B;
     const int32_t* cow_dst = cow_src + a.n_cow;
     const int32_t* cow_rows = cow_dst + a.n_cow;
     const int32_t* upd_idx = cow_rows + a.n_cow;
@@ -143,7 +144,10 @@ __global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t
     const long long stride = (long long)gridDim.x * blockDim.x;
     const long long first = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     if (blockIdx.y == 0) {
-        for (long long i = first; i < B; i += stride) lens[i] = lens_in[i];
+        for (long long i = first; i < B; i += stride) {
+            lens[i] = lens_in[i];
+            rows[i] = rows_in[i];
+        }
         for (long long u = first; u < a.n_upd; u += stride) {
             const int idx = upd_idx[u];
             if (idx >= 0 && idx < a.table_cap) tables[idx] = upd_val[u];
@@ -174,13 +178,13 @@ __global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t
         return;
     }
     const int j = blockIdx.y - 1;
-    const int s = cow_src[j], d = cow_dst[j], rows = cow_rows[j];
-    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || rows < 0 || rows > bs) {
+    const int s = cow_src[j], d = cow_dst[j], n_rows = cow_rows[j];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || n_rows < 0 || n_rows > bs) {
         if (first == 0) report_error(err, PKV_DEVERR_BLOCK_ID);
         return;
     }
-    const long long tile = (long long)bs * row_bytes;           // one (block, head) tile
-    const long long per_head = (long long)rows * row_bytes / 16; // chunks copied per tile
+    const long long tile = (long long)bs * row_bytes;             // one (block, head) tile
+    const long long per_head = (long long)n_rows * row_bytes / 16; // chunks copied per tile
     const long long total = 2LL * H * per_head;
     for (long long i = first; i < total; i += stride) {
         const int which = (int)(i / (H * per_head));
@@ -280,9 +284,9 @@ namespace pkv {
 
 cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
                                  const void* k, const void* v, int in_dtype, int kv_dtype,
-                                 int32_t* tables, int32_t* lens, int H, int D, int bs,
-                                 int num_blocks, float k_scale, float v_scale, uint32_t* err,
-                                 cudaStream_t st) {
+                                 int32_t* tables, int32_t* lens, int32_t* rows, int H, int D,
+                                 int bs, int num_blocks, float k_scale, float v_scale,
+                                 uint32_t* err, cudaStream_t st) {
     constexpr int kThreads = 256;
     const int eb = kv_dtype == PKV_F32 ? 4 : kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
     const int chunks_per_row = kv_dtype == PKV_FP8_E4M3 ? D / 16 : D * eb / 16;
@@ -297,31 +301,55 @@ cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_
         switch (in_dtype) {
             case PKV_F32:
                 step_prologue_kernel<float, true><<<grid, kThreads, 0, st>>>(
-                    a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, H, D, bs,
+                    a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, H, D, bs,
                     num_blocks, k_scale, v_scale, err);
                 break;
             case PKV_F16:
                 step_prologue_kernel<__half, true><<<grid, kThreads, 0, st>>>(
-                    a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, H, D, bs,
+                    a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, H, D, bs,
                     num_blocks, k_scale, v_scale, err);
                 break;
             case PKV_BF16:
                 step_prologue_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, st>>>(
                     a, k_pool, v_pool, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, tables,
-                    lens, H, D, bs, num_blocks, k_scale, v_scale, err);
+                    lens, rows, H, D, bs, num_blocks, k_scale, v_scale, err);
                 break;
             default:
                 return cudaErrorInvalidValue;
         }
     } else if (kv_dtype == PKV_F32) {
         step_prologue_kernel<float, false><<<grid, kThreads, 0, st>>>(
-            a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, H, D, bs,
+            a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, H, D, bs,
             num_blocks, k_scale, v_scale, err);
     } else {
         step_prologue_kernel<__half, false><<<grid, kThreads, 0, st>>>(
-            a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, H, D, bs,
+            a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, H, D, bs,
             num_blocks, k_scale, v_scale, err);
     }
+    return cudaGetLastError();
+}
+
+}  // namespace pkv
+
+namespace pkv {
+namespace {
+__global__ void scatter_rows_kernel(const int32_t* staged, const int32_t* rows, int B,
+                                    int max_blocks, int32_t* tables) {
+    const long long total = (long long)B * max_blocks;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int b = (int)(i / max_blocks);
+        tables[(long long)rows[b] * max_blocks + i % max_blocks] = staged[i];
+    }
+}
+}  // namespace
+
+cudaError_t launch_scatter_rows(const int32_t* staged, const int32_t* rows, int B, int max_blocks,
+                                int32_t* tables, cudaStream_t st) {
+    const long long total = (long long)B * max_blocks;
+    long long grid = (total + 255) / 256;
+    grid = grid < 1 ? 1 : (grid > 148 * 8 ? 148 * 8 : grid);
+    scatter_rows_kernel<<<(unsigned)grid, 256, 0, st>>>(staged, rows, B, max_blocks, tables);
     return cudaGetLastError();
 }
 

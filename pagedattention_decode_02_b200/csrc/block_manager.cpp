@@ -172,6 +172,14 @@ pkv_status BlockManager::release(int64_t seq) {
     return PKV_OK;
 }
 
+void BlockManager::undo_alloc(int64_t seq) {
+    auto it = seqs_.find(seq);
+    if (it == seqs_.end()) return;
+    const std::vector<int32_t>& b = it->second.blocks;
+    for (auto r = b.rbegin(); r != b.rend(); ++r) unpop_front(*r);
+    seqs_.erase(it);
+}
+
 pkv_status BlockManager::export_tables(const int64_t* seqs, int n, int max_blocks, int32_t* tables,
                                        int32_t* lens, int32_t* fills) const {
     if (n < 0 || max_blocks < 0 || (n > 0 && (!seqs || !lens || (max_blocks > 0 && !tables))))

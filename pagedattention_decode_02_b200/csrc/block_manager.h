@@ -35,6 +35,9 @@ class BlockManager {
                             int32_t* cow_dst, int* n_cow);
     pkv_status fork(int64_t parent, int64_t child);
     pkv_status release(int64_t seq);
+    // undo the most recent alloc(seq): its blocks go back to the front of the
+    // free queue in their original order (only valid right after that alloc)
+    void undo_alloc(int64_t seq);
     pkv_status export_tables(const int64_t* seqs, int n, int max_blocks, int32_t* tables,
                              int32_t* lens, int32_t* fills) const;
     pkv_status num_blocks_of(int64_t seq, int32_t* out) const;

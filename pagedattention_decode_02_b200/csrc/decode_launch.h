@@ -37,10 +37,11 @@ cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, cons
 
 // One decode round's small host-side results, passed by value as kernel
 // parameters (no separate host-to-device copy):
-//   data = slots[B] | lens[B] | cow_src[n_cow] | cow_dst[n_cow] | cow_rows[n_cow]
-//          | upd_idx[n_upd] | upd_val[n_upd]
-// cow_rows[j] = rows of the shared block to copy (the fill before the write);
-// upd_* = changed block-table entries (flat index into [max_batch][max_blocks]).
+//   data = slots[B] | lens[B] | rows[B] | cow_src[n_cow] | cow_dst[n_cow]
+//          | cow_rows[n_cow] | upd_idx[n_upd] | upd_val[n_upd]
+// rows[i] = persistent table row of sequence i; cow_rows[j] = rows of the
+// shared block to copy (the fill before the write); upd_* = changed
+// block-table entries (flat index into [table rows][max_blocks]).
 constexpr int kStepArgInts = 990;   // the whole parameter block stays under 4 KB
 struct StepArgs {
     int32_t B, n_cow, n_upd, table_cap;
@@ -52,9 +53,13 @@ struct StepArgs {
 // B new rows (FP8 pools quantise).
 cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
                                  const void* k, const void* v, int in_dtype, int kv_dtype,
-                                 int32_t* tables, int32_t* lens, int n_kv_heads, int head_dim,
-                                 int block_size, int num_blocks, float k_scale, float v_scale,
-                                 uint32_t* err, cudaStream_t st);
+                                 int32_t* tables, int32_t* lens, int32_t* rows, int n_kv_heads,
+                                 int head_dim, int block_size, int num_blocks, float k_scale,
+                                 float v_scale, uint32_t* err, cudaStream_t st);
+
+// Copy staged full tables ([B][max_blocks]) into their persistent rows.
+cudaError_t launch_scatter_rows(const int32_t* staged, const int32_t* rows, int B, int max_blocks,
+                                int32_t* tables, cudaStream_t st);
 
 // Store new rows into their slots (FP8 pools quantise).
 cudaError_t launch_kv_append(uint8_t* k_pool, uint8_t* v_pool, const int32_t* slots, int n_tokens,

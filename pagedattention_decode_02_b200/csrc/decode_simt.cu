@@ -157,9 +157,10 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
     const int n_lb = (t_end - 1) / bs - lb0 + 1;
 
     // the partition's block ids, validated once
-    bool bad = false;
-    for (int i = tid; i < n_lb; i += kThreads) {
-        int32_t b = p.tables[(size_t)seq * p.max_blocks + lb0 + i];
+    const long long trow = table_row(p, seq);
+    bool bad = trow < 0;
+    for (int i = tid; i < n_lb && trow >= 0; i += kThreads) {
+        int32_t b = p.tables[trow * p.max_blocks + lb0 + i];
         bad |= (b < 0 || b >= p.num_blocks);
         blk[i] = b;
     }
@@ -349,6 +350,7 @@ merge_kernel(const DecodeParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x * kMergeWarps + warp;
     const int seq = blockIdx.y;
+    grid_dependency_wait();   // the decode kernel's partials (programmatic launch)
     if (h >= p.H_q) return;
     const int c = p.lens[seq];
     if (c < 1 || c > p.max_blocks * p.block_size) return;   // zeroed by the decode kernel
@@ -444,7 +446,9 @@ cudaError_t launch_simt_q(const DecodeParams& p, int D, int hpc, cudaStream_t st
 
 cudaError_t launch_merge(const DecodeParams& p, int q_dtype, int D, cudaStream_t st) {
     const dim3 grid((p.H_q + kMergeWarps - 1) / kMergeWarps, p.B);
-#define PKV_MERGE(QT, DD) merge_kernel<QT, DD><<<grid, kMergeWarps * 32, 0, st>>>(p)
+    cudaError_t e = cudaSuccess;
+#define PKV_MERGE(QT, DD) \
+    e = launch_kernel(merge_kernel<QT, DD>, grid, dim3(kMergeWarps * 32), 0, st, p.pdl != 0, p)
     if (q_dtype == PKV_F32) {
         if (D == 32) PKV_MERGE(float, 32); else if (D == 64) PKV_MERGE(float, 64); else PKV_MERGE(float, 128);
     } else if (q_dtype == PKV_F16) {
@@ -454,7 +458,7 @@ cudaError_t launch_merge(const DecodeParams& p, int q_dtype, int D, cudaStream_t
         else PKV_MERGE(__nv_bfloat16, 128);
     }
 #undef PKV_MERGE
-    return cudaGetLastError();
+    return e;
 }
 
 int simt_heads_per_cta(int group) {

@@ -145,6 +145,7 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     __shared__ int last_flag;
     grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
+    const long long trow = table_row(p, seq);   // issued together with the length load
     const int c = p.lens[seq];
     if (c < 1 || c > p.max_blocks * bs) {
         if (part == 0) {
@@ -162,9 +163,9 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int lb0 = t_begin >> bs_shift;
     const int n_lb = ((t_end - 1) >> bs_shift) - lb0 + 1;
 
-    bool bad = false;
-    for (int i = tid; i < n_lb; i += NT) {
-        const int32_t b = p.tables[(size_t)seq * p.max_blocks + lb0 + i];
+    bool bad = trow < 0;
+    for (int i = tid; i < n_lb && trow >= 0; i += NT) {
+        const int32_t b = p.tables[trow * p.max_blocks + lb0 + i];
         bad |= (b < 0 || b >= p.num_blocks);
         blk[i] = b;
     }

@@ -136,6 +136,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     float* comb = reinterpret_cast<float*>(smem);                     // [NW][16][D + 2]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS, S>());
     uint64_t* empty = full + TS * kStages;
+    int32_t* blk = reinterpret_cast<int32_t*>(empty + TS * kStages);   // the partition's block ids
 
     const int part = blockIdx.x;
     const int g = blockIdx.y;
@@ -152,6 +153,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     __shared__ int last_flag;
     grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
+    const long long trow = table_row(p, seq);   // issued together with the length load
     const int c = p.lens[seq];
     if (c < 1 || c > p.max_blocks * bs) {
         if (part == 0) {
@@ -166,12 +168,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (part >= nparts) return;
     const int t_begin = part * P;
     const int t_end = min(c, t_begin + P);
-    const int32_t* table = p.tables + (size_t)seq * p.max_blocks;
+    const int32_t* table = p.tables + (trow < 0 ? 0 : trow) * p.max_blocks;
 
-    bool bad = false;
-    for (int lb = t_begin / bs + tid; lb <= (t_end - 1) / bs; lb += NT) {
+    const int lb0 = t_begin / bs;
+    bool bad = trow < 0;
+    for (int lb = lb0 + tid; lb <= (t_end - 1) / bs && trow >= 0; lb += NT) {
         const int32_t b = table[lb];
         bad |= (b < 0 || b >= p.num_blocks);
+        blk[lb - lb0] = b;
     }
     if (tid == 0) {
         for (int i = 0; i < TS * kStages; ++i) {
@@ -222,7 +226,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int bx = 0; bx < n_boxes; ++bx) {
                 const int t0 = a + bx * rows_per_box;
                 const int lb = t0 / bs;
-                const int y = (table[lb] * p.H_kv + g) * bs + (t0 - lb * bs);
+                const int y = (blk[lb - lb0] * p.H_kv + g) * bs + (t0 - lb * bs);
 #pragma unroll
                 for (int hf = 0; hf < HALVES; ++hf) {
                     const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
@@ -465,12 +469,18 @@ template <int D, int MT, int TS, int S>
 constexpr int tc_smem_bytes() {
     return 1024 + tc_union_bytes<D, MT, TS, S>() + 2 * TS * S * 8;
 }
+// plus the partition's block ids: part_tokens / bs + 2 entries
+inline int tc_table_bytes(const DecodeParams& p) {
+    return ((p.part_tokens / p.block_size + 2) * 4 + 15) & ~15;
+}
 
 template <typename T, int D, int MT, int TS, int S = (D == 128 ? 2 : 3)>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                         int q_dtype, cudaStream_t st, cudaEvent_t mid) {
-    constexpr int smem = tc_smem_bytes<D, MT, TS, S>();
-    static_assert(smem <= 227 * 1024 - 64, "shared memory budget");
+    constexpr int base = tc_smem_bytes<D, MT, TS, S>();
+    static_assert(base <= 227 * 1024 - 64, "shared memory budget");
+    const int smem = base + tc_table_bytes(p);
+    if (smem > 227 * 1024 - 64) return cudaErrorInvalidValue;
     auto kern = decode_tc_kernel<T, D, MT, TS, S>;
     static unsigned long long attr_done = 0;
     cudaError_t e = allow_large_smem(kern, &attr_done);

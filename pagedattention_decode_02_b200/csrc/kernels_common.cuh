@@ -250,6 +250,9 @@ struct DecodeParams {
     const int32_t* lens;
     float* ws_ml;    // [B][H_q][max_parts][2]  (running max in log2 units, sum)
     float* ws_acc;   // [B][H_q][max_parts][D]  (unnormalised accumulator)
+    const int32_t* table_rows;  // [B] row of `tables` holding sequence i's table, or null
+                                // (row i); rows outside [0, n_table_rows) are rejected
+    int n_table_rows;
     int pdl;         // host side: launch with programmatic stream serialization
     int* counters;   // [B][H_q] partitions finished, or null: when set, the last
                      // CTA of a split (sequence, head) merges in the decode
@@ -268,6 +271,14 @@ struct DecodeParams {
 }  // namespace pkv
 
 namespace pkv {
+
+// Row of the block-table array that holds sequence `seq`'s table; -1 if the
+// row index is out of range.
+__device__ __forceinline__ long long table_row(const DecodeParams& p, int seq) {
+    if (!p.table_rows) return seq;
+    const int r = p.table_rows[seq];
+    return (r >= 0 && r < p.n_table_rows) ? r : -1;
+}
 
 // Allow the kernel the device's whole opt-in shared memory per block (minus
 // its static shared memory), once per device and kernel; occupancy follows
@@ -312,9 +323,12 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
 // the partition as done; returns true in the CTA that finished last (it then
 // sees every partial and has reset the counter for the next launch).
 __device__ __forceinline__ bool finish_partition(int* counter, int nparts, int* flag_smem) {
-    __threadfence();
+    // the CTA barrier orders every thread's partial-state stores before thread
+    // 0's device-scope fence (fences are cumulative), which orders them
+    // before the counter update that other CTAs observe
     __syncthreads();
     if (threadIdx.x == 0) {
+        __threadfence();
         const int prev = atomicAdd(counter, 1);
         const int last = prev == nparts - 1;
         if (last) {

@@ -70,9 +70,9 @@ def test_step_runtime_split_and_profile():
         pk.pkv_decode_step(step, seqs, to_torch(q, "f16"), to_torch(kn, "f16"), to_torch(vn, "f16"),
                            cfg.scale, out)
         side.orc.append(list(seqs), kn, vn, "f16")
-        # prologue (append) + decode; the split partitions are merged inside
-        # the decode kernel
-        assert step.last_launches == 2
+        # prologue (append) + decode + merge (the one-head CUDA-core kernel
+        # leaves the merge to its own kernel)
+        assert step.last_launches == 3
     ref = side.orc.attend(list(seqs), q, "f16", cfg.scale)
     torch.cuda.synchronize()
     compare_out(to_f64(from_torch(out, "f16"), "f16"), ref, "f16")
@@ -91,7 +91,7 @@ def test_step_runtime_split_merge_every_kernel(kernel):
                               lengths=("uniform", 100, 1200), min_pool_blocks=0)
     side = setup_config(cfg, growth=12)
     worst, launches = run_rounds(cfg, side, 12, partition=64, kernel=kernel)
-    assert launches[-1] == (3 if kernel == pk.PKV_KERNEL_SIMT_BULK else 2)
+    assert launches[-1] == (2 if kernel == pk.PKV_KERNEL_TENSOR else 3)
 
 
 def test_step_runtime_rejects_table_overflow_without_changes():
@@ -134,3 +134,69 @@ def test_step_runtime_reordered_batches(lengths, batch):
         compare_out(to_f64(from_torch(o, "f16"), "f16"), ref, "f16")
     check_pool_bytes(side)
     assert pk.pkv_device_error(side.pool) == 0
+
+
+def test_step_runtime_evicts_rows_of_sequences_not_in_the_batch():
+    # two disjoint batches alternate through a runtime that keeps device rows
+    # for only one batch's worth of sequences: every switch evicts rows and
+    # sends whole tables again
+    import dataclasses
+    cfg = dataclasses.replace(wl.CONFIGS["opt13b"], n_q_heads=2, n_kv_heads=2, batch=8,
+                              lengths=("uniform", 20, 300), min_pool_blocks=0)
+    side = setup_config(cfg, growth=8)
+    a = np.arange(0, 4, dtype=np.int64)
+    b = np.arange(4, 8, dtype=np.int64)
+    step = pk.Step(side.pool, 4, 32, 2, "f16", max_seqs=4)
+    out = torch.empty((4, 2, 128), device="cuda", dtype=torch.float16)
+    for t, seqs in enumerate([a, b, a, a, b, a, b, b]):
+        q, kn, vn = step_inputs(side, seqs, t)
+        pk.pkv_decode_step(step, seqs, to_torch(q, "f16"), to_torch(kn, "f16"), to_torch(vn, "f16"),
+                           cfg.scale, out)
+        side.orc.append(list(seqs), kn, vn, "f16")
+        ref = side.orc.attend(list(seqs), q, "f16", cfg.scale)
+        torch.cuda.synchronize()
+        compare_out(to_f64(from_torch(out, "f16"), "f16"), ref, "f16")
+    assert pk.pkv_device_error(side.pool) == 0
+
+
+@pytest.mark.parametrize("dt,bs", [("f16", 16), ("bf16", 4), ("fp8", 16), ("f32", 1)])
+def test_swap_out_and_in(dt, bs):
+    # "KV 缓存与分页注意力" section 放不下的时候: a sequence gives up all of its blocks
+    # to CPU memory and comes back later; its attention afterwards equals the
+    # oracle's, the host copy holds exactly its stored rows, and its new
+    # blocks follow the free queue like any admission
+    import dataclasses
+    base = "fp8" if dt == "fp8" else "opt13b"
+    cfg = dataclasses.replace(wl.CONFIGS[base], n_q_heads=4, n_kv_heads=2, head_dim=64 if dt != "fp8" else 128,
+                              kv_dtype=dt, q_dtype="f16" if dt == "fp8" else dt, block_size=bs,
+                              batch=5, lengths=("uniform", 30, 200), min_pool_blocks=0)
+    side = setup_config(cfg, growth=4)
+    seqs = list(range(cfg.batch))
+    from paged_harness import decode_step
+    decode_step(side, seqs, 0)
+    victim = 2
+    bb = pk.block_bytes(side.pool)
+    nb = len(side.orc.bm.tables[victim])
+    hk = torch.empty(nb * bb, dtype=torch.uint8).pin_memory()
+    hv = torch.empty(nb * bb, dtype=torch.uint8).pin_memory()
+    n_blocks, n_tokens = pk.kv_swap_out(side.pool, victim, hk, hv)
+    torch.cuda.synchronize()
+    krows, vrows = side.orc.swap_out(victim)
+    assert (n_blocks, n_tokens) == (nb, len(krows))
+    store = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16, "fp8": np.uint8}[dt]
+    img_k = hk.numpy().view(store).reshape(nb, cfg.n_kv_heads, bs, cfg.head_dim)
+    got = np.stack([img_k[t // bs, :, t % bs, :] for t in range(n_tokens)])
+    assert np.array_equal(got.view(np.uint8), krows.view(np.uint8))
+    # the freed blocks are reused by the other sequences' next rounds
+    others = [s for s in seqs if s != victim]
+    decode_step(side, others, 1)
+    with pytest.raises(pk.PagedKVError):
+        pk.kv_swap_in(side.pool, victim, hk[:bb], hv[:bb], n_tokens)        # buffer too small
+    pk.kv_swap_in(side.pool, victim, hk, hv, n_tokens)
+    assert side.orc.swap_in(victim, krows, vrows) is not None
+    tables, _, _ = pk.bt_export(side.pool, [victim], nb)
+    assert tables[0].tolist() == side.orc.bm.tables[victim]
+    side.seqs = sorted(side.orc.bm.tables)
+    gpu, ref, _ = decode_step(side, seqs, 2)
+    compare_out(gpu, ref, "fp8" if dt == "fp8" else dt)
+    check_pool_bytes(side)
