@@ -94,6 +94,8 @@ typedef struct {
     int64_t logical_tokens;   /* sum of sequence lengths (a shared token counts per sequence) */
     int64_t table_slots;      /* sum over sequences of |table| * block_size */
     int64_t cow_count;        /* copy-on-write events since the last bt_reset */
+    int64_t prefix_hit_tokens;/* prompt tokens found in the prefix cache since the last bt_reset */
+    int64_t cached_blocks;    /* blocks registered in the prefix cache (in use or free) */
 } pkv_stats;
 
 typedef struct {
@@ -170,6 +172,29 @@ pkv_status bt_append(pkv_pool* pool, int64_t seq_id, int32_t* slot_out,
  *   Errors: INVALID_ARG, UNKNOWN_SEQ, NO_BLOCKS (state unchanged). */
 pkv_status bt_append_batch(pkv_pool* pool, const int64_t* seq_ids, int n, int32_t* slots_out,
                            int32_t* cow_src_out, int32_t* cow_dst_out, int* n_cow_out);
+
+/* bt_set_prefix_caching - turns automatic prefix caching on (1) or off (0,
+ *   which forgets every registration) ([F55] §后来的做法: each full block is
+ *   hashed over its tokens and everything before it; a new request with the
+ *   same beginning uses the existing blocks; it saves prompt processing only).
+ *   Off by default.  Errors: INVALID_ARG. */
+pkv_status bt_set_prefix_caching(pkv_pool* pool, int enable);
+
+/* bt_alloc_prefix - bt_alloc with the prompt's token ids (host [n_tokens]).
+ *   With prefix caching on, the longest run of leading full blocks whose
+ *   tokens - and all tokens before them - match a registered block is taken
+ *   over (refcount + 1; a registered free block leaves the free queue), the
+ *   rest comes from the free queue, and the new full blocks are registered.
+ *   Registration key: FNV-1a 64 over (parent key, 8 bytes little endian, 0 for
+ *   the first block) followed by the block's token ids (4 bytes little endian
+ *   each); a hit is confirmed against the stored token ids.  A block handed
+ *   out as a fresh block loses its registration.  *n_cached_out receives the
+ *   number of leading tokens whose keys and values are already in the pool
+ *   (a multiple of block_size): the caller appends only tokens
+ *   [*n_cached_out, n_tokens).  slot_mapping_out gets all n_tokens slots.
+ *   Errors: INVALID_ARG, SEQ_EXISTS, NO_BLOCKS (nothing changed). */
+pkv_status bt_alloc_prefix(pkv_pool* pool, int64_t seq_id, const int32_t* token_ids, int n_tokens,
+                           int32_t* slot_mapping_out, int32_t* n_cached_out);
 
 /* bt_fork - child_id gets parent_id's table; every block's refcount + 1
  *   ([IPLEX]: two samples of one prompt point at the same input blocks).
@@ -401,6 +426,58 @@ pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dt
 
 /* paged_decode_static_scratch_bytes - size of the static scratch array. */
 size_t paged_decode_static_scratch_bytes(void);
+
+/* ---------------------------------------------------------------------------
+ * The exhibit's allocation bench on the host ([F55] §实验台): requests arrive,
+ * write their prompt at once and one token per round, and leave; those that
+ * do not fit wait (first come, first served).  Paged memory (block_size > 0,
+ * the block manager's rules) against the contiguous reservations of
+ * [F55] §先占好最长的位置 / §三种浪费, each one run of slots taken up front at
+ * the first place it fits:
+ *   PKV_SIM_MAX    (0)  max_len slots per request;
+ *   PKV_SIM_POW2   (-1) the next power of two >= the request's final length,
+ *                       at most max_len (over-reserves by less than 2x);
+ *   PKV_SIM_ORACLE (-2) exactly the final length (needs the output length in
+ *                       advance, which a real server does not know).
+ * ------------------------------------------------------------------------- */
+#define PKV_SIM_MAX 0
+#define PKV_SIM_POW2 (-1)
+#define PKV_SIM_ORACLE (-2)
+
+typedef struct {
+    int32_t arrival;   /* round the request arrives (non-decreasing over the array) */
+    int32_t prompt;    /* prompt tokens, >= 1 */
+    int32_t output;    /* tokens to generate, >= 1; prompt + output <= max_len */
+} pkv_sim_request;
+
+typedef struct {
+    int32_t rounds;             /* rounds until every request has left */
+    int32_t peak_running;       /* most requests holding memory in one round */
+    int32_t preemptions;        /* paged: requests that gave up their blocks */
+    int32_t admitted;           /* admissions (a preempted request is admitted again) */
+    int64_t stored_token_rounds;   /* sum over rounds of tokens stored */
+    int64_t reserved_slot_rounds;  /* sum over rounds of slots held */
+    int64_t future_slot_rounds;    /* ... of held slots its request writes later
+                                      (the "reservation" waste) */
+    int64_t internal_frag_slot_rounds; /* ... of held slots its request never
+                                          writes (internal fragmentation) */
+    double mean_utilisation;    /* mean over rounds (with slots held) of stored / held */
+} pkv_sim_result;
+
+/* pkv_simulate - runs the bench.  Each round: (1) admission in arrival order
+ *   while the head fits; (2) every request admitted earlier writes one token -
+ *   paged growth that finds no block preempts the most recently admitted
+ *   running request ([F55] §放不下的时候), which rejoins the head of the queue
+ *   and comes back with its written tokens as its new prompt (recomputation);
+ *   (3) finished requests leave.  Readouts are taken after (2).
+ *   block_size: > 0 paged, or one of PKV_SIM_MAX / _POW2 / _ORACLE.
+ *   running_per_round (may be NULL) receives the number of requests holding
+ *   memory in each round (capacity max_rounds).
+ *   Errors: INVALID_ARG (bad request, num_slots not a multiple of block_size,
+ *   unknown mode, or not finished within max_rounds). */
+pkv_status pkv_simulate(const pkv_sim_request* requests, int n, int num_slots, int block_size,
+                        int max_len, int max_rounds, pkv_sim_result* out,
+                        int32_t* running_per_round);
 
 /* pkv_device_error - synchronises the stream, returns the device error word's
  *   bits in *bits_out (may be NULL) and clears it.  Returns PKV_ERR_DEVICE if

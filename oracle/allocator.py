@@ -34,6 +34,20 @@ Readings of what the pages leave open:
 * Batched appends are processed in the given order; a batch is all-or-nothing
   (on NO_BLOCKS nothing changes), mirroring the all-or-nothing rule for a
   sequence's blocks in §放不下的时候.
+
+Automatic prefix caching (§后来的做法: each full block is hashed over its own
+tokens and everything before it, and a new request that starts the same way
+uses the existing blocks; it saves prompt processing only).  Readings:
+
+* Only full blocks of a prompt are registered; the key of block i is FNV-1a 64
+  (the published Fowler-Noll-Vo 1a hash: offset basis 14695981039346656037,
+  prime 1099511628211, one byte at a time) over the key of block i-1 (8 bytes
+  little endian, 0 for block 0) followed by block i's token ids (4 bytes
+  little endian each); a key hit is confirmed against the stored token ids.
+* A new prompt takes over the longest run of leading full blocks that hit;
+  the first miss ends the run.  A hit on a freed block takes it back out of
+  the free queue.  Blocks freed by their last user stay registered until they
+  are handed out again as fresh blocks.
 """
 
 from __future__ import annotations
@@ -55,6 +69,24 @@ class AllocError(Exception):
         self.status = status
 
 
+FNV_OFFSET = 14695981039346656037
+FNV_PRIME = 1099511628211
+
+
+def fnv1a64(data: bytes) -> int:
+    h = FNV_OFFSET
+    for byte in data:
+        h ^= byte
+        h = (h * FNV_PRIME) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def block_key(parent: int, tokens: Sequence[int]) -> int:
+    data = parent.to_bytes(8, "little") + b"".join(
+        (int(t) & 0xFFFFFFFF).to_bytes(4, "little") for t in tokens)
+    return fnv1a64(data)
+
+
 class BlockManager:
     """Block tables, fill counts, refcounts and a FIFO free queue."""
 
@@ -73,6 +105,10 @@ class BlockManager:
         self.tables: Dict[int, List[int]] = {}
         self.lengths: Dict[int, int] = {}
         self.cow_count = 0
+        self.caching = False
+        self.registered: Dict[int, tuple] = {}   # block -> (key, tokens)
+        self.by_key: Dict[int, int] = {}
+        self.hit_tokens = 0
 
     # -- helpers -----------------------------------------------------------
     def _fill_last(self, seq: int) -> int:
@@ -86,7 +122,65 @@ class BlockManager:
         b = self.free.popleft()
         assert self.refcount[b] == 0
         self.refcount[b] = 1
+        self._unregister(b)          # handed out fresh: its old contents go
         return b
+
+    def _unregister(self, b: int) -> None:
+        if b in self.registered:
+            key, _ = self.registered.pop(b)
+            if self.by_key.get(key) == b:
+                del self.by_key[key]
+
+    def set_prefix_caching(self, on: bool) -> None:
+        self.caching = bool(on)
+        if not on:
+            self.registered.clear()
+            self.by_key.clear()
+
+    def alloc_prefix(self, seq: int, tokens: Sequence[int]):
+        """Admission with the prompt's token ids.  Returns (slots, n_cached)."""
+        tokens = [int(t) for t in tokens]
+        n = len(tokens)
+        if not self.caching:
+            return self.alloc(seq, n), 0
+        if seq in self.tables:
+            raise AllocError(SEQ_EXISTS, str(seq))
+        bs = self.block_size
+        need = (n + bs - 1) // bs
+        full = n // bs
+        keys, hits = [], []
+        parent = 0
+        hitting = True
+        for i in range(full):
+            blk = tokens[i * bs:(i + 1) * bs]
+            key = block_key(parent, blk)
+            keys.append(key)
+            parent = key
+            if hitting:
+                b = self.by_key.get(key)
+                if b is not None and self.registered[b][1] == blk:
+                    hits.append(b)
+                else:
+                    hitting = False
+        free_hits = sum(1 for b in hits if self.refcount[b] == 0)
+        if need - len(hits) > len(self.free) - free_hits:
+            raise AllocError(NO_BLOCKS, "prefix admission")
+        table = []
+        for b in hits:
+            if self.refcount[b] == 0:
+                self.free.remove(b)
+            self.refcount[b] += 1
+            table.append(b)
+        for i in range(len(hits), need):
+            b = self._pop()
+            table.append(b)
+            if i < full and keys[i] not in self.by_key:
+                self.registered[b] = (keys[i], tokens[i * bs:(i + 1) * bs])
+                self.by_key[keys[i]] = b
+        self.tables[seq] = table
+        self.lengths[seq] = n
+        self.hit_tokens += len(hits) * bs
+        return [table[t // bs] * bs + t % bs for t in range(n)], len(hits) * bs
 
     def _release(self, b: int) -> None:
         self.refcount[b] -= 1
@@ -211,12 +305,16 @@ class BlockManager:
             "logical_tokens": sum(self.lengths.values()),
             "table_slots": sum(len(t) for t in self.tables.values()) * bs,
             "cow_count": self.cow_count,
+            "prefix_hit_tokens": self.hit_tokens,
+            "cached_blocks": len(self.registered),
         }
 
     # -- snapshots for all-or-nothing batches -------------------------------
     def _snapshot(self):
         return (collections.deque(self.free), list(self.refcount),
-                copy.deepcopy(self.tables), dict(self.lengths), self.cow_count)
+                copy.deepcopy(self.tables), dict(self.lengths), self.cow_count,
+                dict(self.registered), dict(self.by_key))
 
     def _restore(self, snap) -> None:
-        self.free, self.refcount, self.tables, self.lengths, self.cow_count = snap
+        (self.free, self.refcount, self.tables, self.lengths, self.cow_count,
+         self.registered, self.by_key) = snap

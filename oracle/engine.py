@@ -68,6 +68,18 @@ class DecodeOracle:
         self.v_rows[seq] = [vs[t] for t in range(v.shape[0])]
         return slots
 
+    def admit_prefix(self, seq: int, tokens, k: np.ndarray, v: np.ndarray, in_dtype: str):
+        """A prompt with token ids and all of its rows; with prefix caching on
+        the allocator may take over registered blocks for its leading full
+        blocks ("KV 缓存与分页注意力" §后来的做法).  The history is the prompt's own
+        rows either way.  Returns (slots, n_cached)."""
+        slots, n_cached = self.bm.alloc_prefix(seq, tokens)
+        ks = self.stored(k, in_dtype, "k")
+        vs = self.stored(v, in_dtype, "v")
+        self.k_rows[seq] = [ks[t] for t in range(k.shape[0])]
+        self.v_rows[seq] = [vs[t] for t in range(v.shape[0])]
+        return slots, n_cached
+
     def fork(self, parent: int, child: int) -> None:
         self.bm.fork(parent, child)
         self.k_rows[child] = list(self.k_rows[parent])

@@ -46,7 +46,8 @@ class pkv_stats(ctypes.Structure):
                 ("free_blocks", ctypes.c_int32), ("used_blocks", ctypes.c_int32),
                 ("num_seqs", ctypes.c_int32), ("pad_", ctypes.c_int32),
                 ("stored_slots", ctypes.c_int64), ("logical_tokens", ctypes.c_int64),
-                ("table_slots", ctypes.c_int64), ("cow_count", ctypes.c_int64)]
+                ("table_slots", ctypes.c_int64), ("cow_count", ctypes.c_int64),
+                ("prefix_hit_tokens", ctypes.c_int64), ("cached_blocks", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_ if f != "pad_"}
@@ -59,6 +60,21 @@ class pkv_pool_info(ctypes.Structure):
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
                 ("k_buf", ctypes.c_void_p), ("v_buf", ctypes.c_void_p),
                 ("bytes_per_buffer", ctypes.c_size_t), ("error_word", ctypes.c_void_p)]
+
+
+class pkv_sim_request(ctypes.Structure):
+    _fields_ = [("arrival", ctypes.c_int32), ("prompt", ctypes.c_int32), ("output", ctypes.c_int32)]
+
+
+class pkv_sim_result(ctypes.Structure):
+    _fields_ = [("rounds", ctypes.c_int32), ("peak_running", ctypes.c_int32),
+                ("preemptions", ctypes.c_int32), ("admitted", ctypes.c_int32),
+                ("stored_token_rounds", ctypes.c_int64), ("reserved_slot_rounds", ctypes.c_int64),
+                ("future_slot_rounds", ctypes.c_int64), ("internal_frag_slot_rounds", ctypes.c_int64),
+                ("mean_utilisation", ctypes.c_double)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
 
 
 _P = ctypes.c_void_p
@@ -84,6 +100,10 @@ _sig("bt_alloc", _st, _P, ctypes.c_int64, ctypes.c_int, _I32P)
 _sig("bt_append", _st, _P, ctypes.c_int64, _I32P, _I32P, _I32P)
 _sig("bt_append_batch", _st, _P, _I64P, ctypes.c_int, _I32P, _I32P, _I32P, ctypes.POINTER(ctypes.c_int))
 _sig("bt_fork", _st, _P, ctypes.c_int64, ctypes.c_int64)
+_sig("bt_set_prefix_caching", _st, _P, ctypes.c_int)
+_sig("pkv_simulate", _st, ctypes.POINTER(pkv_sim_request), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+     ctypes.c_int, ctypes.c_int, ctypes.POINTER(pkv_sim_result), _I32P)
+_sig("bt_alloc_prefix", _st, _P, ctypes.c_int64, _I32P, ctypes.c_int, _I32P, _I32P)
 _sig("bt_free", _st, _P, ctypes.c_int64)
 _sig("bt_export", _st, _P, _I64P, ctypes.c_int, ctypes.c_int, _I32P, _I32P, _I32P)
 _sig("bt_num_blocks", _st, _P, ctypes.c_int64, _I32P)
@@ -123,6 +143,7 @@ EXPORTED = [
     "pkv_device_error", "pkv_status_str", "pkv_step_create", "pkv_step_destroy", "pkv_decode_step",
     "pkv_step_last_launches", "pkv_step_profile", "pkv_step_profile_read",
     "paged_decode_attention_static", "paged_decode_static_scratch_bytes", "kv_swap_out", "kv_swap_in",
+    "bt_set_prefix_caching", "bt_alloc_prefix", "pkv_simulate",
 ]
 
 
@@ -299,6 +320,21 @@ def bt_append_batch(pool: Pool, seq_ids):
     _check(_lib.bt_append_batch(pool.handle, ids.ctypes.data_as(_I64P), n, _ptr32(slots),
                                 _ptr32(src), _ptr32(dst), ctypes.byref(ncow)), "bt_append_batch")
     return slots, src[: ncow.value].copy(), dst[: ncow.value].copy()
+
+
+def bt_set_prefix_caching(pool: Pool, enable: bool) -> None:
+    _check(_lib.bt_set_prefix_caching(pool.handle, 1 if enable else 0), "bt_set_prefix_caching")
+
+
+def bt_alloc_prefix(pool: Pool, seq_id: int, token_ids):
+    """-> (slots [n] int32, n_cached_tokens)."""
+    toks = _i32(token_ids)
+    n = toks.size
+    slots = np.empty(max(n, 1), np.int32)
+    nc = ctypes.c_int32()
+    _check(_lib.bt_alloc_prefix(pool.handle, int(seq_id), _ptr32(toks) if n else None, int(n),
+                                _ptr32(slots) if n else None, ctypes.byref(nc)), "bt_alloc_prefix")
+    return slots[:n].copy(), nc.value
 
 
 def bt_fork(pool: Pool, parent_id: int, child_id: int) -> None:
@@ -527,3 +563,26 @@ def kv_swap_in(pool: Pool, seq_id: int, h_k, h_v, n_tokens: int, stream=None) ->
     cap = min(h_k.numel() * h_k.element_size(), h_v.numel() * h_v.element_size())
     _check(_lib.kv_swap_in(pool.handle, int(seq_id), h_k.data_ptr(), h_v.data_ptr(), cap,
                            int(n_tokens), _stream_ptr(stream)), "kv_swap_in")
+
+
+# ---------------------------------------------------------------------------
+# the exhibit's allocation bench (host only)
+# ---------------------------------------------------------------------------
+SIM_MAX, SIM_POW2, SIM_ORACLE = 0, -1, -2
+
+
+def pkv_simulate(requests, num_slots: int, block_size: int, max_len: int, max_rounds: int = 10000):
+    """requests: sequence of (arrival, prompt, output).  block_size > 0 pages
+    the memory; SIM_MAX (0), SIM_POW2 (-1) or SIM_ORACLE (-2) reserve one
+    contiguous run per request of max_len slots, the next power of two of its
+    final length, or exactly that length.  -> (result dict, running count per
+    round)."""
+    n = len(requests)
+    arr = (pkv_sim_request * max(n, 1))()
+    for i, (a, p, o) in enumerate(requests):
+        arr[i].arrival, arr[i].prompt, arr[i].output = int(a), int(p), int(o)
+    res = pkv_sim_result()
+    per = np.zeros(max_rounds, np.int32)
+    _check(_lib.pkv_simulate(arr, n, num_slots, block_size, max_len, max_rounds, ctypes.byref(res),
+                             _ptr32(per)), "pkv_simulate")
+    return res.as_dict(), per[: res.rounds].copy()

@@ -33,6 +33,7 @@ SOURCES = [
     "api.cu",
     "no_alloc.cu",
     "swap.cu",
+    "simulator.cpp",
 ]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

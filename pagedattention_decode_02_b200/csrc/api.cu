@@ -205,6 +205,16 @@ pkv_status bt_append_batch(pkv_pool* p, const int64_t* seqs, int n, int32_t* slo
     if (!p) return PKV_ERR_INVALID_ARG;
     return p->bm.append_batch(seqs, n, slots, src, dst, n_cow);
 }
+pkv_status bt_set_prefix_caching(pkv_pool* p, int enable) {
+    if (!p || (enable != 0 && enable != 1)) return PKV_ERR_INVALID_ARG;
+    p->bm.set_prefix_caching(enable != 0);
+    return PKV_OK;
+}
+pkv_status bt_alloc_prefix(pkv_pool* p, int64_t seq, const int32_t* tokens, int n_tokens,
+                           int32_t* slots, int32_t* n_cached) {
+    if (!p) return PKV_ERR_INVALID_ARG;
+    return p->bm.alloc_prefix(seq, tokens, n_tokens, slots, n_cached);
+}
 pkv_status bt_fork(pkv_pool* p, int64_t parent, int64_t child) {
     if (!p) return PKV_ERR_INVALID_ARG;
     return p->bm.fork(parent, child);

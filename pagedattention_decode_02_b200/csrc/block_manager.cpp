@@ -7,7 +7,8 @@
 namespace pkv {
 
 BlockManager::BlockManager(int num_blocks, int block_size)
-    : num_blocks_(num_blocks), block_size_(block_size), ring_(num_blocks), ref_(num_blocks, 0) {
+    : num_blocks_(num_blocks), block_size_(block_size), next_(num_blocks, -1),
+      prev_(num_blocks, -1), ref_(num_blocks, 0), hashed_(num_blocks, 0), hash_(num_blocks, 0) {
     reset(nullptr);
 }
 
@@ -20,12 +21,15 @@ pkv_status BlockManager::reset(const int32_t* order) {
             seen[b] = 1;
         }
     }
-    for (int i = 0; i < num_blocks_; ++i) ring_[i] = order ? order[i] : i;
-    head_ = 0;
-    count_ = num_blocks_;
+    head_ = tail_ = -1;
+    count_ = 0;
+    for (int i = 0; i < num_blocks_; ++i) push_back(order ? order[i] : i);
     std::fill(ref_.begin(), ref_.end(), 0);
     seqs_.clear();
     cow_count_ = 0;
+    std::fill(hashed_.begin(), hashed_.end(), 0);
+    by_hash_.clear();
+    hit_tokens_ = 0;
     return PKV_OK;
 }
 
@@ -34,27 +38,158 @@ int BlockManager::fill_of_last(const Sequence& s) const {
     return (int)(s.length - (int64_t)(s.blocks.size() - 1) * block_size_);
 }
 
-int32_t BlockManager::pop_front() {
-    int32_t b = ring_[head_];
-    head_ = (head_ + 1) % num_blocks_;
+void BlockManager::push_back(int32_t b) {
+    next_[b] = -1;
+    prev_[b] = tail_;
+    if (tail_ >= 0) next_[tail_] = b; else head_ = b;
+    tail_ = b;
+    ++count_;
+}
+
+void BlockManager::remove_free(int32_t b) {
+    if (prev_[b] >= 0) next_[prev_[b]] = next_[b]; else head_ = next_[b];
+    if (next_[b] >= 0) prev_[next_[b]] = prev_[b]; else tail_ = prev_[b];
+    next_[b] = prev_[b] = -1;
     --count_;
+}
+
+// a block handed out as a fresh block loses its registration
+int32_t BlockManager::pop_front() {
+    const int32_t b = head_;
+    remove_free(b);
+    unregister(b);
     ref_[b] = 1;
     return b;
 }
 
 void BlockManager::unpop_front(int32_t b) {
-    head_ = (head_ + num_blocks_ - 1) % num_blocks_;
-    ring_[head_] = b;
+    next_[b] = head_;
+    prev_[b] = -1;
+    if (head_ >= 0) prev_[head_] = b; else tail_ = b;
+    head_ = b;
     ++count_;
     ref_[b] = 0;
 }
 
-void BlockManager::push_back(int32_t b) {
-    ring_[(head_ + count_) % num_blocks_] = b;
-    ++count_;
+void BlockManager::unregister(int32_t b) {
+    if (!hashed_[b]) return;
+    auto it = by_hash_.find(hash_[b]);
+    if (it != by_hash_.end() && it->second == b) by_hash_.erase(it);
+    hashed_[b] = 0;
+    dropped_.emplace_back(b, hash_[b]);
+}
+
+void BlockManager::restore_dropped() {
+    for (auto r = dropped_.rbegin(); r != dropped_.rend(); ++r) {
+        hashed_[r->first] = 1;
+        hash_[r->first] = r->second;
+        by_hash_[r->second] = r->first;
+    }
+    dropped_.clear();
+}
+
+int32_t BlockManager::lookup(uint64_t h, const int32_t* tokens) const {
+    auto it = by_hash_.find(h);
+    if (it == by_hash_.end()) return -1;
+    const int32_t b = it->second;
+    const int32_t* bt = block_tokens_.data() + (size_t)b * block_size_;
+    for (int i = 0; i < block_size_; ++i)
+        if (bt[i] != tokens[i]) return -1;   // a hash collision: not the same tokens
+    return b;
+}
+
+void BlockManager::set_prefix_caching(bool on) {
+    caching_ = on;
+    if (on && block_tokens_.empty()) block_tokens_.assign((size_t)num_blocks_ * block_size_, 0);
+    if (!on) {
+        std::fill(hashed_.begin(), hashed_.end(), 0);
+        by_hash_.clear();
+    }
+}
+
+namespace {
+// FNV-1a, 64 bit (offset basis 14695981039346656037, prime 1099511628211),
+// over the parent hash (8 bytes, little endian) and the block's token ids
+// (4 bytes each, little endian): the chain hash of a full block.
+uint64_t chain_hash(uint64_t parent, const int32_t* tokens, int n) {
+    uint64_t h = 14695981039346656037ull;
+    auto eat = [&h](uint8_t byte) {
+        h ^= byte;
+        h *= 1099511628211ull;
+    };
+    for (int i = 0; i < 8; ++i) eat((uint8_t)(parent >> (8 * i)));
+    for (int t = 0; t < n; ++t) {
+        const uint32_t v = (uint32_t)tokens[t];
+        for (int i = 0; i < 4; ++i) eat((uint8_t)(v >> (8 * i)));
+    }
+    return h;
+}
+}  // namespace
+
+pkv_status BlockManager::alloc_prefix(int64_t seq, const int32_t* tokens, int n_tokens,
+                                      int32_t* slots, int32_t* n_cached) {
+    if (n_tokens < 0 || (n_tokens > 0 && (!slots || !tokens)) || !n_cached)
+        return PKV_ERR_INVALID_ARG;
+    if (!caching_) {
+        const pkv_status st = alloc(seq, n_tokens, slots);
+        if (st == PKV_OK) *n_cached = 0;
+        return st;
+    }
+    dropped_.clear();
+    if (seqs_.count(seq)) return PKV_ERR_SEQ_EXISTS;
+    const int bs = block_size_;
+    const int need = (n_tokens + bs - 1) / bs;
+    const int full = n_tokens / bs;
+    // leading full blocks already registered with the same tokens
+    std::vector<int32_t> hits;
+    std::vector<uint64_t> hashes((size_t)full);
+    uint64_t parent = 0;
+    int free_hits = 0;
+    bool hitting = true;
+    for (int i = 0; i < full; ++i) {
+        hashes[i] = chain_hash(parent, tokens + (size_t)i * bs, bs);
+        parent = hashes[i];
+        if (hitting) {
+            const int32_t b = lookup(hashes[i], tokens + (size_t)i * bs);
+            if (b >= 0) {
+                hits.push_back(b);
+                free_hits += ref_[b] == 0;
+            } else {
+                hitting = false;
+            }
+        }
+    }
+    const int fresh = need - (int)hits.size();
+    if (fresh > count_ - free_hits) return PKV_ERR_NO_BLOCKS;
+    Sequence s;
+    s.blocks.reserve((size_t)need);
+    for (int32_t b : hits) {
+        if (ref_[b] == 0) remove_free(b);
+        ++ref_[b];
+        s.blocks.push_back(b);
+    }
+    for (int i = (int)hits.size(); i < need; ++i) {
+        const int32_t b = pop_front();
+        s.blocks.push_back(b);
+        if (i < full && !by_hash_.count(hashes[i])) {
+            hashed_[b] = 1;
+            hash_[b] = hashes[i];
+            by_hash_[hashes[i]] = b;
+            std::copy(tokens + (size_t)i * bs, tokens + (size_t)(i + 1) * bs,
+                      block_tokens_.begin() + (size_t)b * bs);
+        }
+    }
+    s.length = n_tokens;
+    s.epoch = next_epoch_++;
+    for (int t = 0; t < n_tokens; ++t) slots[t] = s.blocks[t / bs] * bs + t % bs;
+    *n_cached = (int32_t)hits.size() * bs;
+    hit_tokens_ += *n_cached;
+    seqs_.emplace(seq, std::move(s));
+    return PKV_OK;
 }
 
 pkv_status BlockManager::alloc(int64_t seq, int n_tokens, int32_t* slots) {
+    dropped_.clear();
     if (n_tokens < 0 || (n_tokens > 0 && !slots)) return PKV_ERR_INVALID_ARG;
     if (seqs_.count(seq)) return PKV_ERR_SEQ_EXISTS;
     const int64_t need = ((int64_t)n_tokens + block_size_ - 1) / block_size_;
@@ -130,6 +265,7 @@ pkv_status BlockManager::append_batch(const int64_t* seqs, int n, int32_t* slots
                                       int32_t* cow_dst, int* n_cow) {
     if (n < 0 || (n > 0 && (!seqs || !slots || !cow_src || !cow_dst)) || !n_cow)
         return PKV_ERR_INVALID_ARG;
+    dropped_.clear();
     std::vector<Undo> log;
     log.reserve((size_t)n);
     int pairs = 0;
@@ -139,6 +275,7 @@ pkv_status BlockManager::append_batch(const int64_t* seqs, int n, int32_t* slots
         pkv_status st = append_one(seqs[i], &slots[i], &src, &dst, &u);
         if (st != PKV_OK) {
             for (auto r = log.rbegin(); r != log.rend(); ++r) undo_one(*r);
+            restore_dropped();
             return st;
         }
         log.push_back(u);
@@ -178,6 +315,7 @@ void BlockManager::undo_alloc(int64_t seq) {
     const std::vector<int32_t>& b = it->second.blocks;
     for (auto r = b.rbegin(); r != b.rend(); ++r) unpop_front(*r);
     seqs_.erase(it);
+    restore_dropped();
 }
 
 pkv_status BlockManager::export_tables(const int64_t* seqs, int n, int max_blocks, int32_t* tables,
@@ -229,7 +367,8 @@ pkv_status BlockManager::refcount_of(int32_t block, int32_t* out) const {
 
 pkv_status BlockManager::free_queue(int32_t* out, int cap, int* n_out) const {
     if (!n_out || cap < count_ || (count_ > 0 && !out)) return PKV_ERR_INVALID_ARG;
-    for (int i = 0; i < count_; ++i) out[i] = ring_[(head_ + i) % num_blocks_];
+    int i = 0;
+    for (int32_t b = head_; b >= 0; b = next_[b]) out[i++] = b;
     *n_out = count_;
     return PKV_OK;
 }
@@ -255,6 +394,8 @@ void BlockManager::stats(pkv_stats* out) const {
     }
     for (int32_t f : fill) st.stored_slots += f;
     st.cow_count = cow_count_;
+    st.prefix_hit_tokens = hit_tokens_;
+    for (uint8_t h : hashed_) st.cached_blocks += h;
     *out = st;
 }
 

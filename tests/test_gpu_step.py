@@ -200,3 +200,51 @@ def test_swap_out_and_in(dt, bs):
     gpu, ref, _ = decode_step(side, seqs, 2)
     compare_out(gpu, ref, "fp8" if dt == "fp8" else dt)
     check_pool_bytes(side)
+
+
+@pytest.mark.parametrize("bs", [4, 16])
+def test_prefix_cached_prompts(bs):
+    # "KV 缓存与分页注意力" section 后来的做法: prompts that start with the same tokens
+    # share the registered blocks; the rows of a token depend on its prefix
+    # (as a model's would), so the shared blocks hold exactly the rows each
+    # sharer would have written; only the uncached tail is appended
+    import dataclasses
+    import zlib
+    cfg = dataclasses.replace(wl.CONFIGS["opt13b"], n_q_heads=2, n_kv_heads=2, block_size=bs,
+                              batch=4, lengths=("fixed", 0), min_pool_blocks=0)
+    from paged_harness import make_pair, decode_step
+    side = make_pair(cfg, 128, np.random.default_rng(3).permutation(128).astype(np.int32))
+    pk.bt_set_prefix_caching(side.pool, True)
+    side.orc.bm.set_prefix_caching(True)
+    rnd = np.random.default_rng(5)
+    system = rnd.integers(0, 50, size=4 * bs + 3).tolist()
+    prompts = [system + rnd.integers(0, 50, size=5).tolist(),
+               system[: 4 * bs] + rnd.integers(0, 50, size=7).tolist(),
+               system[: 2 * bs + 1] + rnd.integers(0, 50, size=2 * bs).tolist(),
+               rnd.integers(0, 50, size=3 * bs).tolist()]
+
+    def rows(tokens):
+        out_k, out_v = [], []
+        for j in range(len(tokens)):
+            key = zlib.crc32(np.asarray(tokens[: j + 1], np.int32).tobytes())
+            g = np.random.default_rng([11, key])
+            out_k.append(g.standard_normal((2, 128), dtype=np.float32))
+            out_v.append(g.standard_normal((2, 128), dtype=np.float32))
+        return wl.round_to(np.stack(out_k), "f16"), wl.round_to(np.stack(out_v), "f16")
+
+    cached = []
+    for s, toks in enumerate(prompts):
+        k, v = rows(toks)
+        slots, n_cached = pk.bt_alloc_prefix(side.pool, s, toks)
+        o_slots, o_cached = side.orc.admit_prefix(s, toks, k, v, "f16")
+        assert slots.tolist() == o_slots and n_cached == o_cached
+        cached.append(n_cached)
+        if n_cached < len(toks):
+            pk.kv_append(side.pool, torch.from_numpy(slots[n_cached:].copy()).cuda(),
+                         to_torch(k[n_cached:], "f16"), to_torch(v[n_cached:], "f16"))
+        side.seqs.append(s)
+    assert cached == [0, 4 * bs, 2 * bs, 0]
+    assert pk.bt_stats(side.pool)["prefix_hit_tokens"] == 6 * bs
+    gpu, ref, _ = decode_step(side, [0, 1, 2, 3], 0)
+    compare_out(gpu, ref, "f16")
+    check_pool_bytes(side)

@@ -247,3 +247,22 @@ def describe(cfg: Config, seed: int = 0, variant: Optional[str] = None) -> dict:
     if variant:
         d["variant"] = variant
     return d
+
+
+# ---------------------------------------------------------------------------
+# the exhibit's allocation bench
+# ---------------------------------------------------------------------------
+
+EXHIBIT_SLOTS = 176      # 44 blocks of 4 token slots
+EXHIBIT_MAX_LEN = 20     # longest sequence, tokens
+EXHIBIT_MODES = (1, 2, 4, 8, 16, 0)   # block sizes, and 0 for the max-length reservation
+
+
+def exhibit_requests(n: int, seed: int = 0, per_round: int = 2, max_len: int = EXHIBIT_MAX_LEN):
+    """n requests (arrival round, prompt, output), per_round arriving each
+    round; final length uniform on [2, max_len], prompt uniform on [1, length-1]
+    (the exhibit draws lengths at random, not from a trace)."""
+    rng = _rng(seed, 4242, n, per_round)
+    total = rng.integers(2, max_len + 1, size=n)
+    prompt = np.array([rng.integers(1, t) for t in total], dtype=np.int64)
+    return [(i // per_round, int(p), int(t - p)) for i, (p, t) in enumerate(zip(prompt, total))]
