@@ -41,6 +41,7 @@ import workloads as wl  # noqa: E402
 METRIC = "paged decode KV GB/s (% of B200 HBM peak); attended tokens/sec at 1 GPU"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -58,6 +59,9 @@ def parse():
     ap.add_argument("--kernel", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
+                    help="prefill: the prompt phase of the workload's batch (every history "
+                         "attended causally as one prompt)")
     return ap.parse_args()
 
 
@@ -66,6 +70,38 @@ def config_of(args) -> wl.Config:
     if args.block_size:
         cfg = cfg.with_block_size(args.block_size)
     return cfg
+
+
+# DRAM traffic of the decode kernel per launch, as a multiple of its
+# algorithmic KV bytes, from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum) of the same workload with one replica batch; the
+# summary and the command are under profiles/.  Valid only while the kernel's
+# sources hash to the recorded value, else the bench reports null.
+TRAFFIC = {
+    # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
+}
+KERNEL_SOURCES = {
+    "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
+    "decode_tc_kernel": ("decode_tc.cu", "tc_common.cuh", "kernels_common.cuh"),
+    "decode_simt2_kernel": ("decode_simt2.cu", "kernels_common.cuh"),
+    "decode_simt_kernel": ("decode_simt.cu", "kernels_common.cuh"),
+}
+
+
+def kernel_sources_sha(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, ()):
+        with open(os.path.join(ROOT, "pagedattention_decode_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch(cfg_name: str, kernel: str, algorithmic_bytes: float):
+    entry = TRAFFIC.get((cfg_name, kernel))
+    if entry is None or entry[1] != kernel_sources_sha(kernel):
+        return None
+    return int(entry[0] * algorithmic_bytes)
 
 
 def peaks():
@@ -392,6 +428,7 @@ def run_ours(args) -> None:
     clocks.stop()
     pd.barrier()
     elapsed_ms = ev0.elapsed_time(ev1)
+    kernel_used = step.last_kernel
     pro_ms, dec_ms, merge_ms = pk.pkv_step_profile_read(step, K)
     pk.pkv_step_profile(step, 0)
     prof_bytes = step_bytes[::prof_every][: len(dec_ms)]
@@ -399,11 +436,14 @@ def run_ours(args) -> None:
     # end to end through the public API with host buffers: per round the new
     # q/k/v arrive from pinned host memory and the output goes back to the host
     # (a serving loop needs it before the next round)
-    hq = q[0].cpu().pin_memory()
-    hk = kn[0].cpu().pin_memory()
-    hv = vn[0].cpu().pin_memory()
+    # q | k | v of a round travel in one pinned buffer and one copy
+    nq, nk = q[0].numel(), kn[0].numel()
+    hqkv = torch.cat([q[0].flatten(), kn[0].flatten(), vn[0].flatten()]).cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=dt).pin_memory()
-    dq, dk, dv = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    dqkv = torch.empty_like(hqkv, device="cuda")
+    dq = dqkv[:nq].view(q[0].shape)
+    dk = dqkv[nq:nq + nk].view(kn[0].shape)
+    dv = dqkv[nq + nk:].view(vn[0].shape)
     stream = torch.cuda.current_stream()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -413,9 +453,7 @@ def run_ours(args) -> None:
     for k in range(W + K, W + K + E):
         r = k % R
         ctx[r] += 1
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
+        dqkv.copy_(hqkv, non_blocking=True)
         pk.pkv_decode_step(step, groups[r], dq, dk, dv, scale, out)
         hout.copy_(out, non_blocking=True)
         stream.synchronize()
@@ -423,7 +461,7 @@ def run_ours(args) -> None:
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
+    h2d = hqkv.numel() * hqkv.element_size()
     d2h = hout.numel() * hout.element_size()
 
     bits = pk.pkv_device_error(pool)
@@ -451,14 +489,8 @@ def run_ours(args) -> None:
         peak, peak_kind = peaks()
         dec_total_ms = float(np.sum(dec_ms))
         achieved = float(np.sum(prof_bytes)) / (dec_total_ms / 1e3) / 1e9
-        traffic = None
-        tr_path = os.path.join(ROOT, "profiles", f"traffic_{cfg.name}.json")
-        if os.path.exists(tr_path):
-            try:
-                with open(tr_path) as f:
-                    traffic = json.load(f).get("bytes_per_launch")
-            except Exception:
-                traffic = None
+        kernel_name = pk.KERNEL_NAMES.get(kernel_used, "unknown")
+        traffic = traffic_per_launch(cfg.name, kernel_name, float(np.mean(step_bytes)))
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -488,7 +520,7 @@ def run_ours(args) -> None:
             "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS / world, 2),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "paged decode kernel (split partitions merged in-kernel where supported)",
+                "kernel": kernel_name,
                 "achieved": round(achieved, 2),
                 "peak": peak,
                 "peak_kind": peak_kind,
@@ -523,10 +555,121 @@ def run_ours(args) -> None:
     pd.finish()
 
 
+def peak_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def run_prefill(args) -> None:
+    """Prompt phase ("KV 缓存与分页注意力" §一次写一个词元: a whole prompt at once)
+    of one batch of the workload: every sequence's history is its prompt, its
+    keys and values already in the pool, attended causally through the block
+    table.  FLOPs count the unmasked (query, key) pairs: 4 d per pair per
+    query head."""
+    import torch
+
+    import pagedattention_decode_02_b200 as pk
+
+    torch.cuda.set_device(0)
+    cfg = config_of(args)
+    K, W = args.steps, args.warmup
+    pool, groups, ctx = build_batches(cfg, pk, torch, 1, 0, seed=0)
+    seqs, lens = groups[0], ctx[0]
+    max_blocks = max(pk.bt_num_blocks(pool, int(s)) for s in seqs)
+    tables, lens_i32, _ = pk.bt_export(pool, seqs, max_blocks)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16}[cfg.q_dtype]
+    rows = int(lens.sum())
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(99)
+    q = torch.randn((rows, cfg.n_q_heads, cfg.head_dim), generator=gen, device="cuda").to(dt)
+    out = torch.empty_like(q)
+    starts = torch.from_numpy(np.concatenate([[0], np.cumsum(lens_i32)]).astype(np.int32)).cuda()
+    t_tab = torch.from_numpy(tables).cuda()
+    t_len = torch.from_numpy(lens_i32).cuda()
+    max_q = int(lens_i32.max())
+    pairs = float(np.sum(lens.astype(np.float64) * (lens + 1) / 2))
+    flops = 4.0 * cfg.head_dim * cfg.n_q_heads * pairs
+    kv_bytes = float(lens.sum()) * cfg.kv_bytes_per_token
+
+    def call():
+        pk.paged_prefill_attention(pool, q, starts, t_tab, t_len, cfg.scale, max_q_len=max_q,
+                                   out=out)
+
+    for _ in range(W):
+        call()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    ev0.record()
+    for _ in range(K):
+        call()
+    ev1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    ms = ev0.elapsed_time(ev1) / K
+    # end to end: the prompt's queries from pinned host memory, the output back
+    hq = q.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=dt).pin_memory()
+    E = max(3, K // 3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record()
+    for _ in range(E):
+        q.copy_(hq, non_blocking=True)
+        call()
+        hout.copy_(out, non_blocking=True)
+        stream.synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if pk.pkv_device_error(pool):
+        raise SystemExit("device error")
+    peak, kind = peak_tflops()
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "paged prefill attention TFLOP/s (causal, unmasked query-key pairs)",
+        "value": round(achieved, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.q_dtype,
+        "data": "synthetic (seeded torch.randn q/K/V; lengths from workloads.py)",
+        "config": {"workload": "prompt phase of " + cfg.description, "rows": rows,
+                   "mean_prompt": round(float(lens.mean()), 1),
+                   "l2": f"no flush: each call reads {kv_bytes / 1e6:.0f} MB of K/V "
+                         "and writes the output; the K/V of one (sequence, head) is re-read "
+                         "by its row tiles from L2"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "kernel": "prefill_tc_kernel",
+                     "flops_per_launch": flops, "note": "mma.sync m16n8k16 tensor path"},
+        "e2e": {"value": round(flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(hq.numel() * hq.element_size()),
+                "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": K,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "prefill":
+        run_prefill(args)
     else:
         run_ours(args)
 

@@ -281,13 +281,19 @@ pkv_status paged_decode_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_d
 size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, int max_blocks);
 
 /* Kernel selection for paged_decode_attention_ex. */
-#define PKV_KERNEL_AUTO 0          /* TENSOR when supported, else SIMT */
+#define PKV_KERNEL_AUTO 0          /* LEAN for grouped heads (G > 1) when supported, the workspace
+                                      holds its state and partition_tokens is 0; else TENSOR when
+                                      supported; else SIMT */
 #define PKV_KERNEL_SIMT 1          /* CUDA-core dot products: SIMT_TMA when supported, else SIMT_BULK */
 #define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads: F16/BF16 pools with
                                       head_dim 64 or 128, power-of-two block size, 1 < G <= 128 */
 #define PKV_KERNEL_SIMT_BULK 3     /* CUDA-core, 1-D bulk copies per block run (any shape) */
 #define PKV_KERNEL_SIMT_TMA 4      /* CUDA-core, swizzled 2-D TMA boxes, one query head per CTA:
                                       rows of 128/256/512 bytes, power-of-two block size */
+#define PKV_KERNEL_LEAN 5          /* tensor cores, one wave of persistent CTAs sharing the batch's
+                                      16-token stages equally, split pairs merged in the kernel:
+                                      F16/BF16 pools with head_dim 64 or 128, power-of-two block
+                                      size, 1 <= G <= 128, B <= 2048; ignores partition_tokens */
 
 /* paged_decode_attention_ex - paged_decode_attention with explicit choices:
  *   partition_tokens: 0 = automatic, > 0 = tokens per partition (a multiple
@@ -351,6 +357,11 @@ pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const 
 /* pkv_step_last_launches - number of kernels the last pkv_decode_step call
  *   launched (copy-on-write copy, append, decode, merge). */
 int pkv_step_last_launches(const pkv_step* step);
+
+/* pkv_step_last_kernel - the decode kernel (PKV_KERNEL_LEAN, _TENSOR,
+ *   _SIMT_TMA or _SIMT_BULK) the last pkv_decode_step call ran, after the
+ *   automatic choice; 0 before the first call or for an empty batch. */
+int pkv_step_last_kernel(const pkv_step* step);
 
 /* pkv_step_profile - n > 0: every `every`-th later pkv_decode_step call (the
  *   first one included) records CUDA events on its stream before the round's
@@ -423,6 +434,32 @@ pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dt
                                          const int32_t* d_context_lens, int B, int n_q_heads,
                                          float scale, void* d_out, int partition_tokens,
                                          void* stream);
+
+/* paged_prefill_attention - the prompt phase's attention over the paged cache
+ *   ([F55] §一次写一个词元: the whole prompt is computed at once).  Sequence i's
+ *   prompt tokens are rows d_q_starts[i] .. d_q_starts[i+1]-1 of d_q and
+ *   d_out; with n_i = d_q_starts[i+1] - d_q_starts[i] they are the last n_i of
+ *   its d_context_lens[i] = c_i cached tokens, whose keys and values are
+ *   already stored (bt_alloc / bt_alloc_prefix slots, kv_append).  Tokens
+ *   before them - a cached prefix ([F55] §后来的做法) or a recomputed history -
+ *   are attended as well.  For row t of sequence i and query head h, with
+ *   g = floor(h / G) and position P = c_i - n_i + t:
+ *     out[t][h] = sum_{j <= P} softmax_j(scale * <q[t][h], K_i[g][j]>) V_i[g][j].
+ *   d_q, d_out: device [d_q_starts[B]][n_q_heads][head_dim] in the pool dtype
+ *   (F16 or BF16 pools with head_dim 64 or 128 and a power-of-two block size;
+ *   other pools return INVALID_ARG).  d_q_starts: device int32 [B + 1],
+ *   non-decreasing from 0.  d_block_tables: device int32 [B][max_blocks];
+ *   d_context_lens: device int32 [B].  max_q_len >= every n_i (it sizes the
+ *   grid).  n_i == 0 writes nothing.  A length outside [1, max_blocks * bs],
+ *   n_i > c_i or n_i > max_q_len sets PKV_DEVERR_CONTEXT_LEN (that sequence's
+ *   rows are zero where the grid covers them); a block id outside
+ *   [0, num_blocks) sets PKV_DEVERR_BLOCK_ID and zeroes the affected 64-row
+ *   tile.  No workspace.  Errors: INVALID_ARG, CUDA. */
+pkv_status paged_prefill_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
+                                   const int32_t* d_q_starts, int max_q_len,
+                                   const int32_t* d_block_tables, int max_blocks,
+                                   const int32_t* d_context_lens, int B, int n_q_heads,
+                                   float scale, void* d_out, void* stream);
 
 /* paged_decode_static_scratch_bytes - size of the static scratch array. */
 size_t paged_decode_static_scratch_bytes(void);

@@ -81,3 +81,42 @@ def attention_weights(q: np.ndarray, k_hist: np.ndarray, scale: float) -> np.nda
     """softmax(scale * K q) for one head: [c] weights (for the sum-to-one and
     special-case checks)."""
     return softmax(scale * (np.asarray(k_hist, np.float64) @ np.asarray(q, np.float64)))
+
+
+def prefill_attention(q: np.ndarray, k_hist: np.ndarray, v_hist: np.ndarray,
+                      scale: float) -> np.ndarray:
+    """Prompt-phase attention of one sequence over its paged cache.
+
+    "KV 缓存与分页注意力", §一次写一个词元: the prompt phase computes the whole
+    prompt at once.  Its n tokens are the last n of the history (their keys and
+    values already stored, after any cached prefix: §后来的做法, or after a
+    preemption whose prompt and written tokens are recomputed as one new
+    prompt: §放不下的时候).  Token t of them, at position c - n + t, attends to
+    positions 0 .. c - n + t, itself included (causal):
+
+        out[t][h] = sum_{j <= c-n+t} softmax_j(scale * <q[t][h], K_{g,j}>) V_{g,j}
+
+    q [n][H_q][d]; k_hist, v_hist [c][H_kv][d] with c >= n.  Returns
+    [n][H_q][d] float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_hist = np.asarray(k_hist, dtype=np.float64)
+    v_hist = np.asarray(v_hist, dtype=np.float64)
+    n, h_q, _ = q.shape
+    c, h_kv, _ = k_hist.shape
+    if h_q % h_kv:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    if n < 1 or c < n:
+        raise ValueError("need 1 <= n <= c")
+    group = h_q // h_kv
+    pos = np.arange(c - n, c)                          # positions of the n queries
+    visible = np.arange(c)[None, :] <= pos[:, None]    # [n][c] causal mask
+    out = np.empty_like(q)
+    for h in range(h_q):
+        g = h // group
+        s = scale * (q[:, h, :] @ k_hist[:, g, :].T)    # [n][c]
+        s = np.where(visible, s, -np.inf)
+        s = s - s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        out[:, h, :] = (e / e.sum(axis=1, keepdims=True)) @ v_hist[:, g, :]
+    return out

@@ -22,7 +22,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 from .allocator import BlockManager
-from .attention import attend_head, decode_attention
+from .attention import attend_head, decode_attention, prefill_attention
 from .numerics import e4m3_decode, e4m3_quantize_for_pool, to_f64
 
 _STORE_NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16, "fp8": np.uint8}
@@ -141,6 +141,13 @@ class DecodeOracle:
                     attend_head(qd[i][h], kd[:, h // group, :], vd[:, h // group, :], scale)
                     for h in heads]))
         return np.stack(outs)
+
+    def prefill(self, seq: int, q: np.ndarray, q_dtype: str, scale: float) -> np.ndarray:
+        """Prompt-phase attention: q [n][H_q][d] are the queries of the last n
+        stored tokens of the sequence; returns float64 [n][H_q][d]."""
+        kh, vh = self.history(int(seq))
+        return prefill_attention(to_f64(q, q_dtype), self.dequant(kh, "k"), self.dequant(vh, "v"),
+                                 scale)
 
     def step(self, seqs: Sequence[int], q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,
              in_dtype: str, scale: float):

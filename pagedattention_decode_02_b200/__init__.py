@@ -36,6 +36,7 @@ PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = range(4)
 PKV_DEVERR_CONTEXT_LEN, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 PKV_POOL_HOST_ONLY = 0x1
 PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_TENSOR, PKV_KERNEL_SIMT_BULK, PKV_KERNEL_SIMT_TMA = 0, 1, 2, 3, 4
+PKV_KERNEL_LEAN = 5
 
 DTYPE_NAMES = {"f32": PKV_F32, "f16": PKV_F16, "bf16": PKV_BF16, "fp8": PKV_FP8_E4M3}
 ELEM_BYTES = {PKV_F32: 4, PKV_F16: 2, PKV_BF16: 2, PKV_FP8_E4M3: 1}
@@ -120,12 +121,15 @@ _sig("paged_decode_workspace_bytes", ctypes.c_size_t, _P, ctypes.c_int, ctypes.c
 _sig("paged_decode_workspace_bytes_ex", ctypes.c_size_t, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
      ctypes.c_int)
 _sig("pkv_device_error", _st, _P, _P, ctypes.POINTER(ctypes.c_uint32))
+_sig("paged_prefill_attention", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int, _P,
+     ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P)
 _sig("pkv_status_str", ctypes.c_char_p, ctypes.c_int)
 _sig("pkv_step_create", _st, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
      ctypes.c_int, ctypes.c_int, ctypes.POINTER(_P))
 _sig("pkv_step_destroy", None, _P)
 _sig("pkv_decode_step", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
 _sig("pkv_step_last_launches", ctypes.c_int, _P)
+_sig("pkv_step_last_kernel", ctypes.c_int, _P)
 _sig("pkv_step_profile", _st, _P, ctypes.c_int, ctypes.c_int)
 _sig("paged_decode_attention_static", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int,
      ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P)
@@ -141,8 +145,9 @@ EXPORTED = [
     "bt_free_queue", "bt_stats", "kv_append", "block_copy", "paged_decode_attention",
     "paged_decode_attention_ex", "paged_decode_workspace_bytes", "paged_decode_workspace_bytes_ex",
     "pkv_device_error", "pkv_status_str", "pkv_step_create", "pkv_step_destroy", "pkv_decode_step",
-    "pkv_step_last_launches", "pkv_step_profile", "pkv_step_profile_read",
+    "pkv_step_last_launches", "pkv_step_last_kernel", "pkv_step_profile", "pkv_step_profile_read",
     "paged_decode_attention_static", "paged_decode_static_scratch_bytes", "kv_swap_out", "kv_swap_in",
+    "paged_prefill_attention",
     "bt_set_prefix_caching", "bt_alloc_prefix", "pkv_simulate",
 ]
 
@@ -428,6 +433,26 @@ def paged_decode_attention(pool: Pool, q, block_tables, context_lens, scale: flo
     return out
 
 
+def paged_prefill_attention(pool: Pool, q, q_starts, block_tables, context_lens, scale: float,
+                            max_q_len: Optional[int] = None, out=None, stream=None):
+    """Prompt-phase attention.  q: CUDA [rows][H_q][d]; q_starts: int32 CUDA [B+1]
+    (row offsets per sequence); block_tables: int32 CUDA [B][max_blocks];
+    context_lens: int32 CUDA [B] (cached tokens, the prompt's included).
+    max_q_len: the longest prompt (read from q_starts when None).  Returns out."""
+    import torch
+    B = int(context_lens.shape[0])
+    H_q = int(q.shape[1])
+    if out is None:
+        out = torch.empty_like(q)
+    if max_q_len is None:
+        max_q_len = int((q_starts[1:] - q_starts[:-1]).max().item()) if B else 0
+    _check(_lib.paged_prefill_attention(
+        pool.handle, _dev_ptr(q), torch_dtype_code(q.dtype), _dev_ptr(q_starts), int(max_q_len),
+        _dev_ptr(block_tables), int(block_tables.shape[1]), _dev_ptr(context_lens), B, H_q,
+        float(scale), _dev_ptr(out), _stream_ptr(stream)), "paged_prefill_attention")
+    return out
+
+
 def pkv_device_error(pool: Pool, stream=None) -> int:
     """Synchronise, return and clear the device error bits (0 = none)."""
     bits = ctypes.c_uint32()
@@ -471,6 +496,10 @@ class Step:
     def last_launches(self) -> int:
         return int(_lib.pkv_step_last_launches(self.handle))
 
+    @property
+    def last_kernel(self) -> int:
+        return int(_lib.pkv_step_last_kernel(self.handle))
+
     def run_raw(self, ids: np.ndarray, q_ptr: int, k_ptr: int, v_ptr: int, scale: float,
                 out_ptr: int, stream_ptr: int) -> None:
         """pkv_decode_step with pre-resolved device pointers (int64 ``ids``):
@@ -504,6 +533,14 @@ def pkv_decode_step(step: Step, seq_ids, q, k_new, v_new, scale: float, out, str
 
 def pkv_step_last_launches(step: Step) -> int:
     return step.last_launches
+
+
+def pkv_step_last_kernel(step: Step) -> int:
+    return step.last_kernel
+
+
+KERNEL_NAMES = {PKV_KERNEL_LEAN: "decode_lean_kernel", PKV_KERNEL_TENSOR: "decode_tc_kernel",
+                PKV_KERNEL_SIMT_TMA: "decode_simt2_kernel", PKV_KERNEL_SIMT_BULK: "decode_simt_kernel"}
 
 
 def pkv_step_profile(step: Step, n: int, every: int = 1) -> None:

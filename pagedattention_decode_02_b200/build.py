@@ -29,6 +29,8 @@ SOURCES = [
     "append.cu",
     "decode_simt.cu",
     "decode_simt2.cu",
+    "decode_lean.cu",
+    "prefill.cu",
     "decode_tc.cu",
     "api.cu",
     "no_alloc.cu",

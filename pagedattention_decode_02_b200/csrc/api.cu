@@ -284,7 +284,12 @@ size_t paged_decode_workspace_bytes_ex(const pkv_pool* p, int B, int n_q_heads, 
     if (!p || B <= 0 || n_q_heads <= 0 || max_blocks <= 0) return 0;
     const int P = resolve_partition(p, max_blocks, partition_tokens, n_q_heads / p->n_kv_heads);
     if (P <= 0 || P % 16) return 0;
-    return workspace_for(p, B, n_q_heads, parts_for(p, max_blocks, P));
+    const size_t part = workspace_for(p, B, n_q_heads, parts_for(p, max_blocks, P));
+    // the automatic choice may take the stage-balanced kernel: room for it too
+    if (partition_tokens == 0 && !p->host_only && n_q_heads % p->n_kv_heads == 0 &&
+        pkv::lean_supported(p, p->dtype, n_q_heads / p->n_kv_heads, B, max_blocks))
+        return std::max(part, pkv::lean_workspace_bytes(p, B, n_q_heads));
+    return part;
 }
 
 size_t paged_decode_workspace_bytes(const pkv_pool* p, int B, int n_q_heads, int max_blocks) {
@@ -303,7 +308,10 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                  int partition_tokens, int kernel, void* stream,
                                  cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end,
                                  int* counters = nullptr, bool pdl = false,
-                                 const int32_t* table_rows = nullptr, int n_table_rows = 0) {
+                                 const int32_t* table_rows = nullptr, int n_table_rows = 0,
+                                 int* n_launches = nullptr, int* kernel_used = nullptr) {
+    if (n_launches) *n_launches = 0;
+    if (kernel_used) *kernel_used = 0;
     if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
     if (B == 0) return PKV_OK;
     if (!q || !out || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
@@ -317,24 +325,31 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (partition_tokens != 0 && partition_tokens != -1 &&
         (partition_tokens < 16 || partition_tokens % 16))
         return PKV_ERR_INVALID_ARG;
-    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_SIMT_TMA) return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_LEAN) return PKV_ERR_INVALID_ARG;
     if ((long long)max_blocks * p->block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
     if (!same_device(p)) return PKV_ERR_INVALID_ARG;
 
     const int G = n_q_heads / p->n_kv_heads;
-    const int P = resolve_partition(p, max_blocks, partition_tokens, G);
-    const int max_parts = parts_for(p, max_blocks, P);
-    const size_t need = workspace_for(p, B, n_q_heads, max_parts);
-    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
-    if ((long long)max_parts > 0x7fffffffLL || B > 65535) return PKV_ERR_INVALID_ARG;
-
+    const bool lean_ok = pkv::lean_supported(p, q_dtype, G, B, max_blocks);
+    const size_t lean_need = lean_ok ? pkv::lean_workspace_bytes(p, B, n_q_heads) : 0;
+    const bool lean_fits = lean_ok && ws && ws_bytes >= lean_need && aligned16(ws);
     const bool tc_ok = pkv::tensor_path_supported(p, q_dtype, G);
     const bool s2_ok = pkv::simt2_supported(p, G);
     int use = kernel;
-    if (use == PKV_KERNEL_AUTO) use = tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT;
+    if (use == PKV_KERNEL_AUTO)
+        use = (lean_fits && G > 1 && partition_tokens == 0)
+                  ? PKV_KERNEL_LEAN
+                  : (tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT);
     if (use == PKV_KERNEL_SIMT) use = s2_ok ? PKV_KERNEL_SIMT_TMA : PKV_KERNEL_SIMT_BULK;
     if (use == PKV_KERNEL_TENSOR && !tc_ok) return PKV_ERR_INVALID_ARG;
     if (use == PKV_KERNEL_SIMT_TMA && !s2_ok) return PKV_ERR_INVALID_ARG;
+    if (use == PKV_KERNEL_LEAN && !lean_fits) return PKV_ERR_INVALID_ARG;
+
+    const int P = resolve_partition(p, max_blocks, partition_tokens, G);
+    const int max_parts = use == PKV_KERNEL_LEAN ? 1 : parts_for(p, max_blocks, P);
+    const size_t need = workspace_for(p, B, n_q_heads, max_parts);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_parts > 0x7fffffffLL || B > 65535) return PKV_ERR_INVALID_ARG;
 
     pkv::DecodeParams dp{};
     dp.q = q;
@@ -374,7 +389,13 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = ev_begin ? cudaEventRecord(ev_begin, st) : cudaSuccess;
     if (e != cudaSuccess) return PKV_ERR_CUDA;
-    if (use == PKV_KERNEL_TENSOR) {
+    if (use == PKV_KERNEL_LEAN) {
+        dp.counters = counters;
+        dp.max_parts = 1;
+        e = pkv::launch_decode_lean(dp, p, ws, st);
+        if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, st);
+        if (n_launches) *n_launches = 1 + (counters ? 0 : 1);   // the counter memset
+    } else if (use == PKV_KERNEL_TENSOR) {
         e = pkv::launch_decode_tensor(dp, p->tmap_k, p->tmap_v, p->dtype, p->head_dim, st, ev_mid);
     } else if (use == PKV_KERNEL_SIMT_TMA) {
         e = pkv::launch_decode_simt2(dp, p->tmap_k, p->tmap_v, p->dtype, q_dtype, p->head_dim,
@@ -383,6 +404,9 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
         e = pkv::launch_decode_simt(dp, p->dtype, q_dtype, p->head_dim, pkv::simt_heads_per_cta(G),
                                     st, ev_mid);
     }
+    if (kernel_used) *kernel_used = use;
+    if (use != PKV_KERNEL_LEAN && n_launches)
+        *n_launches = 1 + (max_parts > 1 && !(use == PKV_KERNEL_TENSOR && counters) ? 1 : 0);
     if (e == cudaSuccess && ev_end) e = cudaEventRecord(ev_end, st);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
@@ -406,6 +430,40 @@ pkv_status paged_decode_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                   void* stream) {
     return paged_decode_attention_ex(p, q, q_dtype, tables, max_blocks, lens, B, n_q_heads, scale,
                                      out, ws, ws_bytes, 0, PKV_KERNEL_AUTO, stream);
+}
+
+pkv_status paged_prefill_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                   const int32_t* q_starts, int max_q_len, const int32_t* tables,
+                                   int max_blocks, const int32_t* lens, int B, int n_q_heads,
+                                   float scale, void* out, void* stream) {
+    if (!p || p->host_only || B < 0 || max_q_len < 0) return PKV_ERR_INVALID_ARG;
+    if (B == 0 || max_q_len == 0) return PKV_OK;
+    if (!q || !out || !q_starts || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
+    if (n_q_heads < p->n_kv_heads || n_q_heads % p->n_kv_heads) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || B > 65535 || p->n_kv_heads > 65535) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_blocks * p->block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_q_len * (n_q_heads / p->n_kv_heads) > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+    if (!pkv::prefill_supported(p, q_dtype)) return PKV_ERR_INVALID_ARG;
+    if (!same_device(p)) return PKV_ERR_INVALID_ARG;
+    pkv::PrefillParams pp{};
+    pp.q = q;
+    pp.out = out;
+    pp.q_starts = q_starts;
+    pp.tables = tables;
+    pp.lens = lens;
+    pp.err = p->d_err;
+    pp.B = B;
+    pp.H_q = n_q_heads;
+    pp.H_kv = p->n_kv_heads;
+    pp.G = n_q_heads / p->n_kv_heads;
+    pp.max_blocks = max_blocks;
+    pp.block_size = p->block_size;
+    pp.num_blocks = p->num_blocks;
+    pp.max_q_len = max_q_len;
+    pp.q_scale = scale * 1.4426950408889634f;
+    return pkv::launch_prefill(pp, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_device_error(pkv_pool* p, void* stream, uint32_t* bits_out) {
@@ -444,6 +502,7 @@ struct pkv_step {
     int* d_counters = nullptr;        // [max_batch][n_q_heads], zero between launches
     int max_parts = 1;
     int last_launches = 0;
+    int last_kernel = 0;              // decode kernel of the last round (after the auto choice)
     // host mirror of the persistent rows
     std::vector<int64_t> row_seq;     // sequence held, or INT64_MIN
     std::vector<uint64_t> row_epoch;
@@ -467,14 +526,6 @@ struct pkv_step {
 };
 
 namespace {
-// the tensor-core kernel merges split partitions itself when the step runtime
-// hands it its zeroed counters
-bool decode_merges_in_kernel(const pkv_pool* pool, const pkv_step* s) {
-    const int G = s->n_q_heads / pool->n_kv_heads;
-    const bool tc = pkv::tensor_path_supported(pool, s->q_dtype, G);
-    return (s->kernel == PKV_KERNEL_AUTO || s->kernel == PKV_KERNEL_TENSOR) && tc;
-}
-
 void prof_free(pkv_step* s) {
     if (s->prof_ev) {
         for (int i = 0; i < 4 * s->prof_n; ++i)
@@ -551,7 +602,7 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_
     if (partition_tokens != 0 && partition_tokens != -1 &&
         (partition_tokens < 16 || partition_tokens % 16))
         return PKV_ERR_INVALID_ARG;
-    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_SIMT_TMA) return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_KERNEL_AUTO || kernel > PKV_KERNEL_LEAN) return PKV_ERR_INVALID_ARG;
     if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
     pkv_step* s = new (std::nothrow) pkv_step();
     if (!s) return PKV_ERR_INVALID_ARG;
@@ -581,6 +632,9 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_
                                     n_q_heads / pool->n_kv_heads);
     s->max_parts = parts_for(pool, max_blocks, P);
     s->ws_bytes = workspace_for(pool, max_batch, n_q_heads, s->max_parts);
+    if ((kernel == PKV_KERNEL_AUTO || kernel == PKV_KERNEL_LEAN) &&
+        pkv::lean_supported(pool, q_dtype, n_q_heads / pool->n_kv_heads, max_batch, max_blocks))
+        s->ws_bytes = std::max(s->ws_bytes, pkv::lean_workspace_bytes(pool, max_batch, n_q_heads));
     if (ok && s->ws_bytes) ok &= cudaMalloc(&s->d_ws, s->ws_bytes) == cudaSuccess;
     if (ok && s->ws_bytes) {
         const size_t cb = (size_t)max_batch * n_q_heads * sizeof(int);
@@ -601,11 +655,14 @@ void pkv_step_destroy(pkv_step* s) {
 
 int pkv_step_last_launches(const pkv_step* s) { return s ? s->last_launches : 0; }
 
+int pkv_step_last_kernel(const pkv_step* s) { return s ? s->last_kernel : 0; }
+
 pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const void* q,
                            const void* k_new, const void* v_new, float scale, void* out,
                            void* stream) {
     if (!s || B < 0 || B > s->max_batch) return PKV_ERR_INVALID_ARG;
     s->last_launches = 0;
+    s->last_kernel = 0;
     if (B == 0) return PKV_OK;
     if (!seq_ids || !q || !k_new || !v_new || !out) return PKV_ERR_INVALID_ARG;
     if (!aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_INVALID_ARG;
@@ -760,13 +817,14 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     }
     // the decode kernel starts its launch while the prologue runs (programmatic
     // dependent launch), except in profiled rounds whose events sit between
+    int decode_launches = 0;
     ps = decode_attention_impl(pool, q, s->q_dtype, s->d_tables, s->max_blocks, d_lens, B,
                                s->n_q_heads, scale, out, s->d_ws, s->ws_bytes, s->partition_tokens,
                                s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled,
-                               d_rows, s->max_seqs);
+                               d_rows, s->max_seqs, &decode_launches, &s->last_kernel);
     if (ps != PKV_OK) return ps;
     if (profiled) ++s->prof_count;
-    launches += 1 + (s->max_parts > 1 && !decode_merges_in_kernel(pool, s) ? 1 : 0);
+    launches += decode_launches;
     s->last_launches = launches;
     return PKV_OK;
 }

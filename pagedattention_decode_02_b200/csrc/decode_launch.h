@@ -35,6 +35,33 @@ cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, cons
                                  int kv_dtype, int head_dim, cudaStream_t st,
                                  cudaEvent_t mid = nullptr);
 
+// Stage-balanced tensor-core decode (persistent CTAs, in-kernel merge):
+// F16/BF16 pools with row tensor maps, q in the pool dtype, head_dim 64/128,
+// 1 <= G <= 128, B <= 2048.  The workspace holds the pieces' partial states
+// and, when p.counters is null, zeroed (by a memset on st) merge counters.
+bool lean_supported(const pkv_pool* pool, int q_dtype, int group, int B, int max_blocks);
+size_t lean_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads);
+cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, cudaStream_t st);
+
+// Prompt-phase attention (F16/BF16 pools with row tensor maps, q in the pool
+// dtype, head_dim 64/128).  Sequence i's queries are rows
+// q_starts[i] .. q_starts[i+1]-1 of q/out ([rows][H_q][D]); they are the last
+// n_i of its lens[i] cached tokens and attend causally.
+struct PrefillParams {
+    const void* q;
+    void* out;
+    const int32_t* q_starts;   // [B + 1]
+    const int32_t* tables;     // [B][max_blocks]
+    const int32_t* lens;       // [B]
+    uint32_t* err;
+    int B, H_q, H_kv, G;
+    int max_blocks, block_size, num_blocks;
+    int max_q_len;             // >= every n_i (sizes the grid)
+    float q_scale;             // scale * log2(e)
+};
+bool prefill_supported(const pkv_pool* pool, int q_dtype);
+cudaError_t launch_prefill(const PrefillParams& p, const pkv_pool* pool, cudaStream_t st);
+
 // One decode round's small host-side results, passed by value as kernel
 // parameters (no separate host-to-device copy):
 //   data = slots[B] | lens[B] | rows[B] | cow_src[n_cow] | cow_dst[n_cow]

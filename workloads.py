@@ -181,6 +181,12 @@ def step_qkv(cfg: Config, seed: int, seq: int, step: int):
     return q, k, v
 
 
+def prompt_queries(cfg: Config, seed: int, seq: int, n: int) -> np.ndarray:
+    """Queries of a sequence's last n prompt tokens: [n][H_q][d] float32, N(0,1)."""
+    rng = _rng(seed, 7, seq, n)
+    return rng.standard_normal((n, cfg.n_q_heads, cfg.head_dim), dtype=np.float32)
+
+
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
     """Round float32 draws to a storage dtype (round to nearest even).
 
