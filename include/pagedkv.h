@@ -281,7 +281,7 @@ pkv_status paged_decode_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_d
 size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, int max_blocks);
 
 /* Kernel selection for paged_decode_attention_ex. */
-#define PKV_KERNEL_AUTO 0          /* LEAN for grouped heads (G > 1) when supported, the workspace
+#define PKV_KERNEL_AUTO 0          /* LEAN for large groups (G > 16) when supported, the workspace
                                       holds its state and partition_tokens is 0; else TENSOR when
                                       supported; else SIMT */
 #define PKV_KERNEL_SIMT 1          /* CUDA-core dot products: SIMT_TMA when supported, else SIMT_BULK */
@@ -290,8 +290,8 @@ size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, 
 #define PKV_KERNEL_SIMT_BULK 3     /* CUDA-core, 1-D bulk copies per block run (any shape) */
 #define PKV_KERNEL_SIMT_TMA 4      /* CUDA-core, swizzled 2-D TMA boxes, one query head per CTA:
                                       rows of 128/256/512 bytes, power-of-two block size */
-#define PKV_KERNEL_LEAN 5          /* tensor cores, one wave of persistent CTAs sharing the batch's
-                                      16-token stages equally, split pairs merged in the kernel:
+#define PKV_KERNEL_LEAN 5          /* tensor cores, one wave of persistent workers sharing the batch's
+                                      16-token stages equally, split pairs merged by a second launch:
                                       F16/BF16 pools with head_dim 64 or 128, power-of-two block
                                       size, 1 <= G <= 128, B <= 2048; ignores partition_tokens */
 

@@ -48,13 +48,16 @@ constexpr int kAutoPartition = 512;
 
 // With G query heads per KV head, a partition's partial state is G * (d + 2)
 // floats against partition * 2 * d * elem bytes of K/V, so the automatic
-// partition grows with G (about 1.5 % extra traffic at G = 8, d = 128, bf16).
+// partition grows with G; grouped heads take twice the one-head length
+// (measured on the Llama-2-70B-shaped batch: 1024-token partitions beat 512
+// and 2048).
 int resolve_partition(const pkv_pool* pool, int max_blocks, int requested, int group = 1) {
     const long long max_ctx = (long long)max_blocks * pool->block_size;
     const int whole = (int)(((max_ctx + 15) / 16) * 16);
     if (requested < 0) return whole < 16 ? 16 : whole;
     if (requested > 0) return requested;
-    const long long auto_p = (long long)kAutoPartition * ((group + 7) / 8);
+    const long long auto_p =
+        (long long)kAutoPartition * (group > 1 ? 2 : 1) * ((group + 7) / 8);
     if (max_ctx <= (group > 8 ? auto_p : kNoSplitTokens)) return whole < 16 ? 16 : whole;
     return (int)(auto_p < (1 << 30) ? auto_p : (1 << 30));
 }
@@ -336,8 +339,11 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     const bool tc_ok = pkv::tensor_path_supported(p, q_dtype, G);
     const bool s2_ok = pkv::simt2_supported(p, G);
     int use = kernel;
+    // automatic: large groups (one KV head shared by many query heads, a
+    // small latency-bound batch) take the stage-balanced kernel; up to 16
+    // heads per KV head the partitioned tensor-core kernel measured faster
     if (use == PKV_KERNEL_AUTO)
-        use = (lean_fits && G > 1 && partition_tokens == 0)
+        use = (lean_fits && G > 16 && partition_tokens == 0)
                   ? PKV_KERNEL_LEAN
                   : (tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT);
     if (use == PKV_KERNEL_SIMT) use = s2_ok ? PKV_KERNEL_SIMT_TMA : PKV_KERNEL_SIMT_BULK;
@@ -392,9 +398,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (use == PKV_KERNEL_LEAN) {
         dp.counters = counters;
         dp.max_parts = 1;
-        e = pkv::launch_decode_lean(dp, p, ws, st);
-        if (e == cudaSuccess && ev_mid) e = cudaEventRecord(ev_mid, st);
-        if (n_launches) *n_launches = 1 + (counters ? 0 : 1);   // the counter memset
+        e = pkv::launch_decode_lean(dp, p, ws, st, ev_mid);
+        if (n_launches) *n_launches = 1 + (counters ? 0 : 1);   // + the counter memset
     } else if (use == PKV_KERNEL_TENSOR) {
         e = pkv::launch_decode_tensor(dp, p->tmap_k, p->tmap_v, p->dtype, p->head_dim, st, ev_mid);
     } else if (use == PKV_KERNEL_SIMT_TMA) {

@@ -35,13 +35,17 @@ cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, cons
                                  int kv_dtype, int head_dim, cudaStream_t st,
                                  cudaEvent_t mid = nullptr);
 
-// Stage-balanced tensor-core decode (persistent CTAs, in-kernel merge):
-// F16/BF16 pools with row tensor maps, q in the pool dtype, head_dim 64/128,
-// 1 <= G <= 128, B <= 2048.  The workspace holds the pieces' partial states
-// and, when p.counters is null, zeroed (by a memset on st) merge counters.
+// Stage-balanced tensor-core decode (one persistent wave; a split pair merged
+// in the kernel by the worker that finishes its last piece): F16/BF16 pools with row tensor
+// maps, q in the pool dtype, head_dim 64/128, 1 <= G <= 128, B <= 2048.  The
+// workspace holds the pieces' partial states; the per-pair merge counters are
+// p.counters when given (zeroed once by the caller; every launch leaves them
+// zero), else carved from the workspace and zeroed by a memset on st.  mid
+// (may be null) is recorded after the launch.
 bool lean_supported(const pkv_pool* pool, int q_dtype, int group, int B, int max_blocks);
 size_t lean_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads);
-cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, cudaStream_t st);
+cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, cudaStream_t st,
+                               cudaEvent_t mid = nullptr);
 
 // Prompt-phase attention (F16/BF16 pools with row tensor maps, q in the pool
 // dtype, head_dim 64/128).  Sequence i's queries are rows

@@ -14,8 +14,10 @@
 // piece in the workspace, and the worker that finishes the pair's last piece
 // merges them by log-sum-exp (the split-context merge of the decode step).
 //
-// Worker = MT warps (16 query heads of the KV head's group each, as mma.sync
-// m16n8k16 m-tiles); a CTA holds TS workers.  Each worker owns a ring of RG
+// Worker = MT warps of 8 query heads of the KV head's group each; a warp
+// computes S^T = K Q^T and O^T += V^T P^T with mma.sync m16n8k16 (16 tokens
+// or 16 d-rows by 8 heads: no padded rows up to 8 heads per KV head); a CTA
+// holds TS workers.  Each worker owns a ring of RG
 // 16-token stage slots filled by 2-D TMA loads (128-byte swizzle, plain loads
 // of this GPU's own memory) that its first warp issues, RG stages ahead of
 // the one being consumed; with MT > 1 an "empty" mbarrier per slot tells the
@@ -49,13 +51,12 @@ struct LeanCfg {
     static constexpr int kSlot = 2 * kStageTokens * D * 2;   // K and V of one stage
 };
 
-// Workers per CTA, ring slots per worker and merge scratch per worker (floats)
-// for MT m-tile warps per worker.
+// Workers per CTA and ring slots per worker for MT warps (of 8 query heads)
+// per worker.
 template <int D, int MT>
 struct LeanShape {
-    static constexpr int TS = MT == 1 ? 4 : (MT == 2 ? 2 : 1);
+    static constexpr int TS = MT == 1 ? 4 : (MT == 2 ? 2 : 1);   // <= 16 warps per CTA
     static constexpr int RG = D == 128 ? 3 : 4;
-    static constexpr int kMerge = MT == 1 ? 512 : 2048;
 };
 
 // The part of one (sequence, KV head) pair inside a worker's share.
@@ -99,6 +100,172 @@ struct Schedule {
     }
 };
 
+// Merge of a split pair by the worker that finished its last piece (NTH
+// threads, t = 0 .. NTH - 1): the pair's pieces left (running max, sum,
+// accumulator) per head in consecutive workspace slots (pair + first worker
+// .. pair + last worker), combined by log-sum-exp.  Each thread takes 4
+// float4 outputs per pass, two pieces at a time; all loads of a step are
+// issued before any is used.  Kept out of line so that its registers do not
+// count against the streaming loop's.
+template <typename T, int D, int NTH>
+__device__ __noinline__ void merge_pair(const DecodeParams& p, int pair, int first, int n_pieces,
+                                        int t) {
+    constexpr int E = 4;
+    const int G = p.G;
+    const int seq = pair / p.H_kv, g = pair % p.H_kv;
+    const int total = G * (D / 4);
+    const size_t slot0 = (size_t)pair + first;
+    const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + slot0 * G;
+    const float4* acc = reinterpret_cast<const float4*>(p.ws_acc) + slot0 * G * (D / 4);
+    T* out = reinterpret_cast<T*>(p.out) + ((size_t)seq * p.H_q + (size_t)g * G) * D;
+    for (int base = t; base < total; base += NTH * E) {
+        float M[E], L[E];
+        float4 O[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            M[e] = -INFINITY;
+            L[e] = 0.f;
+            O[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll 2
+        for (int j = 0; j < n_pieces; ++j) {
+            float2 v[E];
+            float4 a[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int i = min(base + e * NTH, total - 1);
+                v[e] = __ldcg(ml + (size_t)j * G + i / (D / 4));
+                a[e] = __ldcg(acc + (size_t)j * G * (D / 4) + i);
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                if (v[e].x == -INFINITY) continue;
+                const float Mn = fmaxf(M[e], v[e].x);
+                const float so = exp2f(M[e] - Mn), sn = exp2f(v[e].x - Mn);
+                L[e] = L[e] * so + v[e].y * sn;
+                O[e].x = O[e].x * so + a[e].x * sn;
+                O[e].y = O[e].y * so + a[e].y * sn;
+                O[e].z = O[e].z * so + a[e].z * sn;
+                O[e].w = O[e].w * so + a[e].w * sn;
+                M[e] = Mn;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int i = base + e * NTH;
+            if (i >= total) break;
+            const float s = L[e] > 0.f ? 1.f / L[e] : 0.f;
+            T* o = out + (size_t)i * 4;
+            o[0] = Elem<T>::from_f(O[e].x * s);
+            o[1] = Elem<T>::from_f(O[e].y * s);
+            o[2] = Elem<T>::from_f(O[e].z * s);
+            o[3] = Elem<T>::from_f(O[e].w * s);
+        }
+    }
+}
+
+template <int D, int MT>
+__host__ __device__ constexpr int lean_fixed_smem() {
+    using S = LeanShape<D, MT>;
+    // rings (1024-aligned) + full/empty barriers + slot token counts + per
+    // worker flags + per-warp scan totals; prefix sums follow
+    return 1024 + S::TS * S::RG * LeanCfg<D>::kSlot + 2 * S::TS * S::RG * 8 + S::TS * S::RG * 4 +
+           S::TS * 4 + 32 * 4;
+}
+
+// A walk over a worker's share, one 16-token stage at a time, RG stages ahead
+// of the consumption; held by the worker's first warp (all lanes).
+struct Cursor {
+    long long pos;       // the next piece starts at pos
+    int seq, g;          // piece being walked
+    int s, s1;           // its next stage and its end (s == s1: take the next piece)
+    int trow;            // its table row (-1: invalid)
+    int c;               // its context length
+    int wb, wid;         // table entries wb .. wb + 31, one per lane
+    int count;           // stages walked so far
+};
+
+__device__ __forceinline__ void cursor_init(Cursor& cu, long long lo) {
+    cu.pos = lo;
+    cu.s = cu.s1 = 0;
+    cu.count = 0;
+}
+
+// Moves the cursor over its next stage.  Returns the stage's box count nb
+// (2-D TMA boxes of min(bs, 16) rows each) and, for lane < nb, that box's
+// TMA row in *y (-1 when its block id is out of range, or the table row is
+// invalid); *n = valid tokens of the stage.
+__device__ __forceinline__ int cursor_stage(Cursor& cu, long long hi, const Schedule& sc,
+                                            const DecodeParams& p, int lane, int* y, int* n) {
+    if (cu.s == cu.s1) {
+        const Piece pc = sc.at(cu.pos, hi);
+        cu.pos = pc.start + pc.s1;
+        cu.seq = pc.seq;
+        cu.g = pc.g;
+        cu.s = pc.s0;
+        cu.s1 = pc.s1;
+        cu.trow = (int)table_row(p, pc.seq);
+        cu.c = p.lens[pc.seq];
+        cu.wb = -1;
+    }
+    const int bs = p.block_size;
+    const int rpb = bs < kStageTokens ? bs : kStageTokens;   // rows per box
+    const int a = cu.s * kStageTokens;
+    *n = min(kStageTokens, cu.c - a);
+    const int nb = (*n + rpb - 1) / rpb;
+    const int lb1 = (a + *n - 1) / bs;
+    if (cu.wb < 0 || lb1 >= cu.wb + 32) {
+        cu.wb = a / bs;
+        cu.wid = (cu.trow >= 0 && cu.wb + lane < p.max_blocks)
+                     ? p.tables[(long long)cu.trow * p.max_blocks + cu.wb + lane]
+                     : -1;
+    }
+    const int t0 = a + (lane < nb ? lane : 0) * rpb;
+    const int lb = t0 / bs;
+    const int id = __shfl_sync(kFull, cu.wid, lb - cu.wb);
+    *y = (cu.trow >= 0 && id >= 0 && id < p.num_blocks) ? (id * p.H_kv + cu.g) * bs + (t0 - lb * bs)
+                                                         : -1;
+    ++cu.s;
+    ++cu.count;
+    return nb;
+}
+
+// Load the cursor's next stage into a ring slot: one box per lane < nb, K
+// and V, every 64-column half; a stage with an out-of-range block id is not
+// loaded (slot_n = -1) and its barrier phase completes without bytes.
+template <int D>
+__device__ __forceinline__ void issue_stage(Cursor& cu, long long hi, const Schedule& sc,
+                                            const DecodeParams& p, const CUtensorMap* tk,
+                                            const CUtensorMap* tv, uint8_t* slot_mem,
+                                            uint64_t* full, volatile int* slot_n, uint64_t policy,
+                                            int lane) {
+    constexpr int TILE = LeanCfg<D>::kSlot / 2;
+    constexpr int HALVES = D / 64;
+    int y, n;
+    const int nb = cursor_stage(cu, hi, sc, p, lane, &y, &n);
+    const int rpb = p.block_size < kStageTokens ? p.block_size : kStageTokens;
+    const bool bad = __any_sync(kFull, lane < nb && y < 0);
+    if (lane == 0) {
+        *slot_n = bad ? -1 : n;
+        if (bad) {
+            report_error(p.err, PKV_DEVERR_BLOCK_ID);
+            tc::mbar_arrive(full);
+        } else {
+            mbar_arrive_expect_tx(full, (uint32_t)(2 * HALVES * nb * rpb * 128));
+        }
+    }
+    __syncwarp();
+    if (!bad && lane < nb) {
+#pragma unroll
+        for (int hf = 0; hf < HALVES; ++hf) {
+            const int off = hf * (kStageTokens * 128) + lane * rpb * 128;
+            tc::tma_load_2d(slot_mem + off, tk, hf * 64, y, full, policy);
+            tc::tma_load_2d(slot_mem + TILE + off, tv, hf * 64, y, full, policy);
+        }
+    }
+    __syncwarp();
+}
+
 // Barrier over the MT warps of one worker (named barrier 1 + worker).
 template <int MT>
 __device__ __forceinline__ void worker_sync(int worker) {
@@ -109,184 +276,8 @@ __device__ __forceinline__ void worker_sync(int worker) {
     }
 }
 
-// Merge the pieces' partial states of pair (seq, g) into the output, run by
-// the threads of the worker that finished the pair last.  Round trip 1: every
-// piece's running max per head row -> weights in shared memory; round trip 2:
-// the sums; round trip 3: the accumulators, all loads independent.  `scratch`
-// holds k_merge floats; more pieces than fit take the one-element-at-a-time
-// path.
 template <typename T, int D, int MT>
-__device__ void merge_pieces(const DecodeParams& p, int seq, int g, int first, int n_pieces,
-                             float* scratch, int k_merge, int wtid, int worker) {
-    constexpr int n_thr = MT * 32;
-    const int G = p.G;
-    const size_t slot0 = (size_t)seq * p.H_kv + g + first;
-    T* out = reinterpret_cast<T*>(p.out) + ((size_t)seq * p.H_q + (size_t)g * G) * D;
-    if (n_pieces * G + G <= k_merge) {
-        float* w = scratch;                    // [n_pieces][G] weights
-        float* rowv = scratch + n_pieces * G;  // [G] row max, then 1 / L
-        for (int i = wtid; i < n_pieces * G; i += n_thr)
-            w[i] = __ldcg(p.ws_ml + ((slot0 + i / G) * G + i % G) * 2);
-        worker_sync<MT>(worker);
-        for (int r = wtid; r < G; r += n_thr) {
-            float M = -INFINITY;
-            for (int j = 0; j < n_pieces; ++j) M = fmaxf(M, w[j * G + r]);
-            rowv[r] = M;
-        }
-        worker_sync<MT>(worker);
-        for (int i = wtid; i < n_pieces * G; i += n_thr) {
-            const float m = w[i];
-            w[i] = (m == -INFINITY) ? 0.f : exp2f(m - rowv[i % G]);
-        }
-        worker_sync<MT>(worker);
-        for (int r = wtid; r < G; r += n_thr) {
-            float L = 0.f;
-            for (int j = 0; j < n_pieces; ++j)
-                L = fmaf(w[j * G + r], __ldcg(p.ws_ml + ((slot0 + j) * G + r) * 2 + 1), L);
-            rowv[r] = L > 0.f ? 1.f / L : 0.f;
-        }
-        worker_sync<MT>(worker);
-        for (int i = wtid; i < G * (D / 4); i += n_thr) {
-            const int r = i / (D / 4), d4 = i % (D / 4);
-            float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int j = 0; j < n_pieces; ++j) {
-                const float wj = w[j * G + r];
-                const float4 a = __ldcg(
-                    reinterpret_cast<const float4*>(p.ws_acc + ((slot0 + j) * G + r) * D) + d4);
-                O.x = fmaf(wj, a.x, O.x);
-                O.y = fmaf(wj, a.y, O.y);
-                O.z = fmaf(wj, a.z, O.z);
-                O.w = fmaf(wj, a.w, O.w);
-            }
-            const float inv = rowv[r];
-            T* o = out + (size_t)r * D + 4 * d4;
-            o[0] = Elem<T>::from_f(O.x * inv);
-            o[1] = Elem<T>::from_f(O.y * inv);
-            o[2] = Elem<T>::from_f(O.z * inv);
-            o[3] = Elem<T>::from_f(O.w * inv);
-        }
-        worker_sync<MT>(worker);   // the scratch is free again
-        return;
-    }
-    for (int i = wtid; i < G * (D / 4); i += n_thr) {
-        const int r = i / (D / 4), d4 = i % (D / 4);
-        float M = -INFINITY, L = 0.f;
-        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < n_pieces; ++j) {
-            const size_t row = (slot0 + j) * G + r;
-            const float m = __ldcg(p.ws_ml + row * 2);
-            const float l = __ldcg(p.ws_ml + row * 2 + 1);
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(p.ws_acc + row * D) + d4);
-            if (m == -INFINITY) continue;
-            const float Mn = fmaxf(M, m);
-            const float so = exp2f(M - Mn), sn = exp2f(m - Mn);
-            L = L * so + l * sn;
-            O.x = O.x * so + a.x * sn;
-            O.y = O.y * so + a.y * sn;
-            O.z = O.z * so + a.z * sn;
-            O.w = O.w * so + a.w * sn;
-            M = Mn;
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        T* o = out + (size_t)r * D + 4 * d4;
-        o[0] = Elem<T>::from_f(O.x * inv);
-        o[1] = Elem<T>::from_f(O.y * inv);
-        o[2] = Elem<T>::from_f(O.z * inv);
-        o[3] = Elem<T>::from_f(O.w * inv);
-    }
-}
-
-template <int D, int MT>
-__host__ __device__ constexpr int lean_fixed_smem() {
-    using S = LeanShape<D, MT>;
-    // rings (1024-aligned) + full/empty barriers + slot token counts + per
-    // worker flags + merge scratch + per-warp scan totals; prefix sums follow
-    return 1024 + S::TS * S::RG * LeanCfg<D>::kSlot + 2 * S::TS * S::RG * 8 + S::TS * S::RG * 4 +
-           S::TS * 4 + S::TS * S::kMerge * 4 + 16 * 4;
-}
-
-// The issuing side of a worker: walks the share RG stages ahead of the
-// consumption; held by the worker's first warp (all lanes).
-struct Issuer {
-    long long pos;       // the next piece starts at pos
-    int seq, g;          // piece being issued
-    int s, s1;           // next stage of it to issue, its end (s == s1: take the next piece)
-    int trow;            // its table row (-1: invalid)
-    int c;               // its context length
-    int wb, wid;         // table entries wb .. wb + 31, one per lane
-    int issued;          // stages issued so far
-};
-
-template <int D>
-__device__ __forceinline__ void issue_stage(Issuer& is, long long hi, const Schedule& sc,
-                                            const DecodeParams& p, const CUtensorMap* tk,
-                                            const CUtensorMap* tv, uint8_t* slot_mem,
-                                            uint64_t* full, volatile int* slot_n, uint64_t policy,
-                                            int lane) {
-    constexpr int TILE = LeanCfg<D>::kSlot / 2;
-    constexpr int HALVES = D / 64;
-    if (is.s == is.s1) {
-        const Piece pc = sc.at(is.pos, hi);
-        is.pos = pc.start + pc.s1;
-        is.seq = pc.seq;
-        is.g = pc.g;
-        is.s = pc.s0;
-        is.s1 = pc.s1;
-        is.trow = (int)table_row(p, pc.seq);
-        is.c = p.lens[pc.seq];
-        is.wb = -1;
-    }
-    const int bs = p.block_size;
-    const int rpb = bs < kStageTokens ? bs : kStageTokens;   // rows per box
-    const int a = is.s * kStageTokens;
-    const int n = min(kStageTokens, is.c - a);
-    const int nb = (n + rpb - 1) / rpb;
-    const int lb0 = a / bs;
-    const int lb1 = (a + n - 1) / bs;
-    if (is.wb < 0 || lb1 >= is.wb + 32) {
-        is.wb = lb0;
-        is.wid = (is.trow >= 0 && is.wb + lane < p.max_blocks)
-                     ? p.tables[(long long)is.trow * p.max_blocks + is.wb + lane]
-                     : -1;
-    }
-    bool bad = is.trow < 0;
-    for (int bx = 0; bx < nb; ++bx) {
-        const int id = __shfl_sync(kFull, is.wid, (a + bx * rpb) / bs - is.wb);
-        bad |= id < 0 || id >= p.num_blocks;
-    }
-    if (lane == 0) {
-        *slot_n = bad ? -1 : n;
-        if (bad) {
-            report_error(p.err, PKV_DEVERR_BLOCK_ID);
-            tc::mbar_arrive(full);
-        } else {
-            mbar_arrive_expect_tx(full, (uint32_t)(2 * HALVES * nb * rpb * 128));
-        }
-    }
-    if (!bad) {
-        for (int bx = 0; bx < nb; ++bx) {
-            const int t0 = a + bx * rpb;
-            const int lb = t0 / bs;
-            const int id = __shfl_sync(kFull, is.wid, lb - is.wb);
-            if (lane == 0) {
-                const int y = (id * p.H_kv + is.g) * bs + (t0 - lb * bs);
-#pragma unroll
-                for (int hf = 0; hf < HALVES; ++hf) {
-                    const int off = hf * (kStageTokens * 128) + bx * rpb * 128;
-                    tc::tma_load_2d(slot_mem + off, tk, hf * 64, y, full, policy);
-                    tc::tma_load_2d(slot_mem + TILE + off, tv, hf * 64, y, full, policy);
-                }
-            }
-        }
-    }
-    __syncwarp();
-    ++is.s;
-    ++is.issued;
-}
-
-template <typename T, int D, int MT>
-__global__ void __launch_bounds__(LeanShape<D, MT>::TS * MT * 32)
+__global__ void __launch_bounds__(LeanShape<D, MT>::TS * MT * 32, MT <= 2 ? 2 : 1)
 decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     using S = LeanShape<D, MT>;
@@ -294,9 +285,8 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr int RG = S::RG;
     constexpr int SLOT = LeanCfg<D>::kSlot;
     constexpr int TILE = SLOT / 2;
-    constexpr int DTILES = D / 8;
     constexpr int NT = TS * MT * 32;
-    static_assert(NT / 32 <= 16, "scan totals");
+    static_assert(NT / 32 <= 32, "scan totals");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* rings = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -305,9 +295,8 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t* empties = fulls + TS * RG;                                     // [TS][RG]
     volatile int* slot_ns = reinterpret_cast<volatile int*>(empties + TS * RG);   // [TS][RG]
     volatile int* flags = slot_ns + TS * RG;                                 // [TS] last-piece flag
-    float* merge_scr = reinterpret_cast<float*>(const_cast<int*>(flags + TS));   // [TS][kMerge]
-    int* wsum = reinterpret_cast<int*>(merge_scr + TS * S::kMerge);          // [16]
-    int* pre = wsum + 16;                                                    // [B + 1]
+    int* wsum = const_cast<int*>(flags + TS);                                // [32]
+    int* pre = wsum + 32;                                                    // [B + 1]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -368,28 +357,27 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // with fewer stages than workers the surplus workers stay idle, so that
     // every share is non-empty and a pair's pieces sit in consecutive workers
     const long long total = (long long)H_kv * pre[B];
+    if (total == 0) return;
     const long long n_workers = (long long)gridDim.x * TS;
     const Schedule sc{pre, B, H_kv, (int)(total < n_workers ? total : n_workers), total};
+
+    // ------------------------------------------------------------- workers
     const int worker = warp / MT;
     const int mt = warp % MT;
     const int vw = blockIdx.x * TS + worker;   // this worker's index on the stage line
-    if (vw >= sc.n) return;
-    const long long lo = sc.lo(vw);
-    const long long hi = sc.lo(vw + 1);
+    const long long lo = vw < sc.n ? sc.lo(vw) : 0;
+    const long long hi = vw < sc.n ? sc.lo(vw + 1) : 0;
     const int n_stages = (int)(hi - lo);
 
     uint8_t* ring = rings + worker * RG * SLOT;
     uint64_t* full = fulls + worker * RG;
     uint64_t* empty = empties + worker * RG;
     volatile int* slot_n = slot_ns + worker * RG;
-    float* scratch = merge_scr + worker * S::kMerge;
     const bool issuer = mt == 0;
     const uint64_t policy = l2_evict_first_policy();
 
-    Issuer is;
-    is.pos = lo;
-    is.s = is.s1 = 0;
-    is.issued = 0;
+    Cursor is;
+    cursor_init(is, lo);
     if (issuer) {
         const int pro = min(RG, n_stages);
         for (int k = 0; k < pro; ++k)
@@ -399,9 +387,8 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const int gq = lane >> 2;
     const int tq = lane & 3;
-    const int r0 = mt * 16 + gq;
-    const int r1 = r0 + 8;
-    const int wtid = mt * 32 + lane;
+    const int hw = mt * 8;                    // this warp's first head of the group
+    const int ha = hw + 2 * tq, hb = ha + 1;  // this lane's two heads
     long long pos = lo;
     int it = 0;
     bool abort = false;
@@ -409,12 +396,12 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const Piece pc = sc.at(pos, hi);
         pos = pc.start + pc.s1;
         const int h0 = pc.g * G;
-        uint32_t qa[D / 16][4];
-        tc::load_q_frags<T, D>(qa, reinterpret_cast<const T*>(p.q) + ((size_t)pc.seq * p.H_q + h0) * D,
-                               mt * 16, G, lane);
-        float o[DTILES][4];
+        uint32_t qb[D / 16][2];
+        tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)pc.seq * p.H_q + h0) * D,
+                                hw, G, lane);
+        float o[D / 16][4];
 #pragma unroll
-        for (int j = 0; j < DTILES; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         float m_run[2] = {-INFINITY, -INFINITY};
         float l_run[2] = {0.f, 0.f};
         bool bad = false;
@@ -434,7 +421,7 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (n < 0)
                     bad = true;
                 else
-                    tc::stage_body<T, D>(qa, kt, kt + TILE, n, p.q_scale, o, m_run, l_run, lane);
+                    tc::stage_body_t<T, D>(qb, kt, kt + TILE, n, p.q_scale, o, m_run, l_run, lane);
                 __syncwarp();
             }
             if constexpr (MT > 1) {
@@ -452,66 +439,74 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
         }
+        // sums over the lanes holding the same heads (one per token pair)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 1);
-            l_run[r] += __shfl_xor_sync(kFull, l_run[r], 2);
+        for (int h = 0; h < 2; ++h) {
+            l_run[h] += __shfl_xor_sync(kFull, l_run[h], 4);
+            l_run[h] += __shfl_xor_sync(kFull, l_run[h], 8);
+            l_run[h] += __shfl_xor_sync(kFull, l_run[h], 16);
         }
         if (bad || abort) {
             // the piece contributes nothing
             m_run[0] = m_run[1] = -INFINITY;
             l_run[0] = l_run[1] = 0.f;
 #pragma unroll
-            for (int j = 0; j < DTILES; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         }
         const int first = sc.worker_of(pc.start);
         const int n_pieces = sc.worker_of(pc.start + pc.n_st - 1) - first + 1;
         if (n_pieces == 1) {
             T* out = reinterpret_cast<T*>(p.out) + ((size_t)pc.seq * p.H_q + h0) * D;
-            const float i0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
-            const float i1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+            const float ia = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
+            const float ib = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
 #pragma unroll
-            for (int j = 0; j < DTILES; ++j) {
-                const int col = 8 * j + 2 * tq;
-                if (r0 < G) {
-                    out[(size_t)r0 * D + col] = Elem<T>::from_f(o[j][0] * i0);
-                    out[(size_t)r0 * D + col + 1] = Elem<T>::from_f(o[j][1] * i0);
+            for (int j = 0; j < D / 16; ++j) {
+                const int d = 16 * j + gq;
+                if (ha < G) {
+                    out[(size_t)ha * D + d] = Elem<T>::from_f(o[j][0] * ia);
+                    out[(size_t)ha * D + d + 8] = Elem<T>::from_f(o[j][2] * ia);
                 }
-                if (r1 < G) {
-                    out[(size_t)r1 * D + col] = Elem<T>::from_f(o[j][2] * i1);
-                    out[(size_t)r1 * D + col + 1] = Elem<T>::from_f(o[j][3] * i1);
+                if (hb < G) {
+                    out[(size_t)hb * D + d] = Elem<T>::from_f(o[j][1] * ib);
+                    out[(size_t)hb * D + d + 8] = Elem<T>::from_f(o[j][3] * ib);
                 }
             }
             continue;
         }
-        // partial state of this piece -> its workspace slot
-        const size_t slot_id = (size_t)pc.seq * H_kv + pc.g + vw;
+        // partial state of this piece -> its workspace slot, then hand it to
+        // the merge warp (no wait here)
+        const int pair = pc.seq * H_kv + pc.g;
+        const size_t slot_id = (size_t)pair + vw;
         float* acc = p.ws_acc + slot_id * G * D;
         float* ml = p.ws_ml + slot_id * G * 2;
 #pragma unroll
-        for (int j = 0; j < DTILES; ++j) {
-            const int col = 8 * j + 2 * tq;
-            if (r0 < G)
-                *reinterpret_cast<float2*>(acc + (size_t)r0 * D + col) = make_float2(o[j][0], o[j][1]);
-            if (r1 < G)
-                *reinterpret_cast<float2*>(acc + (size_t)r1 * D + col) = make_float2(o[j][2], o[j][3]);
-        }
-        if (tq == 0) {
-            if (r0 < G) {
-                ml[r0 * 2] = m_run[0];
-                ml[r0 * 2 + 1] = l_run[0];
+        for (int j = 0; j < D / 16; ++j) {
+            const int d = 16 * j + gq;
+            if (ha < G) {
+                acc[(size_t)ha * D + d] = o[j][0];
+                acc[(size_t)ha * D + d + 8] = o[j][2];
             }
-            if (r1 < G) {
-                ml[r1 * 2] = m_run[1];
-                ml[r1 * 2 + 1] = l_run[1];
+            if (hb < G) {
+                acc[(size_t)hb * D + d] = o[j][1];
+                acc[(size_t)hb * D + d + 8] = o[j][3];
+            }
+        }
+        if (gq == 0) {
+            if (ha < G) {
+                ml[ha * 2] = m_run[0];
+                ml[ha * 2 + 1] = l_run[0];
+            }
+            if (hb < G) {
+                ml[hb * 2] = m_run[1];
+                ml[hb * 2 + 1] = l_run[1];
             }
         }
         // the worker barrier orders every warp's stores before the leader's
         // device-scope fence, which orders them before the counter update
         worker_sync<MT>(worker);
-        if (wtid == 0) {
+        if (mt == 0 && lane == 0) {
             __threadfence();
-            int* counter = p.counters + (size_t)pc.seq * H_kv + pc.g;
+            int* counter = p.counters + pair;
             const int last = atomicAdd(counter, 1) == n_pieces - 1;
             if (last) {
                 atomicExch(counter, 0);
@@ -520,14 +515,13 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
             flags[worker] = last;
         }
         worker_sync<MT>(worker);
-        if (flags[worker])
-            merge_pieces<T, D, MT>(p, pc.seq, pc.g, first, n_pieces, scratch, S::kMerge, wtid,
-                                   worker);
+        if (flags[worker]) merge_pair<T, D, MT * 32>(p, pair, first, n_pieces, mt * 32 + lane);
+        worker_sync<MT>(worker);   // the flag is read by every warp before it is reused
     }
     // no copy may outlive the CTA: after an abort, wait (bounded) for the
     // last stages issued
     if (abort && issuer)
-        for (int j = max(0, is.issued - RG); j < is.issued; ++j)
+        for (int j = max(0, is.count - RG); j < is.count; ++j)
             (void)mbar_wait(&full[j % RG], (uint32_t)((j / RG) & 1));
 }
 
@@ -547,7 +541,7 @@ int sm_count(int device) {
 
 template <typename T, int D, int MT>
 cudaError_t launch_lean_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                          int device, cudaStream_t st) {
+                          int device, cudaStream_t st, cudaEvent_t mid) {
     using S = LeanShape<D, MT>;
     constexpr int threads = S::TS * MT * 32;
     const int smem = (lean_fixed_smem<D, MT>() + (p.B + 1) * 4 + 15) & ~15;
@@ -565,21 +559,32 @@ cudaError_t launch_lean_t(const DecodeParams& p, const CUtensorMap* tk, const CU
         last_smem = smem;
     }
     const int grid = std::max(1, sm_count(device)) * last_per_sm;
-    return launch_kernel(kern, dim3(grid), dim3(threads), smem, st, p.pdl != 0, *tk, *tv, p);
+    e = launch_kernel(kern, dim3(grid), dim3(threads), smem, st, p.pdl != 0, *tk, *tv, p);
+    if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
+    return e;
 }
 
 template <typename T, int D>
 cudaError_t launch_lean_d(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                          int device, cudaStream_t st) {
-    switch ((p.G + 15) / 16) {
-        case 1: return launch_lean_t<T, D, 1>(p, tk, tv, device, st);
-        case 2: return launch_lean_t<T, D, 2>(p, tk, tv, device, st);
-        case 3: return launch_lean_t<T, D, 3>(p, tk, tv, device, st);
-        case 4: return launch_lean_t<T, D, 4>(p, tk, tv, device, st);
-        case 5: return launch_lean_t<T, D, 5>(p, tk, tv, device, st);
-        case 6: return launch_lean_t<T, D, 6>(p, tk, tv, device, st);
-        case 7: return launch_lean_t<T, D, 7>(p, tk, tv, device, st);
-        case 8: return launch_lean_t<T, D, 8>(p, tk, tv, device, st);
+                          int device, cudaStream_t st, cudaEvent_t mid) {
+    // warps of 8 query heads each
+    switch ((p.G + 7) / 8) {
+        case 1: return launch_lean_t<T, D, 1>(p, tk, tv, device, st, mid);
+        case 2: return launch_lean_t<T, D, 2>(p, tk, tv, device, st, mid);
+        case 3: return launch_lean_t<T, D, 3>(p, tk, tv, device, st, mid);
+        case 4: return launch_lean_t<T, D, 4>(p, tk, tv, device, st, mid);
+        case 5: return launch_lean_t<T, D, 5>(p, tk, tv, device, st, mid);
+        case 6: return launch_lean_t<T, D, 6>(p, tk, tv, device, st, mid);
+        case 7: return launch_lean_t<T, D, 7>(p, tk, tv, device, st, mid);
+        case 8: return launch_lean_t<T, D, 8>(p, tk, tv, device, st, mid);
+        case 9: return launch_lean_t<T, D, 9>(p, tk, tv, device, st, mid);
+        case 10: return launch_lean_t<T, D, 10>(p, tk, tv, device, st, mid);
+        case 11: return launch_lean_t<T, D, 11>(p, tk, tv, device, st, mid);
+        case 12: return launch_lean_t<T, D, 12>(p, tk, tv, device, st, mid);
+        case 13: return launch_lean_t<T, D, 13>(p, tk, tv, device, st, mid);
+        case 14: return launch_lean_t<T, D, 14>(p, tk, tv, device, st, mid);
+        case 15: return launch_lean_t<T, D, 15>(p, tk, tv, device, st, mid);
+        case 16: return launch_lean_t<T, D, 16>(p, tk, tv, device, st, mid);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -598,37 +603,43 @@ bool lean_supported(const pkv_pool* pool, int q_dtype, int group, int B, int max
     return (long long)B * stages < (1LL << 31) && sm_count(pool->device) > 0;
 }
 
-size_t lean_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads) {
-    const int G = n_q_heads / pool->n_kv_heads;
+// piece slots: pair + worker index
+size_t lean_slots(const pkv_pool* pool, int B) {
     const size_t pairs = (size_t)B * pool->n_kv_heads;
-    const size_t slots = pairs + (size_t)sm_count(pool->device) * kLeanMaxWorkersPerSm;
-    return align256(slots * G * 2 * sizeof(float)) +
-           align256(slots * G * pool->head_dim * sizeof(float)) + align256(pairs * sizeof(int));
+    return pairs + (size_t)sm_count(pool->device) * kLeanMaxWorkersPerSm;
 }
 
-cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, cudaStream_t st) {
-    const size_t pairs = (size_t)p.B * p.H_kv;
-    const size_t slots = pairs + (size_t)sm_count(pool->device) * kLeanMaxWorkersPerSm;
+size_t lean_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads) {
+    const int G = n_q_heads / pool->n_kv_heads;
+    const size_t slots = lean_slots(pool, B);
+    return align256(slots * G * 2 * sizeof(float)) +
+           align256(slots * G * pool->head_dim * sizeof(float)) +
+           align256((size_t)B * pool->n_kv_heads * sizeof(int));
+}
+
+cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, cudaStream_t st,
+                               cudaEvent_t mid) {
+    const size_t slots = lean_slots(pool, p.B);
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.ws_ml = reinterpret_cast<float*>(w);
     w += align256(slots * p.G * 2 * sizeof(float));
     p.ws_acc = reinterpret_cast<float*>(w);
     w += align256(slots * p.G * pool->head_dim * sizeof(float));
     if (!p.counters) {
-        // no persistent zeroed counters from the caller: use the workspace's
+        // no persistent zeroed counters from the caller: the workspace's
         p.counters = reinterpret_cast<int*>(w);
-        cudaError_t e = cudaMemsetAsync(p.counters, 0, pairs * sizeof(int), st);
+        cudaError_t e = cudaMemsetAsync(p.counters, 0, (size_t)p.B * p.H_kv * sizeof(int), st);
         if (e != cudaSuccess) return e;
     }
     const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(pool->tmap_k);
     const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(pool->tmap_v);
     if (pool->dtype == PKV_F16) {
-        if (pool->head_dim == 64) return launch_lean_d<__half, 64>(p, tk, tv, pool->device, st);
-        if (pool->head_dim == 128) return launch_lean_d<__half, 128>(p, tk, tv, pool->device, st);
+        if (pool->head_dim == 64) return launch_lean_d<__half, 64>(p, tk, tv, pool->device, st, mid);
+        if (pool->head_dim == 128) return launch_lean_d<__half, 128>(p, tk, tv, pool->device, st, mid);
     } else if (pool->dtype == PKV_BF16) {
-        if (pool->head_dim == 64) return launch_lean_d<__nv_bfloat16, 64>(p, tk, tv, pool->device, st);
+        if (pool->head_dim == 64) return launch_lean_d<__nv_bfloat16, 64>(p, tk, tv, pool->device, st, mid);
         if (pool->head_dim == 128)
-            return launch_lean_d<__nv_bfloat16, 128>(p, tk, tv, pool->device, st);
+            return launch_lean_d<__nv_bfloat16, 128>(p, tk, tv, pool->device, st, mid);
     }
     return cudaErrorInvalidValue;
 }

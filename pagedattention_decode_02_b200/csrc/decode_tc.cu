@@ -16,13 +16,15 @@
 // 8 x 16-byte ldmatrix read hits 8 different bank groups.  Loads are plain
 // (no multicast) from this GPU's own memory.
 //
-// CTA = (partition, KV head, sequence).  Warps: MT m-tiles of 16 query heads
-// (MT = ceil(G / 16)) x TS token groups.  Each token group owns a ring of
+// CTA = (partition, KV head, sequence).  Warps: MT warps of 8 query heads
+// (MT = ceil(G / 8)) x TS token groups.  Each token group owns a ring of
 // kStages slots; lane 0 of its first warp issues the copies, every warp of the
 // group consumes every stage, and with MT > 1 an "empty" mbarrier per slot
 // (MT arrivals) tells the producer when all of them are done with it.
-// The scores' accumulator fragments are re-packed in registers as the A
-// operand of the P.V product; online softmax runs in base 2 per head row.
+// A warp computes S^T = K Q^T and O^T += V^T P^T (16 tokens or 16 d-rows by
+// its 8 heads, so no padded rows up to 8 heads per KV head), P^T moving to
+// the B-operand layout by register transposes; online softmax in base 2 per
+// head.  The token groups' states are combined through shared memory.
 #include <cuda.h>
 
 #include <cfloat>
@@ -49,7 +51,7 @@ struct TcSmem {
 template <int D, int MT, int TS, int S>
 __host__ __device__ constexpr int tc_union_bytes() {
     const int tiles = TS * S * TcSmem<D>::kSlot;
-    const int comb = MT * TS * 16 * (D + 2) * 4;
+    const int comb = MT * TS * 8 * (D + 2) * 4;
     return ((tiles > comb ? tiles : comb) + 15) & ~15;
 }
 
@@ -63,7 +65,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr int TILE = TcSmem<D>::kTile;
     constexpr int SLOT = TcSmem<D>::kSlot;
     constexpr int KSTEPS = D / 16;       // k-steps of S = Q K^T
-    constexpr int DTILES = D / 8;        // n-tiles of O
     constexpr int HALVES = D / 64;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -72,7 +73,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;                                            // [TS][kStages][SLOT]
-    float* comb = reinterpret_cast<float*>(smem);                     // [NW][16][D + 2]
+    float* comb = reinterpret_cast<float*>(smem);                     // [NW][8][D + 2]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS, S>());
     uint64_t* empty = full + TS * kStages;
     int32_t* blk = reinterpret_cast<int32_t*>(empty + TS * kStages);   // the partition's block ids
@@ -177,16 +178,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         __syncwarp();
     };
 
-    // Q fragments (A operand) of this warp's 16 heads, zero past the group
-    const int gq = lane >> 2;       // fragment row (and row + 8)
-    const int tq = lane & 3;        // fragment column pair
-    uint32_t qa[KSTEPS][4];
-    tc::load_q_frags<T, D>(qa, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
-                           mt * 16, G, lane);
+    // Q^T fragments (B operand) of this warp's 8 heads, zero past the group
+    const int gq = lane >> 2;       // fragment row: d (and d + 8) of O^T
+    const int tq = lane & 3;        // this lane's heads: 2 tq, 2 tq + 1 of the warp's 8
+    uint32_t qb[KSTEPS][2];
+    tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
+                            mt * 8, G, lane);
 
-    float o[DTILES][4];
+    float o[D / 16][4];
 #pragma unroll
-    for (int j = 0; j < DTILES; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    for (int j = 0; j < D / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
 
@@ -207,7 +208,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int n = min(kStageTokens, t_end - a);
         uint8_t* kt = ring + slot * SLOT;
         uint8_t* vt = kt + TILE;
-        tc::stage_body<T, D>(qa, kt, vt, n, p.q_scale, o, m_run, l_run, lane);
+        tc::stage_body_t<T, D>(qb, kt, vt, n, p.q_scale, o, m_run, l_run, lane);
         __syncwarp();
         if constexpr (MT > 1) {
             if (lane == 0) mbar_arrive(&my_empty[slot]);
@@ -231,47 +232,49 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 (void)mbar_wait(&my_full[j % kStages], (uint32_t)((j / kStages) & 1));
     }
 
-    // full row sums: the four lanes of a quad hold disjoint token columns
+    // head sums: the lanes with the same lane % 4 hold disjoint tokens
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+    for (int h = 0; h < 2; ++h) {
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 4);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
     }
     __syncthreads();   // every ring slot consumed: the combine area may be written
-    // per-warp state -> shared memory [NW][16 rows][D + 2]
+    // per-warp state -> shared memory [NW][8 heads][D + 2]
     {
-        float* cw = comb + warp * 16 * (D + 2);
+        float* cw = comb + warp * 8 * (D + 2);
+        const int ra = 2 * tq, rb = ra + 1;
 #pragma unroll
-        for (int j = 0; j < DTILES; ++j) {
-            const int col = 8 * j + 2 * tq;
-            cw[gq * (D + 2) + col] = o[j][0];
-            cw[gq * (D + 2) + col + 1] = o[j][1];
-            cw[(gq + 8) * (D + 2) + col] = o[j][2];
-            cw[(gq + 8) * (D + 2) + col + 1] = o[j][3];
+        for (int j = 0; j < D / 16; ++j) {
+            const int d = 16 * j + gq;
+            cw[ra * (D + 2) + d] = o[j][0];
+            cw[rb * (D + 2) + d] = o[j][1];
+            cw[ra * (D + 2) + d + 8] = o[j][2];
+            cw[rb * (D + 2) + d + 8] = o[j][3];
         }
-        if (tq == 0) {
-            cw[gq * (D + 2) + D] = m_run[0];
-            cw[gq * (D + 2) + D + 1] = l_run[0];
-            cw[(gq + 8) * (D + 2) + D] = m_run[1];
-            cw[(gq + 8) * (D + 2) + D + 1] = l_run[1];
+        if (gq == 0) {
+            cw[ra * (D + 2) + D] = m_run[0];
+            cw[ra * (D + 2) + D + 1] = l_run[0];
+            cw[rb * (D + 2) + D] = m_run[1];
+            cw[rb * (D + 2) + D + 1] = l_run[1];
         }
     }
     __syncthreads();
-    // combine the token groups of each m-tile and write the G real heads
-    for (int i = tid; i < MT * 16 * D; i += NT) {
-        const int m_tile = i / (16 * D);
-        const int row = (i / D) % 16;
+    // combine the token groups of each 8-head group and write the G real heads
+    for (int i = tid; i < MT * 8 * D; i += NT) {
+        const int m_tile = i / (8 * D);
+        const int row = (i / D) % 8;
         const int d = i % D;
-        const int hrow = m_tile * 16 + row;
+        const int hrow = m_tile * 8 + row;
         if (hrow >= G) continue;
         float M = -INFINITY;
 #pragma unroll
         for (int t = 0; t < TS; ++t)
-            M = fmaxf(M, comb[((t * MT + m_tile) * 16 + row) * (D + 2) + D]);
+            M = fmaxf(M, comb[((t * MT + m_tile) * 8 + row) * (D + 2) + D]);
         float L = 0.f, O = 0.f;
 #pragma unroll
         for (int t = 0; t < TS; ++t) {
-            const float* cw = comb + ((t * MT + m_tile) * 16 + row) * (D + 2);
+            const float* cw = comb + ((t * MT + m_tile) * 8 + row) * (D + 2);
             const float w = M == -INFINITY ? 0.f : exp2f(cw[D] - M);
             L = fmaf(cw[D + 1], w, L);
             O = fmaf(cw[d], w, O);
@@ -325,17 +328,25 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUte
 template <typename T, int D>
 cudaError_t launch_tc_d(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                         int q_dtype, cudaStream_t st, cudaEvent_t mid) {
-    const int mt = (p.G + 15) / 16;
+    const int mt = (p.G + 7) / 8;
     switch (mt) {
-        // m-tiles of 16 heads x token groups: about 12 warps per CTA
+        // warps of 8 heads x token groups
         case 1: return launch_tc_t<T, D, 1, 4>(p, tk, tv, q_dtype, st, mid);
         case 2: return launch_tc_t<T, D, 2, 4>(p, tk, tv, q_dtype, st, mid);
-        case 3: return launch_tc_t<T, D, 3, 4>(p, tk, tv, q_dtype, st, mid);
-        case 4: return launch_tc_t<T, D, 4, 3>(p, tk, tv, q_dtype, st, mid);
+        case 3: return launch_tc_t<T, D, 3, 3>(p, tk, tv, q_dtype, st, mid);
+        case 4: return launch_tc_t<T, D, 4, 2>(p, tk, tv, q_dtype, st, mid);
         case 5: return launch_tc_t<T, D, 5, 2>(p, tk, tv, q_dtype, st, mid);
         case 6: return launch_tc_t<T, D, 6, 2>(p, tk, tv, q_dtype, st, mid);
-        case 7: return launch_tc_t<T, D, 7, 2>(p, tk, tv, q_dtype, st, mid);
-        case 8: return launch_tc_t<T, D, 8, 2>(p, tk, tv, q_dtype, st, mid);
+        case 7: return launch_tc_t<T, D, 7, 1>(p, tk, tv, q_dtype, st, mid);
+        case 8: return launch_tc_t<T, D, 8, 1>(p, tk, tv, q_dtype, st, mid);
+        case 9: return launch_tc_t<T, D, 9, 1>(p, tk, tv, q_dtype, st, mid);
+        case 10: return launch_tc_t<T, D, 10, 1>(p, tk, tv, q_dtype, st, mid);
+        case 11: return launch_tc_t<T, D, 11, 1>(p, tk, tv, q_dtype, st, mid);
+        case 12: return launch_tc_t<T, D, 12, 1>(p, tk, tv, q_dtype, st, mid);
+        case 13: return launch_tc_t<T, D, 13, 1>(p, tk, tv, q_dtype, st, mid);
+        case 14: return launch_tc_t<T, D, 14, 1>(p, tk, tv, q_dtype, st, mid);
+        case 15: return launch_tc_t<T, D, 15, 1>(p, tk, tv, q_dtype, st, mid);
+        case 16: return launch_tc_t<T, D, 16, 1>(p, tk, tv, q_dtype, st, mid);
         default: return cudaErrorInvalidValue;
     }
 }

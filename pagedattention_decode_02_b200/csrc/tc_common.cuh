@@ -212,5 +212,118 @@ __device__ __forceinline__ void stage_body(const uint32_t (&qa)[D / 16][4], uint
     }
 }
 
+
+// Transpose of an 8x8 b16 matrix held one 32-bit pair per lane in the mma
+// fragment layout (row lane / 4, columns 2 (lane % 4) and + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+// Q^T fragments (mma B operand, K = d, N = 8 heads) of heads head_base ..
+// head_base + 7 of the [heads][D] block at q: per 16-wide k-step, the pairs
+// (d = 16 kk + 2 (lane % 4), + 1) and (+ 8, + 9) of head head_base + lane / 4;
+// zero for heads >= n_heads.
+template <typename T, int D>
+__device__ __forceinline__ void load_qT_frags(uint32_t (&qb)[D / 16][2], const T* q, int head_base,
+                                              int n_heads, int lane) {
+    const int h = head_base + (lane >> 2);
+    const int tq = lane & 3;
+    const T* qh = q + (size_t)h * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const int c0 = kk * 16 + 2 * tq;
+        qb[kk][0] = h < n_heads ? *reinterpret_cast<const uint32_t*>(qh + c0) : 0u;
+        qb[kk][1] = h < n_heads ? *reinterpret_cast<const uint32_t*>(qh + c0 + 8) : 0u;
+    }
+}
+
+// One 16-token stage for one warp's 8 query heads, in transposed form (no
+// padded rows when a KV head has 8 or fewer query heads):
+//     S^T [16 tokens][8 heads] = K_stage Q^T,
+//     online softmax per head (column) in base 2,
+//     O^T [D][8 heads] = alpha O^T + V_stage^T P^T.
+// P^T moves from the accumulator layout to the B-operand layout with two 8x8
+// transposes (movmatrix).  This lane holds heads 2 (lane % 4) and + 1:
+// m_run / l_run (l partial over this lane's tokens, summed over the lanes of
+// the same lane % 4 at the end), o[mt] = O^T rows d = 16 mt + lane / 4 (and
+// + 8) for those two heads.  Same staging and zeroing rules as stage_body.
+template <typename T, int D>
+__device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], uint8_t* kt,
+                                             uint8_t* vt, int n, float q_scale,
+                                             float (&o)[D / 16][4], float (&m_run)[2],
+                                             float (&l_run)[2], int lane) {
+    constexpr int KSTEPS = D / 16;
+    const int gq = lane >> 2;
+    if (n < kStageTokens) {
+        for (int i = lane; i < (kStageTokens - n) * (D / 8); i += 32) {
+            const int r = n + i / (D / 8), cc = i % (D / 8);
+            *reinterpret_cast<uint4*>(vt + swz(r, cc)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+    }
+    const uint32_t kbase = smem_addr(kt);
+    const uint32_t vbase = smem_addr(vt);
+    const int mi = lane >> 3, r8 = lane & 7;
+
+    // S^T = K Q^T over the d k-steps, four interleaved accumulators
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(kbase + swz((mi & 1) * 8 + r8, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
+        MmaType<T>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
+    }
+    float s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
+    // tokens gq (s[0], s[1]) and gq + 8 (s[2], s[3]); heads 2 tq (even e), 2 tq + 1
+    if (gq >= n) s[0] = s[1] = -INFINITY;
+    if (gq + 8 >= n) s[2] = s[3] = -INFINITY;
+    float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+    }
+    float alpha[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float m_new = fmaxf(m_run[h], mx[h]);
+        alpha[h] = exp2f(m_run[h] - m_new);
+        m_run[h] = m_new;
+    }
+    const float p0 = exp2f(s[0] - m_run[0]);
+    const float p1 = exp2f(s[1] - m_run[1]);
+    const float p2 = exp2f(s[2] - m_run[0]);
+    const float p3 = exp2f(s[3] - m_run[1]);
+    l_run[0] = l_run[0] * alpha[0] + (p0 + p2);
+    l_run[1] = l_run[1] * alpha[1] + (p1 + p3);
+    // P^T as the B operand: b0 = tokens 0-7, b1 = tokens 8-15
+    const uint32_t pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(MmaType<T>::pack(p2, p3));
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            o[mt][0] *= alpha[0];
+            o[mt][1] *= alpha[1];
+            o[mt][2] *= alpha[0];
+            o[mt][3] *= alpha[1];
+        }
+    }
+    // O^T += V^T P^T: one m-tile of 16 d rows per transposed ldmatrix
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_t(vbase + swz((mi >> 1) * 8 + r8, 2 * mt + (mi & 1)), a[0], a[1], a[2], a[3]);
+        MmaType<T>::mma(o[mt], a, pb0, pb1);
+    }
+}
+
 }  // namespace tc
 }  // namespace pkv

@@ -1,8 +1,8 @@
-"""GPU parity of the stage-balanced tensor-core decode (persistent CTAs that
-share the batch's 16-token stages equally, split pairs merged in the kernel)
+"""GPU parity of the stage-balanced tensor-core decode (persistent workers that
+share the batch's 16-token stages equally, split pairs merged by a second launch)
 against the CPU oracle: block sizes, head groupings, ragged and degenerate
 batches, pairs split over many CTAs, invalid lengths and block ids, and the
-decode-step runtime's persistent merge counters over many rounds."""
+decode-step runtime over many rounds."""
 
 import dataclasses
 
@@ -65,7 +65,7 @@ def test_lean_many_short_sequences():
 
 
 def test_lean_mixed_lengths_auto_choice():
-    # the automatic choice for grouped heads is the stage-balanced kernel
+    # the automatic choice and the stage-balanced kernel, round after round
     cfg = small("llama2_70b", n_q_heads=32, n_kv_heads=4, head_dim=128, block_size=16, batch=40,
                 lengths=("loguniform", 1, 3000))
     side = setup_config(cfg, seed=13, growth=2)
@@ -115,8 +115,7 @@ def test_lean_refuses_unsupported():
 
 @pytest.mark.parametrize("hq,hkv", [(64, 8), (71, 1)])
 def test_lean_step_runtime_many_rounds(hq, hkv):
-    # the runtime's merge counters are reset by the kernel itself: every round
-    # of a multi-round run must merge correctly
+    # every round of a multi-round run must merge its split pairs correctly
     d = 128 if hkv == 8 else 64
     dt = "bf16" if hkv == 8 else "f16"
     cfg = small("llama2_70b", n_q_heads=hq, n_kv_heads=hkv, head_dim=d, kv_dtype=dt, q_dtype=dt,
@@ -132,7 +131,7 @@ def test_lean_step_runtime_many_rounds(hq, hkv):
         pk.pkv_decode_step(step, seqs, to_torch(q, dt), to_torch(kn, dt), to_torch(vn, dt),
                            cfg.scale, out)
         if r > 0:                               # tables already resident
-            assert step.last_launches == 2      # prologue + one decode launch
+            assert step.last_launches == 2      # prologue + decode (merge included)
         side.orc.append(list(seqs), kn, vn, dt)
         ref = side.orc.attend(list(seqs), q, dt, cfg.scale)
         torch.cuda.synchronize()

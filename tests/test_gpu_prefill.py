@@ -40,7 +40,8 @@ def run_prefill(side, prompt_lens, seed=0):
     torch.cuda.synchronize()
     assert pk.pkv_device_error(side.pool) == 0
     gpu = to_f64(from_torch(out, cfg.q_dtype), cfg.q_dtype)
-    refs = [side.orc.prefill(s, q, cfg.q_dtype, cfg.scale) for s, q in zip(seqs, qs)]
+    refs = [side.orc.prefill(s, q, cfg.q_dtype, cfg.scale) if q.shape[0] else None
+            for s, q in zip(seqs, qs)]
     return [gpu[starts[i]:starts[i + 1]] for i in range(len(seqs))], refs
 
 
