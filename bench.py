@@ -79,6 +79,18 @@ def config_of(args) -> wl.Config:
 # sources hash to the recorded value, else the bench reports null.
 TRAFFIC = {
     # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
+    # profiles/decode_tc_llama2_70b.md: 294.4 MB for 286.8 MB algorithmic
+    ("llama2_70b", "decode_tc_kernel"):
+        (1.0266, "64993f722e108d3f270476fd336f1c328cea2890f477cafaf1d50ee1b5ca059c"),
+    # profiles/decode_simt2_opt13b.md: 612.6 MB for 604.7 MB
+    ("opt13b", "decode_simt2_kernel"):
+        (1.0130, "fe50e5e6c9b614ccf5d80f6e9ea95a9211cc28a339e220d3e95e5f4d9068cef3"),
+    # profiles/decode_simt2_fp8.md: 1,360.9 MB for 1,344.8 MB
+    ("fp8", "decode_simt2_kernel"):
+        (1.0120, "fe50e5e6c9b614ccf5d80f6e9ea95a9211cc28a339e220d3e95e5f4d9068cef3"),
+    # profiles/decode_lean_falcon7b.md: the 8.3 MB batch is served from L2
+    ("falcon7b", "decode_lean_kernel"):
+        (0.357, "3a1be74a29e84db6960699d5114a3efe634083a65bcd43938bde18213566b812"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
