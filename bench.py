@@ -59,9 +59,10 @@ def parse():
     ap.add_argument("--kernel", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
+    ap.add_argument("--mode", choices=["decode", "prefill", "swap"], default="decode",
                     help="prefill: the prompt phase of the workload's batch (every history "
-                         "attended causally as one prompt)")
+                         "attended causally as one prompt); swap: one sequence's blocks out to "
+                         "pinned host memory and back, per block size")
     return ap.parse_args()
 
 
@@ -676,12 +677,72 @@ def run_prefill(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_swap(args) -> None:
+    """Preemption by swapping ("KV 缓存与分页注意力" §放不下的时候: the blocks go
+    to CPU memory and come back when the sequence's turn comes): one sequence
+    of the workload's shape (2,048 tokens) swapped out to pinned host buffers
+    and back in, for every block size 1 .. 64; bytes moved per second each
+    way.  The page reports that swapping is slower for small blocks."""
+    import torch
+
+    import pagedattention_decode_02_b200 as pk
+
+    torch.cuda.set_device(0)
+    cfg = config_of(args)
+    K, W = args.steps, args.warmup
+    n_tok = 2048
+    res = {}
+    stream = torch.cuda.current_stream()
+    for bs in (1, 2, 4, 8, 16, 32, 64):
+        nb = -(-n_tok // bs) + 4
+        pool = pk.kv_pool_create(nb, bs, cfg.n_kv_heads, cfg.head_dim, cfg.kv_dtype)
+        kb, vb = pool.device_buffers()
+        kb.copy_(torch.randint(0, 120, kb.shape, dtype=torch.uint8, device="cuda"))
+        vb.copy_(torch.randint(0, 120, vb.shape, dtype=torch.uint8, device="cuda"))
+        blk = pk.block_bytes(pool)
+        n_blocks = -(-n_tok // bs)
+        hk = torch.empty(n_blocks * blk, dtype=torch.uint8).pin_memory()
+        hv = torch.empty(n_blocks * blk, dtype=torch.uint8).pin_memory()
+        pk.bt_alloc(pool, 0, n_tok)
+        t_out = t_in = 0.0
+        for i in range(W + K):
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record()
+            pk.kv_swap_out(pool, 0, hk, hv, stream=stream)
+            e1.record()
+            pk.kv_swap_in(pool, 0, hk, hv, n_tok, stream=stream)
+            e2.record()
+            torch.cuda.synchronize()
+            if i >= W:
+                t_out += e0.elapsed_time(e1)
+                t_in += e1.elapsed_time(e2)
+        moved = 2.0 * n_blocks * blk
+        res[str(bs)] = {"bytes": int(moved), "out_gbs": round(moved * K / (t_out / 1e3) / 1e9, 2),
+                        "in_gbs": round(moved * K / (t_in / 1e3) / 1e9, 2),
+                        "out_us": round(t_out / K * 1e3, 2), "in_us": round(t_in / K * 1e3, 2)}
+        if pk.pkv_device_error(pool):
+            raise SystemExit("device error")
+        pool.close()
+    best = max(v["in_gbs"] for v in res.values())
+    print(json.dumps({
+        "metric": "KV swap GB/s per block size (device <-> pinned host, one 2048-token sequence)",
+        "value": res["16"]["in_gbs"], "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": W,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.kv_dtype,
+        "data": "synthetic (random pool bytes)",
+        "config": {"workload": f"one {n_tok}-token sequence of {cfg.description}",
+                   "per_block_size": res, "best_in_gbs": best},
+        "gpu_launches": 2 * K,
+    }), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.mode == "prefill":
         run_prefill(args)
+    elif args.mode == "swap":
+        run_swap(args)
     else:
         run_ours(args)
 

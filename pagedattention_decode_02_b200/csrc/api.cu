@@ -312,7 +312,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                  cudaEvent_t ev_begin, cudaEvent_t ev_mid, cudaEvent_t ev_end,
                                  int* counters = nullptr, bool pdl = false,
                                  const int32_t* table_rows = nullptr, int n_table_rows = 0,
-                                 int* n_launches = nullptr, int* kernel_used = nullptr) {
+                                 int* n_launches = nullptr, int* kernel_used = nullptr,
+                                 const int32_t* order = nullptr) {
     if (n_launches) *n_launches = 0;
     if (kernel_used) *kernel_used = 0;
     if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
@@ -386,6 +387,7 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     dp.pdl = pdl ? 1 : 0;
     dp.table_rows = table_rows;
     dp.n_table_rows = n_table_rows;
+    dp.order = order;
     const float log2e = 1.4426950408889634f;
     dp.q_scale = scale * log2e * p->k_scale;
     dp.v_scale = p->v_scale;
@@ -494,7 +496,7 @@ struct pkv_step {
     int max_batch = 0, max_seqs = 0, max_blocks = 0, n_q_heads = 0;
     pkv_dtype q_dtype = PKV_F16;
     int partition_tokens = 0, kernel = PKV_KERNEL_AUTO;
-    // device: slots | cow src | cow dst | lens | rows  (max_batch each)
+    // device: slots | cow src | cow dst | lens | rows | order  (max_batch each)
     //         | staged tables [max_batch][max_blocks]  (fallback path)
     int32_t* h_stage[kRing] = {};
     cudaEvent_t ev[kRing] = {};
@@ -517,6 +519,7 @@ struct pkv_step {
     std::vector<int32_t> mirror;      // [max_seqs][max_blocks]
     // one round's host scratch
     std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_cow_rows, h_upd_idx, h_upd_val;
+    std::vector<int32_t> h_lens, h_order;   // fast path: lengths, launch order
     pkv::StepArgs args;
     long long fast_rounds = 0, slow_rounds = 0;
     // profiling: every prof_every-th round records four events (before the
@@ -619,7 +622,7 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_
     s->q_dtype = q_dtype;
     s->partition_tokens = partition_tokens;
     s->kernel = kernel;
-    const size_t stage_ints = (size_t)5 * max_batch + (size_t)max_batch * max_blocks;
+    const size_t stage_ints = (size_t)6 * max_batch + (size_t)max_batch * max_blocks;
     bool ok = true;
     for (int i = 0; i < pkv_step::kRing && ok; ++i) {
         ok &= cudaMallocHost(&s->h_stage[i], stage_ints * sizeof(int32_t)) == cudaSuccess;
@@ -712,7 +715,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         s->h_rows[i] = r;
     }
     const size_t limit = (size_t)pkv::kStepArgInts;
-    const size_t fixed = (size_t)3 * B + 3 * (size_t)n_cow;
+    const size_t fixed = (size_t)4 * B + 3 * (size_t)n_cow;
     bool fits = fixed <= limit;
     for (int i = 0; i < B && fits; ++i) {
         const pkv::Sequence* sq = pool->bm.find(seq_ids[i]);
@@ -731,6 +734,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     int launches = 0;
     int32_t* d_lens = s->d_stage + 3 * mb;
     int32_t* d_rows = s->d_stage + 4 * mb;
+    int32_t* d_order = s->d_stage + 5 * mb;
     cudaEvent_t e_pre = nullptr, e0 = nullptr, e1 = nullptr, e2 = nullptr;
     const bool profiled =
         s->prof_n > 0 && ((s->round - 1 - s->prof_start) % s->prof_every) == 0;
@@ -749,12 +753,24 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         a.n_cow = n_cow;
         a.n_upd = (int32_t)s->h_upd_idx.size();
         a.table_cap = s->max_seqs * s->max_blocks;
+        // launch slots longest context first, so that the long sequences'
+        // partitions start in the first waves and the short ones fill the last
+        s->h_lens.resize(B);
+        s->h_order.resize(B);
+        for (int i = 0; i < B; ++i) {
+            s->h_lens[i] = (int32_t)pool->bm.find(seq_ids[i])->length;
+            s->h_order[i] = i;
+        }
+        std::stable_sort(s->h_order.begin(), s->h_order.end(),
+                         [&](int32_t x, int32_t y) { return s->h_lens[x] > s->h_lens[y]; });
         int32_t* d = a.data;
         for (int i = 0; i < B; ++i) d[i] = s->h_slots[i];
         d += B;
-        for (int i = 0; i < B; ++i) d[i] = (int32_t)pool->bm.find(seq_ids[i])->length;
+        for (int z = 0; z < B; ++z) d[z] = s->h_lens[s->h_order[z]];
         d += B;
-        for (int i = 0; i < B; ++i) d[i] = s->h_rows[i];
+        for (int z = 0; z < B; ++z) d[z] = s->h_rows[s->h_order[z]];
+        d += B;
+        for (int z = 0; z < B; ++z) d[z] = s->h_order[z];
         d += B;
         for (int j = 0; j < n_cow; ++j) d[j] = s->h_src[j];
         d += n_cow;
@@ -767,7 +783,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_val[u];
         cudaError_t e = pkv::launch_step_prologue(
             a, pool->k, pool->v, k_new, v_new, s->q_dtype, pool->dtype, s->d_tables, d_lens,
-            d_rows, pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale,
+            d_rows, d_order, pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale,
             pool->v_scale, pool->d_err, st);
         if (e != cudaSuccess) return PKV_ERR_CUDA;
         launches = 1;
@@ -787,17 +803,17 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
             h[2 * mb + j] = s->h_dst[j];
         }
         for (int i = 0; i < B; ++i) h[4 * mb + i] = s->h_rows[i];
-        int32_t* ht = h + 5 * mb;
+        int32_t* ht = h + 6 * mb;
         ps = pool->bm.export_tables(seq_ids, B, s->max_blocks, ht, h + 3 * mb, nullptr);
         if (ps != PKV_OK) return ps;   // cannot happen after the checks above
-        const size_t ints = (size_t)5 * mb + (size_t)B * s->max_blocks;
+        const size_t ints = (size_t)6 * mb + (size_t)B * s->max_blocks;
         if (cudaMemcpyAsync(s->d_stage, h, ints * sizeof(int32_t), cudaMemcpyHostToDevice, st) !=
                 cudaSuccess ||
             cudaEventRecord(s->ev[r], st) != cudaSuccess)
             return PKV_ERR_CUDA;
         s->pending[r] = true;
         s->ring = (r + 1) % pkv_step::kRing;
-        if (pkv::launch_scatter_rows(s->d_stage + 5 * mb, d_rows, B, s->max_blocks, s->d_tables,
+        if (pkv::launch_scatter_rows(s->d_stage + 6 * mb, d_rows, B, s->max_blocks, s->d_tables,
                                      st) != cudaSuccess)
             return PKV_ERR_CUDA;
         ++launches;
@@ -826,7 +842,8 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     ps = decode_attention_impl(pool, q, s->q_dtype, s->d_tables, s->max_blocks, d_lens, B,
                                s->n_q_heads, scale, out, s->d_ws, s->ws_bytes, s->partition_tokens,
                                s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled,
-                               d_rows, s->max_seqs, &decode_launches, &s->last_kernel);
+                               d_rows, s->max_seqs, &decode_launches, &s->last_kernel,
+                               fits ? d_order : nullptr);
     if (ps != PKV_OK) return ps;
     if (profiled) ++s->prof_count;
     launches += decode_launches;

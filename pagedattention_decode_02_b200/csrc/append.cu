@@ -127,14 +127,16 @@ __global__ void kv_append_copy_kernel(uint8_t* k_pool, uint8_t* v_pool, const in
 template <typename IN, bool FP8>
 __global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t* k_pool,
                                      uint8_t* v_pool, const IN* k, const IN* v, int32_t* tables,
-                                     int32_t* lens, int32_t* rows, int H, int D, int bs,
-                                     int num_blocks, float k_scale, float v_scale, uint32_t* err) {
+                                     int32_t* lens, int32_t* rows, int32_t* order, int H, int D,
+                                     int bs, int num_blocks, float k_scale, float v_scale,
+                                     uint32_t* err) {
     allow_dependent_launch();   // the decode kernel may start its launch now
     const int B = a.B;
     const int32_t* slots = a.data;
     const int32_t* lens_in = a.data + B;
     const int32_t* rows_in = a.data + 2 * B;
-    const int32_t* cow_src = a.data + 3 * B;
+    const int32_t* order_in = a.data + 3 * B;
+    const int32_t* cow_src = a.data + 4 * B;
     const int32_t* cow_dst = cow_src + a.n_cow;
     const int32_t* cow_rows = cow_dst + a.n_cow;
     const int32_t* upd_idx = cow_rows + a.n_cow;
@@ -147,6 +149,7 @@ __global__ void step_prologue_kernel(const __grid_constant__ StepArgs a, uint8_t
         for (long long i = first; i < B; i += stride) {
             lens[i] = lens_in[i];
             rows[i] = rows_in[i];
+            order[i] = order_in[i];
         }
         for (long long u = first; u < a.n_upd; u += stride) {
             const int idx = upd_idx[u];
@@ -284,9 +287,9 @@ namespace pkv {
 
 cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
                                  const void* k, const void* v, int in_dtype, int kv_dtype,
-                                 int32_t* tables, int32_t* lens, int32_t* rows, int H, int D,
-                                 int bs, int num_blocks, float k_scale, float v_scale,
-                                 uint32_t* err, cudaStream_t st) {
+                                 int32_t* tables, int32_t* lens, int32_t* rows, int32_t* order,
+                                 int H, int D, int bs, int num_blocks, float k_scale,
+                                 float v_scale, uint32_t* err, cudaStream_t st) {
     constexpr int kThreads = 256;
     const int eb = kv_dtype == PKV_F32 ? 4 : kv_dtype == PKV_FP8_E4M3 ? 1 : 2;
     const int chunks_per_row = kv_dtype == PKV_FP8_E4M3 ? D / 16 : D * eb / 16;
@@ -301,29 +304,29 @@ cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_
         switch (in_dtype) {
             case PKV_F32:
                 step_prologue_kernel<float, true><<<grid, kThreads, 0, st>>>(
-                    a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, H, D, bs,
+                    a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, order, H, D, bs,
                     num_blocks, k_scale, v_scale, err);
                 break;
             case PKV_F16:
                 step_prologue_kernel<__half, true><<<grid, kThreads, 0, st>>>(
-                    a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, H, D, bs,
+                    a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, order, H, D, bs,
                     num_blocks, k_scale, v_scale, err);
                 break;
             case PKV_BF16:
                 step_prologue_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, st>>>(
                     a, k_pool, v_pool, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, tables,
-                    lens, rows, H, D, bs, num_blocks, k_scale, v_scale, err);
+                    lens, rows, order, H, D, bs, num_blocks, k_scale, v_scale, err);
                 break;
             default:
                 return cudaErrorInvalidValue;
         }
     } else if (kv_dtype == PKV_F32) {
         step_prologue_kernel<float, false><<<grid, kThreads, 0, st>>>(
-            a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, H, D, bs,
+            a, k_pool, v_pool, (const float*)k, (const float*)v, tables, lens, rows, order, H, D, bs,
             num_blocks, k_scale, v_scale, err);
     } else {
         step_prologue_kernel<__half, false><<<grid, kThreads, 0, st>>>(
-            a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, H, D, bs,
+            a, k_pool, v_pool, (const __half*)k, (const __half*)v, tables, lens, rows, order, H, D, bs,
             num_blocks, k_scale, v_scale, err);
     }
     return cudaGetLastError();

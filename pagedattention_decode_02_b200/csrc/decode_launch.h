@@ -68,10 +68,12 @@ cudaError_t launch_prefill(const PrefillParams& p, const pkv_pool* pool, cudaStr
 
 // One decode round's small host-side results, passed by value as kernel
 // parameters (no separate host-to-device copy):
-//   data = slots[B] | lens[B] | rows[B] | cow_src[n_cow] | cow_dst[n_cow]
-//          | cow_rows[n_cow] | upd_idx[n_upd] | upd_val[n_upd]
-// rows[i] = persistent table row of sequence i; cow_rows[j] = rows of the
-// shared block to copy (the fill before the write); upd_* = changed
+//   data = slots[B] | lens[B] | rows[B] | order[B] | cow_src[n_cow]
+//          | cow_dst[n_cow] | cow_rows[n_cow] | upd_idx[n_upd] | upd_val[n_upd]
+// slots[i] = append slot of the caller's sequence i; lens, rows and order are
+// by launch slot (longest context first): order[z] = the caller's index of
+// launch slot z, rows[z] = its persistent table row; cow_rows[j] = rows of
+// the shared block to copy (the fill before the write); upd_* = changed
 // block-table entries (flat index into [table rows][max_blocks]).
 constexpr int kStepArgInts = 990;   // the whole parameter block stays under 4 KB
 struct StepArgs {
@@ -79,14 +81,15 @@ struct StepArgs {
     int32_t data[kStepArgInts];
 };
 
-// The round's prologue in one launch: lengths and table updates into the
-// persistent device tables, copy-on-write of the shared rows, append of the
-// B new rows (FP8 pools quantise).
+// The round's prologue in one launch: lengths, rows and launch order by
+// launch slot and table updates into the persistent device tables,
+// copy-on-write of the shared rows, append of the B new rows (FP8 pools
+// quantise).
 cudaError_t launch_step_prologue(const StepArgs& a, uint8_t* k_pool, uint8_t* v_pool,
                                  const void* k, const void* v, int in_dtype, int kv_dtype,
-                                 int32_t* tables, int32_t* lens, int32_t* rows, int n_kv_heads,
-                                 int head_dim, int block_size, int num_blocks, float k_scale,
-                                 float v_scale, uint32_t* err, cudaStream_t st);
+                                 int32_t* tables, int32_t* lens, int32_t* rows, int32_t* order,
+                                 int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                                 float k_scale, float v_scale, uint32_t* err, cudaStream_t st);
 
 // Copy staged full tables ([B][max_blocks]) into their persistent rows.
 cudaError_t launch_scatter_rows(const int32_t* staged, const int32_t* rows, int B, int max_blocks,

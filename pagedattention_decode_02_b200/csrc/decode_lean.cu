@@ -112,7 +112,7 @@ __device__ __noinline__ void merge_pair(const DecodeParams& p, int pair, int fir
                                         int t) {
     constexpr int E = 4;
     const int G = p.G;
-    const int seq = pair / p.H_kv, g = pair % p.H_kv;
+    const int seq = seq_of(p, pair / p.H_kv), g = pair % p.H_kv;
     const int total = G * (D / 4);
     const size_t slot0 = (size_t)pair + first;
     const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + slot0 * G;
@@ -347,10 +347,10 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
 
     // sequences with an invalid length: zero output, error bit
-    for (int seq = blockIdx.x; seq < B; seq += gridDim.x) {
-        if (pre[seq + 1] != pre[seq]) continue;
+    for (int slot = blockIdx.x; slot < B; slot += gridDim.x) {
+        if (pre[slot + 1] != pre[slot]) continue;
         if (tid == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
-        T* out = reinterpret_cast<T*>(p.out) + (size_t)seq * p.H_q * D;
+        T* out = reinterpret_cast<T*>(p.out) + (size_t)seq_of(p, slot) * p.H_q * D;
         for (int i = tid; i < p.H_q * D; i += NT) out[i] = Elem<T>::from_f(0.f);
     }
 
@@ -396,8 +396,9 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const Piece pc = sc.at(pos, hi);
         pos = pc.start + pc.s1;
         const int h0 = pc.g * G;
+        const int oseq = seq_of(p, pc.seq);   // pieces walk launch slots
         uint32_t qb[D / 16][2];
-        tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)pc.seq * p.H_q + h0) * D,
+        tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)oseq * p.H_q + h0) * D,
                                 hw, G, lane);
         float o[D / 16][4];
 #pragma unroll
@@ -456,7 +457,7 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int first = sc.worker_of(pc.start);
         const int n_pieces = sc.worker_of(pc.start + pc.n_st - 1) - first + 1;
         if (n_pieces == 1) {
-            T* out = reinterpret_cast<T*>(p.out) + ((size_t)pc.seq * p.H_q + h0) * D;
+            T* out = reinterpret_cast<T*>(p.out) + ((size_t)oseq * p.H_q + h0) * D;
             const float ia = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f;
             const float ib = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
 #pragma unroll

@@ -129,7 +129,7 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
 
     const int part = blockIdx.x;
     const int h0 = blockIdx.y * HPC;
-    const int seq = blockIdx.z;
+    const int slot = blockIdx.z;   // launch slot: length and table row
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -137,7 +137,8 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
     const int bs = p.block_size;
     const int P = p.part_tokens;
 
-    const int c = p.lens[seq];
+    const int c = p.lens[slot];
+    const int seq = seq_of(p, slot);   // the caller's sequence: q, out, partials
     const int max_ctx = p.max_blocks * bs;
     if (c < 1 || c > max_ctx) {
         // invalid length: partition 0 zeroes the output, nothing is read
@@ -157,7 +158,7 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
     const int n_lb = (t_end - 1) / bs - lb0 + 1;
 
     // the partition's block ids, validated once
-    const long long trow = table_row(p, seq);
+    const long long trow = table_row(p, slot);
     bool bad = trow < 0;
     for (int i = tid; i < n_lb && trow >= 0; i += kThreads) {
         int32_t b = p.tables[trow * p.max_blocks + lb0 + i];
@@ -349,10 +350,11 @@ merge_kernel(const DecodeParams p) {
     constexpr int VEC = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x * kMergeWarps + warp;
-    const int seq = blockIdx.y;
+    const int slot = blockIdx.y;
     grid_dependency_wait();   // the decode kernel's partials (programmatic launch)
     if (h >= p.H_q) return;
-    const int c = p.lens[seq];
+    const int c = p.lens[slot];
+    const int seq = seq_of(p, slot);
     if (c < 1 || c > p.max_blocks * p.block_size) return;   // zeroed by the decode kernel
     const int nparts = (c + p.part_tokens - 1) / p.part_tokens;
     if (nparts <= 1) return;                                   // written by the decode kernel

@@ -80,7 +80,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     const int part = blockIdx.x;
     const int g = blockIdx.y;
-    const int seq = blockIdx.z;
+    const int slot = blockIdx.z;   // launch slot: length and table row
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -93,8 +93,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     __shared__ int last_flag;
     grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
-    const long long trow = table_row(p, seq);   // issued together with the length load
-    const int c = p.lens[seq];
+    const long long trow = table_row(p, slot);   // issued together with the length load
+    const int c = p.lens[slot];
+    const int seq = seq_of(p, slot);             // the caller's sequence: q, out, partials
     if (c < 1 || c > p.max_blocks * bs) {
         if (part == 0) {
             if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);

@@ -250,8 +250,11 @@ struct DecodeParams {
     const int32_t* lens;
     float* ws_ml;    // [B][H_q][max_parts][2]  (running max in log2 units, sum)
     float* ws_acc;   // [B][H_q][max_parts][D]  (unnormalised accumulator)
-    const int32_t* table_rows;  // [B] row of `tables` holding sequence i's table, or null
+    const int32_t* table_rows;  // [B] row of `tables` holding launch slot i's table, or null
                                 // (row i); rows outside [0, n_table_rows) are rejected
+    const int32_t* order;       // [B] launch slot -> the caller's sequence index (q, out,
+                                // partials), or null (identity); lens and table_rows are
+                                // indexed by launch slot
     int n_table_rows;
     int pdl;         // host side: launch with programmatic stream serialization
     int* counters;   // [B][H_q] partitions finished, or null: when set, the last
@@ -272,12 +275,17 @@ struct DecodeParams {
 
 namespace pkv {
 
-// Row of the block-table array that holds sequence `seq`'s table; -1 if the
-// row index is out of range.
-__device__ __forceinline__ long long table_row(const DecodeParams& p, int seq) {
-    if (!p.table_rows) return seq;
-    const int r = p.table_rows[seq];
+// Row of the block-table array that holds launch slot `slot`'s table; -1 if
+// the row index is out of range.
+__device__ __forceinline__ long long table_row(const DecodeParams& p, int slot) {
+    if (!p.table_rows) return slot;
+    const int r = p.table_rows[slot];
     return (r >= 0 && r < p.n_table_rows) ? r : -1;
+}
+
+// The caller's sequence index of launch slot `slot`.
+__device__ __forceinline__ int seq_of(const DecodeParams& p, int slot) {
+    return p.order ? p.order[slot] : slot;
 }
 
 // Allow the kernel the device's whole opt-in shared memory per block (minus
