@@ -283,15 +283,19 @@ size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, 
 /* Kernel selection for paged_decode_attention_ex. */
 #define PKV_KERNEL_AUTO 0          /* LEAN for large groups (G > 16) when supported, the workspace
                                       holds its state and partition_tokens is 0; else TENSOR when
-                                      supported; else SIMT */
+                                      supported (not for FP8 pools with G = 1); else SIMT */
 #define PKV_KERNEL_SIMT 1          /* CUDA-core dot products: SIMT_TMA when supported, else SIMT_BULK */
 #define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads: F16/BF16 pools with
-                                      head_dim 64 or 128, power-of-two block size, 1 < G <= 128 */
+                                      q in the pool dtype, head_dim 64 or 128, power-of-two block
+                                      size, 1 < G <= 128; FP8-E4M3 pools with F16 q, head_dim 128,
+                                      power-of-two block size, 1 <= G <= 8 (codes converted to f16
+                                      in registers) */
 #define PKV_KERNEL_SIMT_BULK 3     /* CUDA-core, 1-D bulk copies per block run (any shape) */
 #define PKV_KERNEL_SIMT_TMA 4      /* CUDA-core, swizzled 2-D TMA boxes, one query head per CTA:
                                       rows of 128/256/512 bytes, power-of-two block size */
 #define PKV_KERNEL_LEAN 5          /* tensor cores, one wave of persistent workers sharing the batch's
-                                      16-token stages equally, split pairs merged by a second launch:
+                                      16-token stages equally, a split pair merged in the kernel by
+                                      the worker that finishes its last piece:
                                       F16/BF16 pools with head_dim 64 or 128, power-of-two block
                                       size, 1 <= G <= 128, B <= 2048; ignores partition_tokens */
 

@@ -342,11 +342,14 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     int use = kernel;
     // automatic: large groups (one KV head shared by many query heads, a
     // small latency-bound batch) take the stage-balanced kernel; up to 16
-    // heads per KV head the partitioned tensor-core kernel measured faster
+    // heads per KV head the partitioned tensor-core kernel measured faster.
+    // An FP8 pool with one query head per KV head stays on the CUDA cores
+    // (measured faster than converting its codes for the tensor cores).
+    const bool tc_auto = tc_ok && !(p->dtype == PKV_FP8_E4M3 && G == 1);
     if (use == PKV_KERNEL_AUTO)
         use = (lean_fits && G > 16 && partition_tokens == 0)
                   ? PKV_KERNEL_LEAN
-                  : (tc_ok ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT);
+                  : (tc_auto ? PKV_KERNEL_TENSOR : PKV_KERNEL_SIMT);
     if (use == PKV_KERNEL_SIMT) use = s2_ok ? PKV_KERNEL_SIMT_TMA : PKV_KERNEL_SIMT_BULK;
     if (use == PKV_KERNEL_TENSOR && !tc_ok) return PKV_ERR_INVALID_ARG;
     if (use == PKV_KERNEL_SIMT_TMA && !s2_ok) return PKV_ERR_INVALID_ARG;

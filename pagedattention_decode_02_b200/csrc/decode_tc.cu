@@ -28,6 +28,7 @@
 #include <cuda.h>
 
 #include <cfloat>
+#include <type_traits>
 
 #include "decode_launch.h"
 #include "kernels_common.cuh"
@@ -42,30 +43,35 @@ using tc::kStageTokens;
 using tc::mbar_arrive;
 using tc::tma_load_2d;
 
-template <int D>
+// EB: bytes per stored K/V element (2: f16/bf16 pools, 1: FP8 pools)
+template <int D, int EB>
 struct TcSmem {
-    static constexpr int kTile = kStageTokens * D * 2;   // bytes of K (or V) of one stage
+    static constexpr int kTile = kStageTokens * D * EB;   // bytes of K (or V) of one stage
     static constexpr int kSlot = 2 * kTile;
 };
 
-template <int D, int MT, int TS, int S>
+template <int D, int MT, int TS, int S, int EB>
 __host__ __device__ constexpr int tc_union_bytes() {
-    const int tiles = TS * S * TcSmem<D>::kSlot;
+    const int tiles = TS * S * TcSmem<D, EB>::kSlot;
     const int comb = MT * TS * 8 * (D + 2) * 4;
     return ((tiles > comb ? tiles : comb) + 15) & ~15;
 }
 
-template <typename T, int D, int MT, int TS, int S>
+template <typename T, int D, int MT, int TS, int S, int EB>
 __global__ void __launch_bounds__(MT * TS * 32)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
     constexpr int kStages = S;
     constexpr int NW = MT * TS;
     constexpr int NT = NW * 32;
-    constexpr int TILE = TcSmem<D>::kTile;
-    constexpr int SLOT = TcSmem<D>::kSlot;
+    constexpr int TILE = TcSmem<D, EB>::kTile;
+    constexpr int SLOT = TcSmem<D, EB>::kSlot;
     constexpr int KSTEPS = D / 16;       // k-steps of S = Q K^T
-    constexpr int HALVES = D / 64;
+    constexpr int HALVES = D * EB / 128;   // 128-byte column boxes per row
+    static_assert(EB == 2 || (EB == 1 && D == 128), "FP8 stages have 128-byte rows");
+    // early slot release holds a whole stage's fragments in registers: with
+    // up to 8 warps (255 registers a thread) and for FP8 (raw codes, 32 registers)
+    constexpr bool kEarly = EB == 1 || NT <= 256;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment of the swizzled tiles; the combine area reuses the
@@ -74,7 +80,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                ~uintptr_t(1023));
     uint8_t* tiles = smem;                                            // [TS][kStages][SLOT]
     float* comb = reinterpret_cast<float*>(smem);                     // [NW][8][D + 2]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS, S>());
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_union_bytes<D, MT, TS, S, EB>());
     uint64_t* empty = full + TS * kStages;
     int32_t* blk = reinterpret_cast<int32_t*>(empty + TS * kStages);   // the partition's block ids
 
@@ -141,7 +147,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (split && p.counters &&
             finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
             merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
-                                     tc_union_bytes<D, MT, TS, S>() / 4);
+                                     tc_union_bytes<D, MT, TS, S, EB>() / 4);
         return;
     }
 
@@ -171,8 +177,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                 for (int hf = 0; hf < HALVES; ++hf) {
                     const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
-                    tma_load_2d(kd + off, &tmap_k, hf * 64, y, &my_full[slot], policy);
-                    tma_load_2d(vd + off, &tmap_v, hf * 64, y, &my_full[slot], policy);
+                    tma_load_2d(kd + off, &tmap_k, hf * (128 / EB), y, &my_full[slot], policy);
+                    tma_load_2d(vd + off, &tmap_v, hf * (128 / EB), y, &my_full[slot], policy);
                 }
             }
         }
@@ -183,8 +189,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int gq = lane >> 2;       // fragment row: d (and d + 8) of O^T
     const int tq = lane & 3;        // this lane's heads: 2 tq, 2 tq + 1 of the warp's 8
     uint32_t qb[KSTEPS][2];
-    tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
-                            mt * 8, G, lane);
+    if constexpr (EB == 1)
+        tc::load_qT_frags_fp8(qb, reinterpret_cast<const __half*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
+                              mt * 8, G, lane);
+    else
+        tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
+                                mt * 8, G, lane);
 
     float o[D / 16][4];
 #pragma unroll
@@ -207,22 +217,49 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         const int a = t_begin + (ts + k * TS) * kStageTokens;
         const int n = min(kStageTokens, t_end - a);
-        uint8_t* kt = ring + slot * SLOT;
-        uint8_t* vt = kt + TILE;
-        tc::stage_body_t<T, D>(qb, kt, vt, n, p.q_scale, o, m_run, l_run, lane);
-        __syncwarp();
-        if constexpr (MT > 1) {
-            if (lane == 0) mbar_arrive(&my_empty[slot]);
-        }
-        if (producer && k + kStages < my_n) {
+        const uint8_t* kt = ring + slot * SLOT;
+        const uint8_t* vt = kt + TILE;
+        // hand the slot back for the next copy: the producer waits (MT > 1)
+        // until every warp of the group has read it
+        auto release = [&]() -> bool {
+            fence_proxy_async_smem();   // these reads before the async proxy's refill
+            __syncwarp();
             if constexpr (MT > 1) {
-                if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1))) {
-                    timed_out = true;
-                    ++k;
-                    break;
-                }
+                if (lane == 0) mbar_arrive(&my_empty[slot]);
             }
-            issue(k + kStages, slot);
+            if (producer && k + kStages < my_n) {
+                if constexpr (MT > 1) {
+                    if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1))) return false;
+                }
+                issue(k + kStages, slot);
+            }
+            return true;
+        };
+        if constexpr (kEarly) {
+            // the stage moves into registers, the slot is released, and the
+            // math runs while the next copy is in flight
+            using Frags = std::conditional_t<EB == 1, tc::Fp8Raw, tc::StageFrags<D>>;
+            Frags f;
+            if constexpr (EB == 1)
+                tc::stage_raw_fp8(kt, vt, n, f, lane);
+            else
+                tc::stage_frags_t<D>(kt, vt, n, f, lane);
+            if (!release()) {
+                timed_out = true;
+                ++k;
+                break;
+            }
+            if constexpr (EB == 1)
+                tc::stage_math_fp8(qb, f, n, p.q_scale, o, m_run, l_run, lane);
+            else
+                tc::stage_math_t<T, D>(qb, f, n, p.q_scale, o, m_run, l_run, lane);
+        } else {
+            tc::stage_body_t<T, D>(qb, kt, vt, n, p.q_scale, o, m_run, l_run, lane);
+            if (!release()) {
+                timed_out = true;
+                ++k;
+                break;
+            }
         }
     }
     if (timed_out) {
@@ -233,6 +270,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 (void)mbar_wait(&my_full[j % kStages], (uint32_t)((j / kStages) & 1));
     }
 
+    if constexpr (EB == 1) {
+        // FP8 V was used as codes: its scale applies to the accumulator
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j) {
+            o[j][0] *= p.v_scale;
+            o[j][1] *= p.v_scale;
+            o[j][2] *= p.v_scale;
+            o[j][3] *= p.v_scale;
+        }
+    }
     // head sums: the lanes with the same lane % 4 hold disjoint tokens
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -245,13 +292,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     {
         float* cw = comb + warp * 8 * (D + 2);
         const int ra = 2 * tq, rb = ra + 1;
+        // o[j] rows: d = 16 j + gq and + 8 (FP8: d = 16 gq + 2 j and + 1)
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
-            const int d = 16 * j + gq;
-            cw[ra * (D + 2) + d] = o[j][0];
-            cw[rb * (D + 2) + d] = o[j][1];
-            cw[ra * (D + 2) + d + 8] = o[j][2];
-            cw[rb * (D + 2) + d + 8] = o[j][3];
+            const int d0 = EB == 1 ? 16 * gq + 2 * j : 16 * j + gq;
+            const int d1 = EB == 1 ? d0 + 1 : d0 + 8;
+            cw[ra * (D + 2) + d0] = o[j][0];
+            cw[rb * (D + 2) + d0] = o[j][1];
+            cw[ra * (D + 2) + d1] = o[j][2];
+            cw[rb * (D + 2) + d1] = o[j][3];
         }
         if (gq == 0) {
             cw[ra * (D + 2) + D] = m_run[0];
@@ -296,26 +345,26 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (split && p.counters &&
         finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
         merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
-                                 tc_union_bytes<D, MT, TS, S>() / 4);
+                                 tc_union_bytes<D, MT, TS, S, EB>() / 4);
 }
 
-template <int D, int MT, int TS, int S>
+template <int D, int MT, int TS, int S, int EB>
 constexpr int tc_smem_bytes() {
-    return 1024 + tc_union_bytes<D, MT, TS, S>() + 2 * TS * S * 8;
+    return 1024 + tc_union_bytes<D, MT, TS, S, EB>() + 2 * TS * S * 8;
 }
 // plus the partition's block ids: part_tokens / bs + 2 entries
 inline int tc_table_bytes(const DecodeParams& p) {
     return ((p.part_tokens / p.block_size + 2) * 4 + 15) & ~15;
 }
 
-template <typename T, int D, int MT, int TS, int S = (D == 128 ? 2 : 3)>
+template <typename T, int D, int MT, int TS, int S = (D == 128 ? 2 : 3), int EB = 2>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                         int q_dtype, cudaStream_t st, cudaEvent_t mid) {
-    constexpr int base = tc_smem_bytes<D, MT, TS, S>();
+    constexpr int base = tc_smem_bytes<D, MT, TS, S, EB>();
     static_assert(base <= 227 * 1024 - 64, "shared memory budget");
     const int smem = base + tc_table_bytes(p);
     if (smem > 227 * 1024 - 64) return cudaErrorInvalidValue;
-    auto kern = decode_tc_kernel<T, D, MT, TS, S>;
+    auto kern = decode_tc_kernel<T, D, MT, TS, S, EB>;
     static unsigned long long attr_done = 0;
     cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
@@ -414,15 +463,24 @@ void pool_init_device_extras(pkv_pool* p) {
 bool pool_has_row_maps(const pkv_pool* pool) { return pool->has_tmaps; }
 
 bool tensor_path_supported(const pkv_pool* pool, int q_dtype, int group) {
-    return pool->has_tmaps && (pool->dtype == PKV_F16 || pool->dtype == PKV_BF16) &&
-           q_dtype == pool->dtype && (pool->head_dim == 64 || pool->head_dim == 128) &&
-           group > 1 && group <= 128;
+    if (!pool->has_tmaps) return false;
+    // FP8 codes are converted to f16 in registers: f16 queries, 128-byte rows,
+    // one warp of up to 8 heads per KV head
+    if (pool->dtype == PKV_FP8_E4M3)
+        return q_dtype == PKV_F16 && pool->head_dim == 128 && group >= 1 && group <= 8;
+    return (pool->dtype == PKV_F16 || pool->dtype == PKV_BF16) && q_dtype == pool->dtype &&
+           (pool->head_dim == 64 || pool->head_dim == 128) && group > 1 && group <= 128;
 }
 
 cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, const void* tmap_v,
                                  int kv_dtype, int D, cudaStream_t st, cudaEvent_t mid) {
     const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(tmap_k);
     const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(tmap_v);
+    if (kv_dtype == PKV_FP8_E4M3) {
+        // 4 KB stages: 4-slot rings per token group
+        if (D == 128 && p.G <= 8) return launch_tc_t<__half, 128, 1, 4, 4, 1>(p, tk, tv, PKV_F16, st, mid);
+        return cudaErrorInvalidValue;
+    }
     if (kv_dtype == PKV_F16) {
         if (D == 64) return launch_tc_d<__half, 64>(p, tk, tv, PKV_F16, st, mid);
         if (D == 128) return launch_tc_d<__half, 128>(p, tk, tv, PKV_F16, st, mid);

@@ -1,8 +1,9 @@
 // Tensor-core building blocks of the grouped-head decode kernels (sm_100a):
 // mma.sync m16n8k16 wrappers for f16/bf16 inputs with fp32 accumulation,
 // ldmatrix loads, the 2-D tiled TMA load and the 128-byte swizzle of a staged
-// 16-token tile, and the per-stage body (scores, online softmax, P.V) that the
-// partitioned and the stage-balanced kernels share.
+// 16-token tile, and the per-stage math (scores, online softmax, P.V) that the
+// partitioned and the stage-balanced kernels share, for f16/bf16 pools and,
+// converted in registers, FP8-E4M3 pools.
 #pragma once
 
 #include <cuda.h>
@@ -79,140 +80,6 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 
-// Q fragments (mma A operand) of one warp's 16 query-head rows: rows
-// r0 = row_base + lane / 4 and r0 + 8 of the [rows][D] block at q, zero for
-// rows >= n_rows.
-template <typename T, int D>
-__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[D / 16][4], const T* q, int row_base,
-                                             int n_rows, int lane) {
-    const int r0 = row_base + (lane >> 2), r1 = r0 + 8;
-    const int tq = lane & 3;
-    const T* q0 = q + (size_t)r0 * D;
-    const T* q1 = q + (size_t)r1 * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const int c0 = kk * 16 + 2 * tq;
-        qa[kk][0] = r0 < n_rows ? *reinterpret_cast<const uint32_t*>(q0 + c0) : 0u;
-        qa[kk][1] = r1 < n_rows ? *reinterpret_cast<const uint32_t*>(q1 + c0) : 0u;
-        qa[kk][2] = r0 < n_rows ? *reinterpret_cast<const uint32_t*>(q0 + c0 + 8) : 0u;
-        qa[kk][3] = r1 < n_rows ? *reinterpret_cast<const uint32_t*>(q1 + c0 + 8) : 0u;
-    }
-}
-
-// One 16-token stage for one warp's 16 head rows:
-//     S = Q K_stage^T (q_scale folds the softmax scale and log2 e), online
-//     softmax per row in base 2, O = alpha O + P V_stage.
-// kt / vt: the stage's swizzled K and V tiles; n (1..16) tokens are valid.
-// V rows past n hold stale bytes and are zeroed first (every warp zeroes its
-// own view; the values are identical, so overlapping writes are harmless),
-// then a proxy fence, since the async proxy refills the slot later.  Scores
-// of tokens past n are -inf, so P is exactly 0 there.
-template <typename T, int D>
-__device__ __forceinline__ void stage_body(const uint32_t (&qa)[D / 16][4], uint8_t* kt,
-                                           uint8_t* vt, int n, float q_scale,
-                                           float (&o)[D / 8][4], float (&m_run)[2],
-                                           float (&l_run)[2], int lane) {
-    constexpr int KSTEPS = D / 16;
-    constexpr int DTILES = D / 8;
-    const int tq = lane & 3;
-    if (n < kStageTokens) {
-        for (int i = lane; i < (kStageTokens - n) * (D / 8); i += 32) {
-            const int r = n + i / (D / 8), cc = i % (D / 8);
-            *reinterpret_cast<uint4*>(vt + swz(r, cc)) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-    }
-    const uint32_t kbase = smem_addr(kt);
-    const uint32_t vbase = smem_addr(vt);
-
-    // S = Q K^T : two n-tiles of 8 tokens; even and odd k-steps go to
-    // separate accumulators to halve the dependent mma chain
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
-        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        const int mi = lane >> 3, r = lane & 7;
-        const int tok = (mi >> 1) * 8 + r;
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kbase + swz(tok, 2 * kk + (mi & 1)), b0, b1, b2, b3);
-            if (kk & 1) {
-                MmaType<T>::mma(s2[0], qa[kk], b0, b1);
-                MmaType<T>::mma(s2[1], qa[kk], b2, b3);
-            } else {
-                MmaType<T>::mma(s[0], qa[kk], b0, b1);
-                MmaType<T>::mma(s[1], qa[kk], b2, b3);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
-    }
-    // online softmax over this stage's tokens, per head row (lane / 4, + 8)
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int tok = 8 * j + 2 * tq + (e & 1);
-            float v = s[j][e] * q_scale;
-            v = tok < n ? v : -INFINITY;
-            s[j][e] = v;
-            mx[e >> 1] = fmaxf(mx[e >> 1], v);
-        }
-    float alpha[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-        const float m_new = fmaxf(m_run[r], mx[r]);
-        alpha[r] = exp2f(m_run[r] - m_new);
-        m_run[r] = m_new;
-        l_run[r] *= alpha[r];
-    }
-    uint32_t pa[4];
-    {
-        float pr[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                pr[j][e] = exp2f(s[j][e] - m_run[e >> 1]);
-                l_run[e >> 1] += pr[j][e];
-            }
-        pa[0] = MmaType<T>::pack(pr[0][0], pr[0][1]);
-        pa[1] = MmaType<T>::pack(pr[0][2], pr[0][3]);
-        pa[2] = MmaType<T>::pack(pr[1][0], pr[1][1]);
-        pa[3] = MmaType<T>::pack(pr[1][2], pr[1][3]);
-    }
-    // rescale the accumulator only when some row's running max moved
-    // (alpha == 1 exactly otherwise): late in a sequence it rarely does
-    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-        for (int j = 0; j < DTILES; ++j) {
-            o[j][0] *= alpha[0];
-            o[j][1] *= alpha[0];
-            o[j][2] *= alpha[1];
-            o[j][3] *= alpha[1];
-        }
-    }
-    // O += P V : V^T fragments by transposed ldmatrix, two d-tiles per load
-    {
-        const int mi = lane >> 3, r = lane & 7;
-        const int tok = (mi & 1) * 8 + r;
-#pragma unroll
-        for (int j = 0; j < DTILES; j += 2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vbase + swz(tok, j + (mi >> 1)), b0, b1, b2, b3);
-            MmaType<T>::mma(o[j], pa, b0, b1);
-            MmaType<T>::mma(o[j + 1], pa, b2, b3);
-        }
-    }
-}
-
-
 // Transpose of an 8x8 b16 matrix held one 32-bit pair per lane in the mma
 // fragment layout (row lane / 4, columns 2 (lane % 4) and + 1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
@@ -239,51 +106,64 @@ __device__ __forceinline__ void load_qT_frags(uint32_t (&qb)[D / 16][2], const T
     }
 }
 
-// One 16-token stage for one warp's 8 query heads, in transposed form (no
-// padded rows when a KV head has 8 or fewer query heads):
-//     S^T [16 tokens][8 heads] = K_stage Q^T,
-//     online softmax per head (column) in base 2,
-//     O^T [D][8 heads] = alpha O^T + V_stage^T P^T.
-// P^T moves from the accumulator layout to the B-operand layout with two 8x8
-// transposes (movmatrix).  This lane holds heads 2 (lane % 4) and + 1:
-// m_run / l_run (l partial over this lane's tokens, summed over the lanes of
-// the same lane % 4 at the end), o[mt] = O^T rows d = 16 mt + lane / 4 (and
-// + 8) for those two heads.  Same staging and zeroing rules as stage_body.
-template <typename T, int D>
-__device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], uint8_t* kt,
-                                             uint8_t* vt, int n, float q_scale,
-                                             float (&o)[D / 16][4], float (&m_run)[2],
-                                             float (&l_run)[2], int lane) {
-    constexpr int KSTEPS = D / 16;
-    const int gq = lane >> 2;
-    if (n < kStageTokens) {
-        for (int i = lane; i < (kStageTokens - n) * (D / 8); i += 32) {
-            const int r = n + i / (D / 8), cc = i % (D / 8);
-            *reinterpret_cast<uint4*>(vt + swz(r, cc)) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-    }
+// The A fragments of one staged 16-token tile, read out of shared memory so
+// that the ring slot can be refilled while the math uses them.
+//   k[kk]: K rows (tokens) x d columns 16 kk .. 16 kk + 15 (S^T = K Q^T);
+//   v[mt]: V^T rows d = 16 mt .. 16 mt + 15 x tokens (O^T += V^T P^T).
+template <int D>
+struct StageFrags {
+    uint32_t k[D / 16][4];
+    uint32_t v[D / 16][4];
+};
+
+// Fill f from the swizzled K and V tiles of a stage with n valid tokens.  V of
+// the tokens past n may hold anything (stale or never-written rows): its
+// values are replaced by 0, so that 0-weight tokens add 0 (not NaN).
+template <int D>
+__device__ __forceinline__ void stage_frags_t(const uint8_t* kt, const uint8_t* vt, int n,
+                                              StageFrags<D>& f, int lane) {
     const uint32_t kbase = smem_addr(kt);
     const uint32_t vbase = smem_addr(vt);
     const int mi = lane >> 3, r8 = lane & 7;
-
-    // S^T = K Q^T over the d k-steps, four interleaved accumulators
-    float acc[4][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+    for (int kk = 0; kk < D / 16; ++kk)
+        ldsm_x4(kbase + swz((mi & 1) * 8 + r8, 2 * kk + (mi >> 1)), f.k[kk][0], f.k[kk][1],
+                f.k[kk][2], f.k[kk][3]);
 #pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-        uint32_t a[4];
-        ldsm_x4(kbase + swz((mi & 1) * 8 + r8, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
-        MmaType<T>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
+    for (int mt = 0; mt < D / 16; ++mt)
+        ldsm_x4_t(vbase + swz((mi >> 1) * 8 + r8, 2 * mt + (mi & 1)), f.v[mt][0], f.v[mt][1],
+                  f.v[mt][2], f.v[mt][3]);
+    if (n < kStageTokens) {
+        // registers 0/1 hold tokens 2 tq (low half) and 2 tq + 1 (high half),
+        // registers 2/3 tokens 2 tq + 8 and 2 tq + 9
+        const int t0 = 2 * (lane & 3);
+        const uint32_t m01 = (t0 < n ? 0x0000ffffu : 0u) | (t0 + 1 < n ? 0xffff0000u : 0u);
+        const uint32_t m23 = (t0 + 8 < n ? 0x0000ffffu : 0u) | (t0 + 9 < n ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            f.v[mt][0] &= m01;
+            f.v[mt][1] &= m01;
+            f.v[mt][2] &= m23;
+            f.v[mt][3] &= m23;
+        }
     }
-    float s[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
-    // tokens gq (s[0], s[1]) and gq + 8 (s[2], s[3]); heads 2 tq (even e), 2 tq + 1
+}
+
+// Scores of one stage: S^T fragment (tokens gq, gq + 8; heads 2 tq, 2 tq + 1)
+// scaled to base 2, tokens past n at -inf.
+__device__ __forceinline__ void mask_scores(float (&s)[4], int n, int lane) {
+    const int gq = lane >> 2;
     if (gq >= n) s[0] = s[1] = -INFINITY;
     if (gq + 8 >= n) s[2] = s[3] = -INFINITY;
+}
+
+// Online-softmax update of one stage for this lane's two heads; returns P^T
+// as the B operand of the P.V product (pb0 = tokens 0-7, pb1 = tokens 8-15)
+// and rescales o when a running maximum moved.
+template <typename T, int MTILES>
+__device__ __forceinline__ void softmax_step(const float (&s)[4], float (&o)[MTILES][4],
+                                             float (&m_run)[2], float (&l_run)[2], uint32_t& pb0,
+                                             uint32_t& pb1) {
     float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -304,24 +184,210 @@ __device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], ui
     const float p3 = exp2f(s[3] - m_run[1]);
     l_run[0] = l_run[0] * alpha[0] + (p0 + p2);
     l_run[1] = l_run[1] * alpha[1] + (p1 + p3);
-    // P^T as the B operand: b0 = tokens 0-7, b1 = tokens 8-15
-    const uint32_t pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
-    const uint32_t pb1 = movmatrix_trans(MmaType<T>::pack(p2, p3));
+    pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
+    pb1 = movmatrix_trans(MmaType<T>::pack(p2, p3));
     if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
+        for (int mt = 0; mt < MTILES; ++mt) {
             o[mt][0] *= alpha[0];
             o[mt][1] *= alpha[1];
             o[mt][2] *= alpha[0];
             o[mt][3] *= alpha[1];
         }
     }
-    // O^T += V^T P^T: one m-tile of 16 d rows per transposed ldmatrix
+}
+
+// One 16-token stage for one warp's 8 query heads, in transposed form (no
+// padded rows when a KV head has 8 or fewer query heads):
+//     S^T [16 tokens][8 heads] = K_stage Q^T,
+//     online softmax per head (column) in base 2,
+//     O^T [D][8 heads] = alpha O^T + V_stage^T P^T.
+// P^T moves from the accumulator layout to the B-operand layout with two 8x8
+// transposes (movmatrix).  This lane holds heads 2 (lane % 4) and + 1:
+// m_run / l_run (l partial over this lane's tokens, summed over the lanes of
+// the same lane % 4 at the end), o[mt] = O^T rows d = 16 mt + lane / 4 (and
+// + 8) for those two heads.
+template <typename T, int D>
+__device__ __forceinline__ void stage_math_t(const uint32_t (&qb)[D / 16][2],
+                                             const StageFrags<D>& f, int n, float q_scale,
+                                             float (&o)[D / 16][4], float (&m_run)[2],
+                                             float (&l_run)[2], int lane) {
+    float acc[4][4];
 #pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) MmaType<T>::mma(acc[kk & 3], f.k[kk], qb[kk][0], qb[kk][1]);
+    float s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
+    mask_scores(s, n, lane);
+    uint32_t pb0, pb1;
+    softmax_step<T, D / 16>(s, o, m_run, l_run, pb0, pb1);
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) MmaType<T>::mma(o[mt], f.v[mt], pb0, pb1);
+}
+
+// stage_frags_t + stage_math_t with each fragment loaded next to its use
+// (fewer live registers; the slot is released after the whole stage).
+template <typename T, int D>
+__device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], const uint8_t* kt,
+                                             const uint8_t* vt, int n, float q_scale,
+                                             float (&o)[D / 16][4], float (&m_run)[2],
+                                             float (&l_run)[2], int lane) {
+    const uint32_t kbase = smem_addr(kt);
+    const uint32_t vbase = smem_addr(vt);
+    const int mi = lane >> 3, r8 = lane & 7;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t a[4];
-        ldsm_x4_t(vbase + swz((mi >> 1) * 8 + r8, 2 * mt + (mi & 1)), a[0], a[1], a[2], a[3]);
-        MmaType<T>::mma(o[mt], a, pb0, pb1);
+        ldsm_x4(kbase + swz((mi & 1) * 8 + r8, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
+        MmaType<T>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
+    }
+    float s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
+    mask_scores(s, n, lane);
+    uint32_t pb0, pb1;
+    softmax_step<T, D / 16>(s, o, m_run, l_run, pb0, pb1);
+    if (n == kStageTokens) {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_t(vbase + swz((mi >> 1) * 8 + r8, 2 * mt + (mi & 1)), a[0], a[1], a[2], a[3]);
+            MmaType<T>::mma(o[mt], a, pb0, pb1);
+        }
+    } else {
+        // V of the tokens past n replaced by 0 (see stage_frags_t)
+        const int t0 = 2 * (lane & 3);
+        const uint32_t m01 = (t0 < n ? 0x0000ffffu : 0u) | (t0 + 1 < n ? 0xffff0000u : 0u);
+        const uint32_t m23 = (t0 + 8 < n ? 0x0000ffffu : 0u) | (t0 + 9 < n ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_t(vbase + swz((mi >> 1) * 8 + r8, 2 * mt + (mi & 1)), a[0], a[1], a[2], a[3]);
+            a[0] &= m01;
+            a[1] &= m01;
+            a[2] &= m23;
+            a[3] &= m23;
+            MmaType<T>::mma(o[mt], a, pb0, pb1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FP8-E4M3 pools (d = 128, f16 queries): the stage's K and V tiles hold codes
+// in 128-byte rows.  Each lane reads its codes with four 16-byte loads per
+// tile, contiguous and free of bank conflicts, and converts them to f16 in
+// registers.  To make that possible the d index is permuted, which leaves
+// both products unchanged (a sum over d in any order; O^T rows in any order):
+//   S^T k-step kk, fragment columns 2 tq + {0, 1} / 2 tq + {8, 9}
+//       <-> d = 32 tq + 4 kk + {0, 1} / + {2, 3};
+//   O^T m-tile mt, fragment row gq / gq + 8  <->  d = 16 gq + 2 mt / + 1.
+// ---------------------------------------------------------------------------
+
+// Two FP8-E4M3 codes (low byte first) -> f16x2, exact (every e4m3 value is an
+// f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Byte offset of the 16-byte chunk c (0..7) of row r in a 16-row tile of
+// 128-byte rows staged with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz_chunk(int r, int c) {
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// This lane's codes of one stage:
+//   k[i][j]: K row gq + 8 i, bytes 32 tq + 16 j .. + 15;
+//   v[i]:    V row 2 tq + (i & 1) + 8 (i >> 1), bytes 16 gq .. 16 gq + 15
+//            (zero for rows at or past n).
+struct Fp8Raw {
+    uint4 k[2][2];
+    uint4 v[4];
+};
+
+__device__ __forceinline__ void stage_raw_fp8(const uint8_t* kt, const uint8_t* vt, int n,
+                                              Fp8Raw& r, int lane) {
+    const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            r.k[i][j] = *reinterpret_cast<const uint4*>(kt + swz_chunk(gq + 8 * i, 2 * tq + j));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int row = 2 * tq + (i & 1) + 8 * (i >> 1);
+        r.v[i] = row < n ? *reinterpret_cast<const uint4*>(vt + swz_chunk(row, gq))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// Q^T fragments for the permuted contraction: k-step kk, b0 = q[head][32 tq
+// + 4 kk + {0, 1}], b1 = q[head][32 tq + 4 kk + {2, 3}], head = head_base +
+// lane / 4, zero for heads >= n_heads.
+__device__ __forceinline__ void load_qT_frags_fp8(uint32_t (&qb)[8][2], const __half* q,
+                                                  int head_base, int n_heads, int lane) {
+    const int h = head_base + (lane >> 2);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(q + (size_t)h * 128 + 32 * (lane & 3));
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        qb[kk][0] = h < n_heads ? src[2 * kk] : 0u;
+        qb[kk][1] = h < n_heads ? src[2 * kk + 1] : 0u;
+    }
+}
+
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t y, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(y), "r"(sel));
+    return d;
+}
+
+// The stage math of stage_math_t on an FP8 stage (scales folded by the
+// caller: q_scale includes k_scale, the output is multiplied by v_scale).
+// o[mt] = O^T rows d = 16 gq + 2 mt (o[mt][0..1]) and + 1 (o[mt][2..3]).
+__device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const Fp8Raw& r, int n,
+                                               float q_scale, float (&o)[8][4],
+                                               float (&m_run)[2], float (&l_run)[2], int lane) {
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+    const uint32_t* k0 = reinterpret_cast<const uint32_t*>(&r.k[0][0]);   // row gq, 8 words
+    const uint32_t* k1 = reinterpret_cast<const uint32_t*>(&r.k[1][0]);   // row gq + 8
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        // word kk: d = 32 tq + 4 kk .. + 3
+        const uint32_t a[4] = {e4m3x2_to_f16x2(k0[kk]), e4m3x2_to_f16x2(k1[kk]),
+                               e4m3x2_to_f16x2(k0[kk] >> 16), e4m3x2_to_f16x2(k1[kk] >> 16)};
+        MmaType<__half>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
+    }
+    float s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
+    mask_scores(s, n, lane);
+    uint32_t pb0, pb1;
+    softmax_step<__half, 8>(s, o, m_run, l_run, pb0, pb1);
+    // V^T fragments: a token pair's codes of one d interleaved byte by byte
+    const uint32_t* x0 = reinterpret_cast<const uint32_t*>(&r.v[0]);   // token 2 tq
+    const uint32_t* y0 = reinterpret_cast<const uint32_t*>(&r.v[1]);   // token 2 tq + 1
+    const uint32_t* x1 = reinterpret_cast<const uint32_t*>(&r.v[2]);   // token 2 tq + 8
+    const uint32_t* y1 = reinterpret_cast<const uint32_t*>(&r.v[3]);   // token 2 tq + 9
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // word j: d = 16 gq + 4 j .. + 3 -> m-tiles 2 j (d + 0, + 1) and 2 j + 1 (d + 2, + 3)
+        const uint32_t lo01 = byte_perm(x0[j], y0[j], 0x5140u);
+        const uint32_t hi01 = byte_perm(x0[j], y0[j], 0x7362u);
+        const uint32_t lo23 = byte_perm(x1[j], y1[j], 0x5140u);
+        const uint32_t hi23 = byte_perm(x1[j], y1[j], 0x7362u);
+        const uint32_t a0[4] = {e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo01 >> 16),
+                                e4m3x2_to_f16x2(lo23), e4m3x2_to_f16x2(lo23 >> 16)};
+        MmaType<__half>::mma(o[2 * j], a0, pb0, pb1);
+        const uint32_t a1[4] = {e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi01 >> 16),
+                                e4m3x2_to_f16x2(hi23), e4m3x2_to_f16x2(hi23 >> 16)};
+        MmaType<__half>::mma(o[2 * j + 1], a1, pb0, pb1);
     }
 }
 

@@ -102,6 +102,34 @@ def test_fp8_small(bs, qdt, kernel):
     check_pool_bytes(side)
 
 
+@pytest.mark.parametrize("bs", [1, 2, 4, 8, 16, 64])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (16, 2), (8, 1), (5, 1)])
+@pytest.mark.parametrize("part", [0, 32])
+def test_fp8_tensor_small(bs, hq, hkv, part):
+    # FP8 codes converted to f16 in registers feed the tensor-core stage math
+    cfg = small("fp8", n_q_heads=hq, n_kv_heads=hkv, block_size=bs, batch=5,
+                lengths=("uniform", 1, 300))
+    side = setup_config(cfg, seed=bs * 3 + hq)
+    gpu, ref, _ = decode_step(side, list(range(cfg.batch)), 0, partition_tokens=part,
+                              kernel=pk.PKV_KERNEL_TENSOR)
+    compare_out(gpu, ref, "fp8")
+
+
+def test_fp8_tensor_refusals():
+    # bf16 queries, head_dim 64 and more than 8 heads per KV head stay on the CUDA cores
+    tables = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
+    lens = torch.ones(1, dtype=torch.int32, device="cuda")
+    for d, hq, qdt in ((128, 4, torch.bfloat16), (64, 4, torch.float16), (128, 16, torch.float16)):
+        pool = pk.kv_pool_create(8, 16, 1, d, "fp8")
+        for buf in pool.device_buffers():
+            buf.zero_()
+        q = torch.zeros(1, hq, d, device="cuda", dtype=qdt)
+        with pytest.raises(pk.PagedKVError):
+            pk.paged_decode_attention(pool, q, tables, lens, 0.1, kernel=pk.PKV_KERNEL_TENSOR)
+        out = pk.paged_decode_attention(pool, q, tables, lens, 0.1)   # the automatic choice runs
+        assert torch.all(torch.isfinite(out.float()))
+
+
 # ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------
@@ -255,6 +283,18 @@ def test_falcon7b_sharing_all_steps(variant):
     # prompt blocks stay shared by all four samples
     t0 = side.orc.bm.tables[0]
     assert pk.bt_refcount(side.pool, t0[0]) == 4
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("kernel", [pk.PKV_KERNEL_AUTO, pk.PKV_KERNEL_TENSOR, pk.PKV_KERNEL_SIMT])
+def test_fp8_gqa_full(kernel):
+    # the Llama-2-70B-shaped batch on an FP8 pool (f16 q/out), sampled heads
+    cfg = wl.CONFIGS["fp8_gqa"]
+    side = setup_config(cfg)
+    heads = _sampled_heads(cfg, 8)
+    seqs = list(range(cfg.batch))
+    gpu, ref, _ = decode_step(side, seqs, 0, kernel=kernel, check_heads=heads)
+    compare_out(gpu, ref, "fp8", heads)
 
 
 @pytest.mark.slow

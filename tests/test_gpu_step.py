@@ -94,6 +94,32 @@ def test_step_runtime_split_merge_every_kernel(kernel):
     assert launches[-1] == (2 if kernel == pk.PKV_KERNEL_TENSOR else 3)
 
 
+@pytest.mark.parametrize("base,hq,hkv,expect", [
+    ("opt13b", 4, 4, pk.PKV_KERNEL_SIMT_TMA),      # MHA f16
+    ("llama2_70b", 16, 2, pk.PKV_KERNEL_TENSOR),   # GQA bf16, 8 heads per KV head
+    ("falcon7b", 71, 1, pk.PKV_KERNEL_LEAN),       # MQA, 71 heads per KV head
+    ("fp8", 4, 4, pk.PKV_KERNEL_SIMT_TMA),         # FP8 MHA stays on the CUDA cores
+    ("fp8_gqa", 16, 2, pk.PKV_KERNEL_TENSOR),      # FP8 GQA on the tensor cores
+])
+def test_step_runtime_automatic_kernel(base, hq, hkv, expect):
+    import dataclasses
+    cfg = dataclasses.replace(wl.CONFIGS[base], n_q_heads=hq, n_kv_heads=hkv, batch=6,
+                              lengths=("uniform", 1, 700), samples_per_prompt=1,
+                              min_pool_blocks=0)
+    side = setup_config(cfg, growth=5)
+    run_rounds(cfg, side, 3)            # parity of the automatic choice, round by round
+    seqs = np.asarray(side.seqs, dtype=np.int64)
+    max_blocks = max(len(side.orc.bm.tables[s]) for s in side.seqs) + 2
+    step = pk.Step(side.pool, len(seqs), max_blocks, cfg.n_q_heads, cfg.q_dtype)
+    out = torch.empty((len(seqs), hq, cfg.head_dim), device="cuda",
+                      dtype=torch.bfloat16 if cfg.q_dtype == "bf16" else torch.float16)
+    q, kn, vn = step_inputs(side, seqs, 3)
+    pk.pkv_decode_step(step, seqs, to_torch(q, cfg.q_dtype), to_torch(kn, cfg.q_dtype),
+                       to_torch(vn, cfg.q_dtype), cfg.scale, out)
+    torch.cuda.synchronize()
+    assert step.last_kernel == expect
+
+
 def test_step_runtime_rejects_table_overflow_without_changes():
     cfg = wl.CONFIGS["toy"]
     side = setup_config(cfg)

@@ -103,6 +103,11 @@ CONFIGS = {
         "fp8", 40, 40, 128, "fp8", "f16", 16, 128, ("uniform", 1, 2048),
         permute=True,
         description="OPT-13B layer, FP8-E4M3 pool, fp16 q/out, 128 seqs, history U[1,2048]"),
+    "fp8_gqa": Config(
+        "fp8_gqa", 64, 8, 128, "fp8", "f16", 16, 64, ("loguniform", 128, 4096),
+        permute=True,
+        description="Llama-2-70B layer, FP8-E4M3 pool, fp16 q/out: 64/8 GQA x128, bs 16, "
+                    "64 seqs, history log-U[128,4096]"),
 }
 
 FP8_BLOCK_SIZES = (1, 2, 4, 8, 16, 32, 64)
