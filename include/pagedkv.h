@@ -263,7 +263,9 @@ pkv_status block_copy(pkv_pool* pool, const int32_t* d_src, const int32_t* d_dst
  *   d_block_tables: device int32 [B][max_blocks]; d_context_lens: device [B].
  *   n_q_heads must be a multiple of n_kv_heads.
  *   Long contexts are split into partitions whose partial softmax states are
- *   merged by log-sum-exp in a second kernel; that needs d_workspace (device,
+ *   merged by log-sum-exp (unless the unsplit grid already has two waves of
+ *   CTAs at three per SM: B * n_q_heads CTAs for one head per KV head,
+ *   B * n_kv_heads * ceil(G / 8) for grouped heads); that needs d_workspace (device,
  *   ws_bytes >= paged_decode_workspace_bytes(...), 16-byte aligned, caller
  *   owned, contents scratch).  Without enough workspace the call returns
  *   INVALID_ARG.  A context length outside [1, max_blocks * bs] sets
@@ -300,9 +302,12 @@ size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, 
                                       size, 1 <= G <= 128, B <= 2048; ignores partition_tokens */
 
 /* paged_decode_attention_ex - paged_decode_attention with explicit choices:
- *   partition_tokens: 0 = automatic, > 0 = tokens per partition (a multiple
- *   of 16), -1 = never split; kernel: PKV_KERNEL_*.  The workspace needed for
- *   the same choices is paged_decode_workspace_bytes_ex(). */
+ *   partition_tokens: 0 = automatic, > 0 = the longest partition (a multiple
+ *   of 16), -1 = never split; kernel: PKV_KERNEL_*.  A context of c tokens is
+ *   split into ceil(c / P) partitions; the tensor-core and TMA kernels give
+ *   them equal lengths (rounded up to 16 tokens, the last one shorter), the
+ *   bulk-copy kernel cuts at multiples of P.  The workspace needed for the
+ *   same choices is paged_decode_workspace_bytes_ex(). */
 pkv_status paged_decode_attention_ex(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
                                      const int32_t* d_block_tables, int max_blocks,
                                      const int32_t* d_context_lens, int B, int n_q_heads,

@@ -48,16 +48,39 @@ constexpr int kAutoPartition = 512;
 
 // With G query heads per KV head, a partition's partial state is G * (d + 2)
 // floats against partition * 2 * d * elem bytes of K/V, so the automatic
-// partition grows with G; grouped heads take twice the one-head length
-// (measured on the Llama-2-70B-shaped batch: 1024-token partitions beat 512
-// and 2048).
-int resolve_partition(const pkv_pool* pool, int max_blocks, int requested, int group = 1) {
+// partition grows with G; grouped heads take three times the one-head length
+// per 8 heads (measured on the Llama-2-70B-shaped batch with equal-length
+// partitions launched longest first: 1536 tokens 0.78 of the copy peak,
+// against 0.72 for 1024 and 1280 and 0.70 for 2048).
+//
+// units: CTAs of the unsplit grid (0: unknown).  With at least two waves of
+// them (three CTAs per SM) the batch alone fills the GPU and is not split:
+// no partial states, no merge (measured on the OPT-13B-shaped batch, 1,200
+// one-head CTAs: unsplit 0.97 of the copy peak against 0.92-0.93 for 512 to
+// 1024-token partitions).
+int pool_sms(const pkv_pool* pool) {
+    int n = 0;
+    if (pool->device < 0 ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, pool->device) != cudaSuccess ||
+        n <= 0)
+        return 148;
+    return n;
+}
+
+long long unsplit_units(const pkv_pool* pool, int B, int n_q_heads) {
+    const int G = n_q_heads / pool->n_kv_heads;
+    return (long long)B * (G <= 1 ? n_q_heads : (long long)pool->n_kv_heads * ((G + 7) / 8));
+}
+
+int resolve_partition(const pkv_pool* pool, int max_blocks, int requested, int group = 1,
+                      long long units = 0) {
     const long long max_ctx = (long long)max_blocks * pool->block_size;
     const int whole = (int)(((max_ctx + 15) / 16) * 16);
     if (requested < 0) return whole < 16 ? 16 : whole;
     if (requested > 0) return requested;
+    if (units > 0 && units >= 6LL * pool_sms(pool)) return whole < 16 ? 16 : whole;
     const long long auto_p =
-        (long long)kAutoPartition * (group > 1 ? 2 : 1) * ((group + 7) / 8);
+        (long long)kAutoPartition * (group > 1 ? 3 : 1) * ((group + 7) / 8);
     if (max_ctx <= (group > 8 ? auto_p : kNoSplitTokens)) return whole < 16 ? 16 : whole;
     return (int)(auto_p < (1 << 30) ? auto_p : (1 << 30));
 }
@@ -285,7 +308,8 @@ pkv_status block_copy(pkv_pool* p, const int32_t* src, const int32_t* dst, int n
 size_t paged_decode_workspace_bytes_ex(const pkv_pool* p, int B, int n_q_heads, int max_blocks,
                                        int partition_tokens) {
     if (!p || B <= 0 || n_q_heads <= 0 || max_blocks <= 0) return 0;
-    const int P = resolve_partition(p, max_blocks, partition_tokens, n_q_heads / p->n_kv_heads);
+    const int P = resolve_partition(p, max_blocks, partition_tokens, n_q_heads / p->n_kv_heads,
+                                    unsplit_units(p, B, n_q_heads));
     if (P <= 0 || P % 16) return 0;
     const size_t part = workspace_for(p, B, n_q_heads, parts_for(p, max_blocks, P));
     // the automatic choice may take the stage-balanced kernel: room for it too
@@ -355,7 +379,7 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     if (use == PKV_KERNEL_SIMT_TMA && !s2_ok) return PKV_ERR_INVALID_ARG;
     if (use == PKV_KERNEL_LEAN && !lean_fits) return PKV_ERR_INVALID_ARG;
 
-    const int P = resolve_partition(p, max_blocks, partition_tokens, G);
+    const int P = resolve_partition(p, max_blocks, partition_tokens, G, unsplit_units(p, B, n_q_heads));
     const int max_parts = use == PKV_KERNEL_LEAN ? 1 : parts_for(p, max_blocks, P);
     const size_t need = workspace_for(p, B, n_q_heads, max_parts);
     if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return PKV_ERR_INVALID_ARG;
@@ -522,7 +546,7 @@ struct pkv_step {
     std::vector<int32_t> mirror;      // [max_seqs][max_blocks]
     // one round's host scratch
     std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_cow_rows, h_upd_idx, h_upd_val;
-    std::vector<int32_t> h_lens, h_order;   // fast path: lengths, launch order
+    std::vector<int32_t> h_lens, h_order, h_key;   // fast path: lengths, launch order, sort key
     pkv::StepArgs args;
     long long fast_rounds = 0, slow_rounds = 0;
     // profiling: every prof_every-th round records four events (before the
@@ -756,16 +780,23 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         a.n_cow = n_cow;
         a.n_upd = (int32_t)s->h_upd_idx.size();
         a.table_cap = s->max_seqs * s->max_blocks;
-        // launch slots longest context first, so that the long sequences'
-        // partitions start in the first waves and the short ones fill the last
+        // launch slots by partition length, longest first: a sequence's
+        // partitions are equally long, so the grid runs the longest
+        // partitions in the first waves and the short ones fill the last
         s->h_lens.resize(B);
         s->h_order.resize(B);
+        s->h_key.resize(B);
+        // the partition length this round's launch resolves to
+        const int P_round = resolve_partition(pool, s->max_blocks, s->partition_tokens,
+                                              s->n_q_heads / pool->n_kv_heads,
+                                              unsplit_units(pool, B, s->n_q_heads));
         for (int i = 0; i < B; ++i) {
             s->h_lens[i] = (int32_t)pool->bm.find(seq_ids[i])->length;
+            s->h_key[i] = pkv::balanced_part_tokens(s->h_lens[i], P_round);
             s->h_order[i] = i;
         }
         std::stable_sort(s->h_order.begin(), s->h_order.end(),
-                         [&](int32_t x, int32_t y) { return s->h_lens[x] > s->h_lens[y]; });
+                         [&](int32_t x, int32_t y) { return s->h_key[x] > s->h_key[y]; });
         int32_t* d = a.data;
         for (int i = 0; i < B; ++i) d[i] = s->h_slots[i];
         d += B;

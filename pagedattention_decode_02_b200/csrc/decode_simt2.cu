@@ -159,8 +159,9 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
     const int nparts = (c + P - 1) / P;
     if (part >= nparts) return;
-    const int t_begin = part * P;
-    const int t_end = min(c, t_begin + P);
+    const int Ps = balanced_part_tokens(c, P);
+    const int t_begin = part * Ps;
+    const int t_end = min(c, t_begin + Ps);
     const int lb0 = t_begin >> bs_shift;
     const int n_lb = ((t_end - 1) >> bs_shift) - lb0 + 1;
 

@@ -113,8 +113,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
     const int nparts = (c + P - 1) / P;
     if (part >= nparts) return;
-    const int t_begin = part * P;
-    const int t_end = min(c, t_begin + P);
+    const int Ps = balanced_part_tokens(c, P);
+    const int t_begin = part * Ps;
+    const int t_end = min(c, t_begin + Ps);
     const int32_t* table = p.tables + (trow < 0 ? 0 : trow) * p.max_blocks;
 
     const int lb0 = t_begin / bs;

@@ -263,7 +263,7 @@ struct DecodeParams {
     uint32_t* err;
     int B, H_q, H_kv, G;
     int max_blocks, block_size, num_blocks;
-    int part_tokens;  // tokens per partition (multiple of 16)
+    int part_tokens;  // longest partition (multiple of 16): ceil(c / part_tokens) partitions
     int max_parts;    // partitions of the longest possible context
     float q_scale;    // scale * log2(e) * k_scale: folded into q
     float v_scale;    // FP8 V dequantisation (1 otherwise)
@@ -415,6 +415,18 @@ __device__ void merge_in_cta(const DecodeParams& p, int seq, int h, int nparts) 
         reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h) * D + d] =
             Elem<QT>::from_f(L > 0.f ? O / L : 0.f);
     }
+}
+
+// Tokens per partition of a c-token context split into n = ceil(c / P)
+// partitions of equal length, rounded up to a whole 16-token stage (the last
+// partition is shorter by less than 16 n tokens; (n - 1) * result < c since the
+// result is at most P).  All partitions of a sequence then cost the same, so
+// launching sequences in decreasing order of this length schedules the
+// partitions longest first.  Host and device use the same formula.
+__host__ __device__ __forceinline__ int balanced_part_tokens(int c, int P) {
+    const int n = (c + P - 1) / P;
+    const int per = (c + n - 1) / n;
+    return (per + 15) & ~15;
 }
 
 }  // namespace pkv

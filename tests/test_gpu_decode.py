@@ -239,11 +239,13 @@ def _sampled_heads(cfg, k=6):
 
 
 @pytest.mark.slow
-def test_opt13b_full():
+@pytest.mark.parametrize("partition", [0, 512])   # automatic (unsplit: 1,200 CTAs fill the GPU), split
+def test_opt13b_full(partition):
     cfg = wl.CONFIGS["opt13b"]
     side = setup_config(cfg)
     heads = _sampled_heads(cfg)
-    gpu, ref, info = decode_step(side, list(range(cfg.batch)), 0, check_heads=heads)
+    gpu, ref, info = decode_step(side, list(range(cfg.batch)), 0, partition_tokens=partition,
+                                 check_heads=heads)
     compare_out(gpu, ref, "f16", heads)
     check_pool_bytes(side)
     assert side.pool.num_blocks == max(982, wl.pool_blocks(cfg, wl.history_lengths(cfg, 0), 1))
