@@ -83,22 +83,22 @@ def config_of(args) -> wl.Config:
 # sources hash to the recorded value, else the bench reports null.
 TRAFFIC = {
     # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
-    # profiles/decode_tc_llama2_70b.md: 294.7 MB for 286.8 MB algorithmic
+    # profiles/decode_tc_llama2_70b.md: 293.6 MB for 286.5 MB algorithmic
     ("llama2_70b", "decode_tc_kernel"):
-        (1.0274, "45060315d86f88c44c2ed83de5ce87e8375baeb3b4d93a25afc53b518dbe357f"),
-    # profiles/decode_tc_fp8_gqa.md: 149.1 MB for 143.4 MB
+        (1.0246, "842062b2b223be4935749be5c717b576c5963d48e2c3ec1603a7a87ed9b35605"),
+    # profiles/decode_tc_fp8_gqa.md: 149.1 MB for 143.3 MB
     ("fp8_gqa", "decode_tc_kernel"):
-        (1.0396, "45060315d86f88c44c2ed83de5ce87e8375baeb3b4d93a25afc53b518dbe357f"),
-    # profiles/decode_simt2_opt13b.md: 613.0 MB for 604.7 MB
+        (1.0405, "842062b2b223be4935749be5c717b576c5963d48e2c3ec1603a7a87ed9b35605"),
+    # profiles/decode_simt2_opt13b.md: 612.2 MB for 604.1 MB
     ("opt13b", "decode_simt2_kernel"):
-        (1.0137, "72b85098f5d06533b78a6af863d58e10effb0b2385b2a0cd9a9b50e610933516"),
-    # profiles/decode_simt2_fp8.md: 1,361.1 MB for 1,344.8 MB
+        (1.0134, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
+    # profiles/decode_simt2_fp8.md: 1,358.7 MB for 1,343.5 MB
     ("fp8", "decode_simt2_kernel"):
-        (1.0121, "72b85098f5d06533b78a6af863d58e10effb0b2385b2a0cd9a9b50e610933516"),
-    # profiles/decode_lean_falcon7b.md: 2.98 MB for 8.33 MB (the samples of one
+        (1.0113, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
+    # profiles/decode_lean_falcon7b.md: 2.98 MB for 8.31 MB (the samples of one
     # prompt share its blocks; the re-reads within a launch hit L2)
     ("falcon7b", "decode_lean_kernel"):
-        (0.3574, "8149649fd7afa49f9fb5f901d9dd199e6f567eecad77990458cd399ab10c9586"),
+        (0.3581, "602b6701d45a4cad9cbb5d3d18bd1abb961b167f84464ecf7cfb28fd20274f1c"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
