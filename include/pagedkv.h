@@ -285,7 +285,8 @@ size_t paged_decode_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads, 
 /* Kernel selection for paged_decode_attention_ex. */
 #define PKV_KERNEL_AUTO 0          /* LEAN for large groups (G > 16) when supported, the workspace
                                       holds its state and partition_tokens is 0; else TENSOR when
-                                      supported (not for FP8 pools with G = 1); else SIMT */
+                                      supported (not for FP8 pools with G = 1 and block size 1);
+                                      else SIMT */
 #define PKV_KERNEL_SIMT 1          /* CUDA-core dot products: SIMT_TMA when supported, else SIMT_BULK */
 #define PKV_KERNEL_TENSOR 2        /* tensor-core contraction of grouped heads: F16/BF16 pools with
                                       q in the pool dtype, head_dim 64 or 128, power-of-two block

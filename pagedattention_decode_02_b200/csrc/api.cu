@@ -366,10 +366,13 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     int use = kernel;
     // automatic: large groups (one KV head shared by many query heads, a
     // small latency-bound batch) take the stage-balanced kernel; up to 16
-    // heads per KV head the partitioned tensor-core kernel measured faster.
-    // An FP8 pool with one query head per KV head stays on the CUDA cores
-    // (measured faster than converting its codes for the tensor cores).
-    const bool tc_auto = tc_ok && !(p->dtype == PKV_FP8_E4M3 && G == 1);
+    // heads per KV head the partitioned tensor-core kernel measured faster,
+    // and FP8 pools take it from one head per KV head (the CUDA-core kernel
+    // is issue-bound on the conversions), except with one token per block,
+    // where its 16 one-row boxes per stage made it slower (OPT-13B-shaped
+    // FP8 batch: 0.28 of the copy peak against 0.40 on the CUDA cores).
+    const bool tc_auto =
+        tc_ok && !(p->dtype == PKV_FP8_E4M3 && G == 1 && p->block_size == 1);
     if (use == PKV_KERNEL_AUTO)
         use = (lean_fits && G > 16 && partition_tokens == 0)
                   ? PKV_KERNEL_LEAN

@@ -478,8 +478,11 @@ cudaError_t launch_decode_tensor(const DecodeParams& p, const void* tmap_k, cons
     const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(tmap_k);
     const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(tmap_v);
     if (kv_dtype == PKV_FP8_E4M3) {
-        // 4 KB stages: 4-slot rings per token group
-        if (D == 128 && p.G <= 8) return launch_tc_t<__half, 128, 1, 4, 4, 1>(p, tk, tv, PKV_F16, st, mid);
+        // 4 KB stages, 3-slot rings per token group: 48 KB a CTA, four CTAs
+        // (16 warps) per SM to hide the conversion and softmax latency
+        // (measured: 0.84 of the copy peak on the OPT-13B-shaped FP8 batch
+        // against 0.78 with 4-slot rings at three CTAs per SM)
+        if (D == 128 && p.G <= 8) return launch_tc_t<__half, 128, 1, 4, 3, 1>(p, tk, tv, PKV_F16, st, mid);
         return cudaErrorInvalidValue;
     }
     if (kv_dtype == PKV_F16) {

@@ -94,18 +94,19 @@ def test_step_runtime_split_merge_every_kernel(kernel):
     assert launches[-1] == (2 if kernel == pk.PKV_KERNEL_TENSOR else 3)
 
 
-@pytest.mark.parametrize("base,hq,hkv,expect", [
-    ("opt13b", 4, 4, pk.PKV_KERNEL_SIMT_TMA),      # MHA f16
-    ("llama2_70b", 16, 2, pk.PKV_KERNEL_TENSOR),   # GQA bf16, 8 heads per KV head
-    ("falcon7b", 71, 1, pk.PKV_KERNEL_LEAN),       # MQA, 71 heads per KV head
-    ("fp8", 4, 4, pk.PKV_KERNEL_SIMT_TMA),         # FP8 MHA stays on the CUDA cores
-    ("fp8_gqa", 16, 2, pk.PKV_KERNEL_TENSOR),      # FP8 GQA on the tensor cores
+@pytest.mark.parametrize("base,hq,hkv,bs,expect", [
+    ("opt13b", 4, 4, 16, pk.PKV_KERNEL_SIMT_TMA),      # MHA f16
+    ("llama2_70b", 16, 2, 16, pk.PKV_KERNEL_TENSOR),   # GQA bf16, 8 heads per KV head
+    ("falcon7b", 71, 1, 16, pk.PKV_KERNEL_LEAN),       # MQA, 71 heads per KV head
+    ("fp8", 4, 4, 16, pk.PKV_KERNEL_TENSOR),           # FP8 MHA: codes converted for the tensor cores
+    ("fp8", 4, 4, 1, pk.PKV_KERNEL_SIMT_TMA),          # ... but not with one token per block
+    ("fp8_gqa", 16, 2, 16, pk.PKV_KERNEL_TENSOR),      # FP8 GQA on the tensor cores
 ])
-def test_step_runtime_automatic_kernel(base, hq, hkv, expect):
+def test_step_runtime_automatic_kernel(base, hq, hkv, bs, expect):
     import dataclasses
     cfg = dataclasses.replace(wl.CONFIGS[base], n_q_heads=hq, n_kv_heads=hkv, batch=6,
                               lengths=("uniform", 1, 700), samples_per_prompt=1,
-                              min_pool_blocks=0)
+                              min_pool_blocks=0, block_size=bs)
     side = setup_config(cfg, growth=5)
     run_rounds(cfg, side, 3)            # parity of the automatic choice, round by round
     seqs = np.asarray(side.seqs, dtype=np.int64)
