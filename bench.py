@@ -85,10 +85,13 @@ TRAFFIC = {
     # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
     # profiles/decode_tc_llama2_70b.md: 293.6 MB for 286.5 MB algorithmic
     ("llama2_70b", "decode_tc_kernel"):
-        (1.0246, "842062b2b223be4935749be5c717b576c5963d48e2c3ec1603a7a87ed9b35605"),
-    # profiles/decode_tc_fp8_gqa.md: 149.1 MB for 143.3 MB
+        (1.0246, "6ec2258201f5b3d03564f5581282039422efbdb1ccdef741568c55bcb1f27d29"),
+    # profiles/decode_tc_fp8_gqa.md: 148.7 MB for 143.3 MB
     ("fp8_gqa", "decode_tc_kernel"):
-        (1.0405, "842062b2b223be4935749be5c717b576c5963d48e2c3ec1603a7a87ed9b35605"),
+        (1.0381, "6ec2258201f5b3d03564f5581282039422efbdb1ccdef741568c55bcb1f27d29"),
+    # profiles/decode_tc_fp8.md: 1,359.0 MB for 1,343.5 MB
+    ("fp8", "decode_tc_kernel"):
+        (1.0115, "6ec2258201f5b3d03564f5581282039422efbdb1ccdef741568c55bcb1f27d29"),
     # profiles/decode_simt2_opt13b.md: 612.2 MB for 604.1 MB
     ("opt13b", "decode_simt2_kernel"):
         (1.0134, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
@@ -117,8 +120,11 @@ def kernel_sources_sha(kernel: str) -> str:
     return h.hexdigest()
 
 
-def traffic_per_launch(cfg_name: str, kernel: str, algorithmic_bytes: float):
-    entry = TRAFFIC.get((cfg_name, kernel))
+def traffic_per_launch(cfg: wl.Config, kernel: str, algorithmic_bytes: float):
+    # captured at each workload's own block size
+    if cfg.block_size != wl.CONFIGS[cfg.name].block_size:
+        return None
+    entry = TRAFFIC.get((cfg.name, kernel))
     if entry is None or entry[1] != kernel_sources_sha(kernel):
         return None
     return int(entry[0] * algorithmic_bytes)
@@ -526,7 +532,7 @@ def run_ours(args) -> None:
         dec_total_ms = float(np.sum(dec_ms))
         achieved = float(np.sum(prof_bytes)) / (dec_total_ms / 1e3) / 1e9
         kernel_name = pk.KERNEL_NAMES.get(kernel_used, "unknown")
-        traffic = traffic_per_launch(cfg.name, kernel_name, float(np.mean(step_bytes)))
+        traffic = traffic_per_launch(cfg, kernel_name, float(np.mean(step_bytes)))
         line = {
             "metric": METRIC,
             "value": round(value, 2),
