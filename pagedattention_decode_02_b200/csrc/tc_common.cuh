@@ -157,6 +157,15 @@ __device__ __forceinline__ void mask_scores(float (&s)[4], int n, int lane) {
     if (gq + 8 >= n) s[2] = s[3] = -INFINITY;
 }
 
+// 2^x on the special-function unit (ex2.approx, flush-to-zero): its relative
+// error (a few units in the last place of fp32) is far below the f16/bf16
+// rounding of the probabilities it feeds; 2^-inf = 0.
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Online-softmax update of one stage for this lane's two heads; returns P^T
 // as the B operand of the P.V product (pb0 = tokens 0-7, pb1 = tokens 8-15)
 // and rescales o when a running maximum moved.
@@ -175,13 +184,13 @@ __device__ __forceinline__ void softmax_step(const float (&s)[4], float (&o)[MTI
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const float m_new = fmaxf(m_run[h], mx[h]);
-        alpha[h] = exp2f(m_run[h] - m_new);
+        alpha[h] = ex2_fast(m_run[h] - m_new);
         m_run[h] = m_new;
     }
-    const float p0 = exp2f(s[0] - m_run[0]);
-    const float p1 = exp2f(s[1] - m_run[1]);
-    const float p2 = exp2f(s[2] - m_run[0]);
-    const float p3 = exp2f(s[3] - m_run[1]);
+    const float p0 = ex2_fast(s[0] - m_run[0]);
+    const float p1 = ex2_fast(s[1] - m_run[1]);
+    const float p2 = ex2_fast(s[2] - m_run[0]);
+    const float p3 = ex2_fast(s[3] - m_run[1]);
     l_run[0] = l_run[0] * alpha[0] + (p0 + p2);
     l_run[1] = l_run[1] * alpha[1] + (p1 + p3);
     pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
@@ -288,11 +297,16 @@ __device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], co
 //   O^T m-tile mt, fragment row gq / gq + 8  <->  d = 16 gq + 2 mt / + 1.
 // ---------------------------------------------------------------------------
 
-// Two FP8-E4M3 codes (low byte first) -> f16x2, exact (every e4m3 value is an
-// f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-    return *reinterpret_cast<const uint32_t*>(&h);
+// Four FP8-E4M3 codes (one word, low byte first) -> two f16x2: lo = codes 0
+// and 1, hi = codes 2 and 3; exact (every e4m3 value is an f16 value).  The
+// word's 16-bit halves go to the converts as they are, with no shifts or masks.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // Byte offset of the 16-byte chunk c (0..7) of row r in a 16-row tile of
@@ -360,8 +374,9 @@ __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         // word kk: d = 32 tq + 4 kk .. + 3
-        const uint32_t a[4] = {e4m3x2_to_f16x2(k0[kk]), e4m3x2_to_f16x2(k1[kk]),
-                               e4m3x2_to_f16x2(k0[kk] >> 16), e4m3x2_to_f16x2(k1[kk] >> 16)};
+        uint32_t a[4];
+        e4m3x4_to_f16x2(k0[kk], a[0], a[2]);
+        e4m3x4_to_f16x2(k1[kk], a[1], a[3]);
         MmaType<__half>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
     }
     float s[4];
@@ -382,11 +397,12 @@ __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const
         const uint32_t hi01 = byte_perm(x0[j], y0[j], 0x7362u);
         const uint32_t lo23 = byte_perm(x1[j], y1[j], 0x5140u);
         const uint32_t hi23 = byte_perm(x1[j], y1[j], 0x7362u);
-        const uint32_t a0[4] = {e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo01 >> 16),
-                                e4m3x2_to_f16x2(lo23), e4m3x2_to_f16x2(lo23 >> 16)};
+        uint32_t a0[4], a1[4];
+        e4m3x4_to_f16x2(lo01, a0[0], a0[1]);
+        e4m3x4_to_f16x2(lo23, a0[2], a0[3]);
         MmaType<__half>::mma(o[2 * j], a0, pb0, pb1);
-        const uint32_t a1[4] = {e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi01 >> 16),
-                                e4m3x2_to_f16x2(hi23), e4m3x2_to_f16x2(hi23 >> 16)};
+        e4m3x4_to_f16x2(hi01, a1[0], a1[1]);
+        e4m3x4_to_f16x2(hi23, a1[2], a1[3]);
         MmaType<__half>::mma(o[2 * j + 1], a1, pb0, pb1);
     }
 }
