@@ -364,6 +364,22 @@ pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const 
                            const void* d_k_new, const void* d_v_new, float scale, void* d_out,
                            void* stream);
 
+/* pkv_decode_step_host - pkv_decode_step with the round's q, new K/V rows and
+ *   output in HOST memory, for callers whose data lives on the host: the call
+ *   copies h_q, h_k_new and h_v_new into the runtime's own device buffers
+ *   (one cudaMemcpyAsync each on `stream`; made on the first call, sized for
+ *   max_batch), runs the round as pkv_decode_step, copies the output into
+ *   h_out and waits for the stream: h_out holds the round's attention output
+ *   when the call returns.  Pinned host buffers make the copies asynchronous
+ *   and fastest; pageable ones work too.  Shapes and dtype as pkv_decode_step:
+ *   h_q, h_out [B][n_q_heads][head_dim]; h_k_new, h_v_new
+ *   [B][n_kv_heads][head_dim]; all in the step's q_dtype.  Errors as
+ *   pkv_decode_step (nothing changed when it rejects the batch), CUDA for a
+ *   failed copy or allocation. */
+pkv_status pkv_decode_step_host(pkv_step* step, const int64_t* seq_ids, int B, const void* h_q,
+                                const void* h_k_new, const void* h_v_new, float scale,
+                                void* h_out, void* stream);
+
 /* pkv_step_last_launches - number of kernels the last pkv_decode_step call
  *   launched (copy-on-write copy, append, decode, merge). */
 int pkv_step_last_launches(const pkv_step* step);

@@ -128,6 +128,7 @@ _sig("pkv_step_create", _st, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctype
      ctypes.c_int, ctypes.c_int, ctypes.POINTER(_P))
 _sig("pkv_step_destroy", None, _P)
 _sig("pkv_decode_step", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
+_sig("pkv_decode_step_host", _st, _P, _I64P, ctypes.c_int, _P, _P, _P, ctypes.c_float, _P, _P)
 _sig("pkv_step_last_launches", ctypes.c_int, _P)
 _sig("pkv_step_last_kernel", ctypes.c_int, _P)
 _sig("pkv_step_profile", _st, _P, ctypes.c_int, ctypes.c_int)
@@ -145,6 +146,7 @@ EXPORTED = [
     "bt_free_queue", "bt_stats", "kv_append", "block_copy", "paged_decode_attention",
     "paged_decode_attention_ex", "paged_decode_workspace_bytes", "paged_decode_workspace_bytes_ex",
     "pkv_device_error", "pkv_status_str", "pkv_step_create", "pkv_step_destroy", "pkv_decode_step",
+    "pkv_decode_step_host",
     "pkv_step_last_launches", "pkv_step_last_kernel", "pkv_step_profile", "pkv_step_profile_read",
     "paged_decode_attention_static", "paged_decode_static_scratch_bytes", "kv_swap_out", "kv_swap_in",
     "paged_prefill_attention",
@@ -509,6 +511,15 @@ class Step:
         if st != PKV_OK:
             raise PagedKVError(st, "pkv_decode_step")
 
+    def run_host_raw(self, ids: np.ndarray, q_ptr: int, k_ptr: int, v_ptr: int, scale: float,
+                     out_ptr: int, stream_ptr: int) -> None:
+        """pkv_decode_step_host with pre-resolved HOST pointers: returns with the
+        round's output in the host buffer at ``out_ptr``."""
+        st = _lib.pkv_decode_step_host(self.handle, ids.ctypes.data_as(_I64P), int(ids.size),
+                                       q_ptr, k_ptr, v_ptr, scale, out_ptr, stream_ptr)
+        if st != PKV_OK:
+            raise PagedKVError(st, "pkv_decode_step_host")
+
 
 def pkv_step_create(pool: Pool, max_batch: int, max_blocks: int, n_q_heads: int, q_dtype,
                     partition_tokens: int = 0, kernel: int = PKV_KERNEL_AUTO,
@@ -529,6 +540,33 @@ def pkv_decode_step(step: Step, seq_ids, q, k_new, v_new, scale: float, out, str
     _check(_lib.pkv_decode_step(step.handle, ids.ctypes.data_as(_I64P), int(ids.size),
                                 _dev_ptr(q), _dev_ptr(k_new), _dev_ptr(v_new), float(scale),
                                 _dev_ptr(out), _stream_ptr(stream)), "pkv_decode_step")
+
+
+def _host_ptr(t) -> int:
+    """Address of a contiguous host buffer: a CPU torch tensor (pinned or not)
+    or a numpy array."""
+    if isinstance(t, np.ndarray):
+        if not t.flags["C_CONTIGUOUS"]:
+            raise ValueError("expected a contiguous array")
+        return t.ctypes.data
+    if t.is_cuda:
+        raise ValueError("expected a host tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def pkv_decode_step_host(step: Step, seq_ids, q, k_new, v_new, scale: float, out,
+                         stream=None) -> None:
+    """pkv_decode_step with q, k_new, v_new and out in host memory (CPU torch
+    tensors, pinned for speed, or numpy arrays of the q dtype's bits); returns
+    with the round's attention output in ``out``."""
+    ids = seq_ids if isinstance(seq_ids, np.ndarray) and seq_ids.dtype == np.int64 \
+        else np.ascontiguousarray(seq_ids, dtype=np.int64)
+    _check(_lib.pkv_decode_step_host(step.handle, ids.ctypes.data_as(_I64P), int(ids.size),
+                                     _host_ptr(q), _host_ptr(k_new), _host_ptr(v_new),
+                                     float(scale), _host_ptr(out), _stream_ptr(stream)),
+           "pkv_decode_step_host")
 
 
 def pkv_step_last_launches(step: Step) -> int:

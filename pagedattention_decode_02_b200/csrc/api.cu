@@ -537,6 +537,7 @@ struct pkv_step {
     void* d_ws = nullptr;
     size_t ws_bytes = 0;
     int* d_counters = nullptr;        // [max_batch][n_q_heads], zero between launches
+    uint8_t* d_io = nullptr;          // pkv_decode_step_host: q | k | v | out, made on first use
     int max_parts = 1;
     int last_launches = 0;
     int last_kernel = 0;              // decode kernel of the last round (after the auto choice)
@@ -588,6 +589,7 @@ void step_free(pkv_step* s) {
     if (s->d_tables) cudaFree(s->d_tables);
     if (s->d_ws) cudaFree(s->d_ws);
     if (s->d_counters) cudaFree(s->d_counters);
+    if (s->d_io) cudaFree(s->d_io);
     delete s;
 }
 
@@ -689,6 +691,46 @@ pkv_status pkv_step_create(pkv_pool* pool, int max_batch, int max_seqs, int max_
 
 void pkv_step_destroy(pkv_step* s) {
     if (s) step_free(s);
+}
+
+pkv_status pkv_decode_step_host(pkv_step* s, const int64_t* seq_ids, int B, const void* h_q,
+                                const void* h_k_new, const void* h_v_new, float scale,
+                                void* h_out, void* stream) {
+    if (!s || B < 0 || B > s->max_batch) return PKV_ERR_INVALID_ARG;
+    if (B == 0) {
+        s->last_launches = 0;
+        s->last_kernel = 0;
+        return PKV_OK;
+    }
+    if (!seq_ids || !h_q || !h_k_new || !h_v_new || !h_out) return PKV_ERR_INVALID_ARG;
+    pkv_pool* pool = s->pool;
+    if (!same_device(pool)) return PKV_ERR_INVALID_ARG;
+    const size_t elem = s->q_dtype == PKV_F32 ? 4 : 2;
+    const size_t q_row = (size_t)s->n_q_heads * pool->head_dim * elem;
+    const size_t kv_row = (size_t)pool->n_kv_heads * pool->head_dim * elem;
+    auto up16 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t q_cap = up16(q_row * s->max_batch), kv_cap = up16(kv_row * s->max_batch);
+    if (!s->d_io && cudaMalloc(&s->d_io, 2 * q_cap + 2 * kv_cap) != cudaSuccess) {
+        s->d_io = nullptr;
+        return PKV_ERR_CUDA;
+    }
+    uint8_t* d_q = s->d_io;
+    uint8_t* d_k = d_q + q_cap;
+    uint8_t* d_v = d_k + kv_cap;
+    uint8_t* d_out = d_v + kv_cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(d_q, h_q, q_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_k, h_k_new, kv_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_v, h_v_new, kv_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const pkv_status ps = pkv_decode_step(s, seq_ids, B, d_q, d_k, d_v, scale, d_out, stream);
+    if (ps != PKV_OK) {
+        cudaStreamSynchronize(st);   // the input copies read the caller's buffers
+        return ps;
+    }
+    if (cudaMemcpyAsync(h_out, d_out, q_row * B, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 int pkv_step_last_launches(const pkv_step* s) { return s ? s->last_launches : 0; }

@@ -275,3 +275,36 @@ def test_prefix_cached_prompts(bs):
     gpu, ref, _ = decode_step(side, [0, 1, 2, 3], 0)
     compare_out(gpu, ref, "f16")
     check_pool_bytes(side)
+
+
+@pytest.mark.parametrize("base,dt,pinned", [("opt13b", "f16", True), ("llama2_70b", "bf16", False),
+                                            ("fp8_gqa", "f16", True)])
+def test_step_runtime_host_buffers(base, dt, pinned):
+    # the host-buffer entry point: q/k/v in from host memory, out back to it,
+    # round after round against the oracle
+    import dataclasses
+    cfg = dataclasses.replace(wl.CONFIGS[base], n_q_heads=8, n_kv_heads=2 if base != "opt13b" else 8,
+                              batch=7, lengths=("uniform", 1, 900), min_pool_blocks=0)
+    side = setup_config(cfg, growth=4)
+    seqs = np.asarray(side.seqs, dtype=np.int64)
+    max_blocks = max(len(side.orc.bm.tables[s]) for s in side.seqs) + 2
+    step = pk.Step(side.pool, len(seqs), max_blocks, cfg.n_q_heads, cfg.q_dtype)
+    tdt = torch.bfloat16 if cfg.q_dtype == "bf16" else torch.float16
+    out = torch.empty((len(seqs), cfg.n_q_heads, cfg.head_dim), dtype=tdt)
+    if pinned:
+        out = out.pin_memory()
+    for t in range(4):
+        q, kn, vn = step_inputs(side, seqs, t)
+        hq, hk, hv = (to_torch(a, cfg.q_dtype).cpu() for a in (q, kn, vn))
+        if pinned:
+            hq, hk, hv = hq.pin_memory(), hk.pin_memory(), hv.pin_memory()
+        pk.pkv_decode_step_host(step, seqs, hq, hk, hv, cfg.scale, out)
+        side.orc.append(list(seqs), kn, vn, cfg.q_dtype)
+        ref = side.orc.attend(list(seqs), q, cfg.q_dtype, cfg.scale)
+        gpu = to_f64(from_torch(out, cfg.q_dtype), cfg.q_dtype)   # no synchronize: the call waited
+        compare_out(gpu, ref, "fp8" if cfg.kv_dtype == "fp8" else cfg.q_dtype)
+    assert pk.pkv_device_error(side.pool) == 0
+    # a rejected batch (table overflow) changes nothing and reports INVALID_ARG
+    small = pk.Step(side.pool, len(seqs), 1, cfg.n_q_heads, cfg.q_dtype)
+    with pytest.raises(pk.PagedKVError):
+        pk.pkv_decode_step_host(small, seqs, hq, hk, hv, cfg.scale, out)
