@@ -368,7 +368,9 @@ pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const 
  *   output in HOST memory, for callers whose data lives on the host: the call
  *   copies h_q, h_k_new and h_v_new into the runtime's own device buffers
  *   (one cudaMemcpyAsync each on `stream`; made on the first call, sized for
- *   max_batch), runs the round as pkv_decode_step, copies the output into
+ *   max_batch; when h_k_new and h_v_new directly follow h_q in one packed
+ *   host buffer q | k | v, the three travel in a single copy), runs the round
+ *   as pkv_decode_step, copies the output into
  *   h_out and waits for the stream: h_out holds the round's attention output
  *   when the call returns.  Pinned host buffers make the copies asynchronous
  *   and fastest; pageable ones work too.  Shapes and dtype as pkv_decode_step:

@@ -714,15 +714,27 @@ pkv_status pkv_decode_step_host(pkv_step* s, const int64_t* seq_ids, int B, cons
         s->d_io = nullptr;
         return PKV_ERR_CUDA;
     }
+    // q | k | v back to back on the device (rows are multiples of 16 bytes), so
+    // that a caller's packed host buffer travels in one copy
     uint8_t* d_q = s->d_io;
-    uint8_t* d_k = d_q + q_cap;
-    uint8_t* d_v = d_k + kv_cap;
-    uint8_t* d_out = d_v + kv_cap;
+    uint8_t* d_k = d_q + q_row * B;
+    uint8_t* d_v = d_k + kv_row * B;
+    uint8_t* d_out = s->d_io + q_cap + 2 * kv_cap;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(d_q, h_q, q_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(d_k, h_k_new, kv_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(d_v, h_v_new, kv_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    const uint8_t* hq8 = static_cast<const uint8_t*>(h_q);
+    const bool packed = static_cast<const uint8_t*>(h_k_new) == hq8 + q_row * B &&
+                        static_cast<const uint8_t*>(h_v_new) == hq8 + q_row * B + kv_row * B;
+    if (packed) {
+        if (cudaMemcpyAsync(d_q, h_q, (q_row + 2 * kv_row) * B, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess)
+            return PKV_ERR_CUDA;
+    } else if (cudaMemcpyAsync(d_q, h_q, q_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+               cudaMemcpyAsync(d_k, h_k_new, kv_row * B, cudaMemcpyHostToDevice, st) !=
+                   cudaSuccess ||
+               cudaMemcpyAsync(d_v, h_v_new, kv_row * B, cudaMemcpyHostToDevice, st) !=
+                   cudaSuccess) {
         return PKV_ERR_CUDA;
+    }
     const pkv_status ps = pkv_decode_step(s, seq_ids, B, d_q, d_k, d_v, scale, d_out, stream);
     if (ps != PKV_OK) {
         cudaStreamSynchronize(st);   // the input copies read the caller's buffers

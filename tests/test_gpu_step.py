@@ -277,9 +277,11 @@ def test_prefix_cached_prompts(bs):
     check_pool_bytes(side)
 
 
-@pytest.mark.parametrize("base,dt,pinned", [("opt13b", "f16", True), ("llama2_70b", "bf16", False),
-                                            ("fp8_gqa", "f16", True)])
-def test_step_runtime_host_buffers(base, dt, pinned):
+@pytest.mark.parametrize("base,dt,pinned,packed", [("opt13b", "f16", True, False),
+                                                   ("llama2_70b", "bf16", False, False),
+                                                   ("fp8_gqa", "f16", True, True),
+                                                   ("opt13b", "f16", False, True)])
+def test_step_runtime_host_buffers(base, dt, pinned, packed):
     # the host-buffer entry point: q/k/v in from host memory, out back to it,
     # round after round against the oracle
     import dataclasses
@@ -296,7 +298,12 @@ def test_step_runtime_host_buffers(base, dt, pinned):
     for t in range(4):
         q, kn, vn = step_inputs(side, seqs, t)
         hq, hk, hv = (to_torch(a, cfg.q_dtype).cpu() for a in (q, kn, vn))
-        if pinned:
+        if packed:   # one host buffer q | k | v: the inputs travel in one copy
+            buf = torch.cat([hq.flatten(), hk.flatten(), hv.flatten()])
+            buf = buf.pin_memory() if pinned else buf
+            nq, nk = hq.numel(), hk.numel()
+            hq, hk, hv = buf[:nq].view(hq.shape), buf[nq:nq + nk].view(hk.shape), buf[nq + nk:].view(hv.shape)
+        elif pinned:
             hq, hk, hv = hq.pin_memory(), hk.pin_memory(), hv.pin_memory()
         pk.pkv_decode_step_host(step, seqs, hq, hk, hv, cfg.scale, out)
         side.orc.append(list(seqs), kn, vn, cfg.q_dtype)
