@@ -724,24 +724,27 @@ pkv_status pkv_decode_step_host(pkv_step* s, const int64_t* seq_ids, int B, cons
     const uint8_t* hq8 = static_cast<const uint8_t*>(h_q);
     const bool packed = static_cast<const uint8_t*>(h_k_new) == hq8 + q_row * B &&
                         static_cast<const uint8_t*>(h_v_new) == hq8 + q_row * B + kv_row * B;
+    // on any failure, wait for copies already queued: they read or write the
+    // caller's buffers, which the caller may release once the call returns
+    auto fail = [&](pkv_status e) {
+        cudaStreamSynchronize(st);
+        return e;
+    };
     if (packed) {
         if (cudaMemcpyAsync(d_q, h_q, (q_row + 2 * kv_row) * B, cudaMemcpyHostToDevice, st) !=
             cudaSuccess)
-            return PKV_ERR_CUDA;
+            return fail(PKV_ERR_CUDA);
     } else if (cudaMemcpyAsync(d_q, h_q, q_row * B, cudaMemcpyHostToDevice, st) != cudaSuccess ||
                cudaMemcpyAsync(d_k, h_k_new, kv_row * B, cudaMemcpyHostToDevice, st) !=
                    cudaSuccess ||
                cudaMemcpyAsync(d_v, h_v_new, kv_row * B, cudaMemcpyHostToDevice, st) !=
                    cudaSuccess) {
-        return PKV_ERR_CUDA;
+        return fail(PKV_ERR_CUDA);
     }
     const pkv_status ps = pkv_decode_step(s, seq_ids, B, d_q, d_k, d_v, scale, d_out, stream);
-    if (ps != PKV_OK) {
-        cudaStreamSynchronize(st);   // the input copies read the caller's buffers
-        return ps;
-    }
+    if (ps != PKV_OK) return fail(ps);
     if (cudaMemcpyAsync(h_out, d_out, q_row * B, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return PKV_ERR_CUDA;
+        return fail(PKV_ERR_CUDA);
     return cudaStreamSynchronize(st) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
