@@ -58,14 +58,7 @@ constexpr int kAutoPartition = 512;
 // no partial states, no merge (measured on the OPT-13B-shaped batch, 1,200
 // one-head CTAs: unsplit 0.97 of the copy peak against 0.92-0.93 for 512 to
 // 1024-token partitions).
-int pool_sms(const pkv_pool* pool) {
-    int n = 0;
-    if (pool->device < 0 ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, pool->device) != cudaSuccess ||
-        n <= 0)
-        return 148;
-    return n;
-}
+int pool_sms(const pkv_pool* pool) { return pool->sm_count > 0 ? pool->sm_count : 148; }
 
 long long unsplit_units(const pkv_pool* pool, int B, int n_q_heads) {
     const int G = n_q_heads / pool->n_kv_heads;
@@ -146,7 +139,9 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
     p->host_only = host_only;
     p->bytes = bytes;
     if (!host_only) {
-        if (cudaGetDevice(&p->device) != cudaSuccess) {
+        if (cudaGetDevice(&p->device) != cudaSuccess ||
+            cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
+                cudaSuccess) {
             delete p;
             return PKV_ERR_CUDA;
         }

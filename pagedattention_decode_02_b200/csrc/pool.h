@@ -20,6 +20,7 @@ struct pkv_pool {
     bool host_only = false;
     bool owns_buffers = false;
     int device = -1;
+    int sm_count = 0;       // streaming multiprocessors of `device` (0: unknown)
     uint8_t* k = nullptr;   // device [num_blocks][n_kv_heads][block_size][head_dim]
     uint8_t* v = nullptr;
     size_t bytes = 0;       // bytes of one of the two buffers
