@@ -101,7 +101,7 @@ TRAFFIC = {
     # profiles/decode_lean_falcon7b.md: 2.98 MB for 8.31 MB (the samples of one
     # prompt share its blocks; the re-reads within a launch hit L2)
     ("falcon7b", "decode_lean_kernel"):
-        (0.3579, "4453b2bd0e811c0dded26785d384cc2f2c0cee824f73dc24064abae01d74fb6d"),
+        (0.3579, "b86acad210bccc586492a5dc87259763a1a6bc49bd327097f9d1f6005d917aba"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),

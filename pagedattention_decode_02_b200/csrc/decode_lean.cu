@@ -474,8 +474,8 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             continue;
         }
-        // partial state of this piece -> its workspace slot, then hand it to
-        // the merge warp (no wait here)
+        // partial state of this piece -> its workspace slot; the worker that
+        // finishes the pair's last piece merges them all (counter below)
         const int pair = pc.seq * H_kv + pc.g;
         const size_t slot_id = (size_t)pair + vw;
         float* acc = p.ws_acc + slot_id * G * D;
