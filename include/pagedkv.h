@@ -359,7 +359,14 @@ void pkv_step_destroy(pkv_step* step);
  *   [B][n_kv_heads][head_dim]; d_out: device [B][n_q_heads][head_dim]; all in
  *   q_dtype.  Returns INVALID_ARG if a table would exceed max_blocks (nothing
  *   changed).  The host returns once the work is queued; staging slots are
- *   reused only after their copies completed. */
+ *   reused only after their copies completed.
+ *   Errors: INVALID_ARG, UNKNOWN_SEQ, NO_BLOCKS - returned by step 1 or
+ *   before it, with nothing changed; CUDA - a copy or launch of steps 2-3
+ *   failed after step 1 had been applied: the block manager then holds the
+ *   round's appends (lengths, new blocks, copy-on-write) although no key or
+ *   value was written, so the caller must bt_free (or bt_reset) the batch's
+ *   sequences before using them again.  A failed launch usually means the
+ *   CUDA context itself is lost. */
 pkv_status pkv_decode_step(pkv_step* step, const int64_t* seq_ids, int B, const void* d_q,
                            const void* d_k_new, const void* d_v_new, float scale, void* d_out,
                            void* stream);
@@ -441,17 +448,24 @@ pkv_status kv_swap_in(pkv_pool* pool, int64_t seq_id, const void* h_k, const voi
  *   counterpart: this is a deployment variant of the same computation.
  *   Arguments and results as paged_decode_attention_ex with kernel = AUTO,
  *   except that no workspace is passed: the split-context scratch is a
- *   file-scope device array of paged_decode_static_scratch_bytes() (8 MiB),
- *   held by every GPU that loads the library until the process exits.  This
- *   call allocates nothing.
- *   partition_tokens: 0 = automatic - the library's choice, or longer
- *   partitions (less scratch) until the scratch fits, down to an unsplit pass
- *   that needs none; > 0 (a multiple of 16) or -1 as in
+ *   file-scope device array of paged_decode_static_scratch_bytes() (8 MiB).
+ *   Placing that array on a device is itself an allocation (CUDA loads the
+ *   library's device code lazily), so kv_pool_create does it for the pool's
+ *   device, while allocating is still allowed: from the first pool created
+ *   on a device, that device holds the array until the process exits, and
+ *   this call allocates nothing there.  Create the pool before another
+ *   allocator takes the GPU.  On a device with no pool created yet, the
+ *   first call looks the array up itself (cudaGetSymbolAddress, with that
+ *   device current), which places it - make such a call before any stream
+ *   capture; if that fails the call returns PKV_ERR_CUDA.
+ *   partition_tokens: 0 = automatic - the library's choice as
+ *   paged_decode_attention makes it (without the stage-balanced kernel when
+ *   only its share exceeds the scratch), else partitions lengthened from the
+ *   automatic length (less scratch) until the scratch fits, down to an
+ *   unsplit pass that needs none; > 0 (a multiple of 16) or -1 as in
  *   paged_decode_attention_ex, and a request whose scratch exceeds the limit
  *   returns PKV_ERR_SCRATCH_LIMIT without launching anything.
- *   The first call on a device looks up the array's device address for that
- *   device (cudaGetSymbolAddress, with that device current); make that first
- *   call before any stream capture.  All calls share the one array and it
+ *   All calls share the one array and it
  *   keeps the last call's contents; nothing in it needs to start at zero
  *   (every partition's state is written before the merge reads it), but calls
  *   whose kernels overlap on the GPU - on different streams, or from several

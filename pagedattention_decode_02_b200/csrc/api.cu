@@ -14,6 +14,7 @@
 #include "decode_launch.h"
 #include "pagedkv.h"
 #include "pool.h"
+#include "trace.h"
 
 using pkv::BlockManager;
 
@@ -91,6 +92,25 @@ size_t workspace_for(const pkv_pool* pool, int B, int n_q_heads, int max_parts) 
 }
 
 }  // namespace
+
+namespace pkv {
+// The automatic partition length and the workspace the partitioned kernels
+// need for it, without the stage-balanced kernel's share (used by the
+// no-allocation call to keep the library's own choice when only that share
+// would not fit its scratch).
+int decode_auto_partition(const pkv_pool* pool, int B, int n_q_heads, int max_blocks) {
+    return resolve_partition(pool, max_blocks, 0, n_q_heads / pool->n_kv_heads,
+                             unsplit_units(pool, B, n_q_heads));
+}
+size_t decode_workspace_bytes_partitioned(const pkv_pool* pool, int B, int n_q_heads,
+                                          int max_blocks, int partition_tokens) {
+    const int P = resolve_partition(pool, max_blocks, partition_tokens,
+                                    n_q_heads / pool->n_kv_heads,
+                                    unsplit_units(pool, B, n_q_heads));
+    if (P <= 0 || P % 16) return 0;
+    return workspace_for(pool, B, n_q_heads, parts_for(pool, max_blocks, P));
+}
+}  // namespace pkv
 
 extern "C" {
 
@@ -172,6 +192,10 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
             return PKV_ERR_CUDA;
         }
         pkv::pool_init_device_extras(p);
+        // the no-allocation decode call's scratch array: placed on this device
+        // now, while allocating is allowed (a failure here is not fatal; that
+        // call looks it up again and reports PKV_ERR_CUDA if it still fails)
+        (void)pkv::static_scratch_prepare(p->device);
     }
     *out = p;
     return PKV_OK;
@@ -272,6 +296,7 @@ pkv_status bt_stats(const pkv_pool* p, pkv_stats* out) {
 // ---------------------------------------------------------------------------
 pkv_status kv_append(pkv_pool* p, const int32_t* slots, int n_tokens, const void* k, const void* v,
                      pkv_dtype in_dtype, void* stream) {
+    PKV_TRACE("kv_append");
     if (!p || p->host_only || n_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (!valid_dtype(in_dtype)) return PKV_ERR_INVALID_ARG;
     if (p->dtype == PKV_FP8_E4M3 ? in_dtype == PKV_FP8_E4M3 : in_dtype != p->dtype)
@@ -288,6 +313,7 @@ pkv_status kv_append(pkv_pool* p, const int32_t* slots, int n_tokens, const void
 
 pkv_status block_copy(pkv_pool* p, const int32_t* src, const int32_t* dst, int n_pairs,
                       void* stream) {
+    PKV_TRACE("block_copy");
     if (!p || p->host_only || n_pairs < 0) return PKV_ERR_INVALID_ARG;
     if (n_pairs == 0) return PKV_OK;
     if (!src || !dst) return PKV_ERR_INVALID_ARG;
@@ -451,6 +477,7 @@ pkv_status paged_decode_attention_ex(pkv_pool* p, const void* q, pkv_dtype q_dty
                                      int B, int n_q_heads, float scale, void* out, void* ws,
                                      size_t ws_bytes, int partition_tokens, int kernel,
                                      void* stream) {
+    PKV_TRACE("paged_decode_attention_ex");
     return decode_attention_impl(p, q, q_dtype, tables, max_blocks, lens, B, n_q_heads, scale, out,
                                  ws, ws_bytes, partition_tokens, kernel, stream, nullptr, nullptr,
                                  nullptr);
@@ -468,6 +495,7 @@ pkv_status paged_prefill_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype
                                    const int32_t* q_starts, int max_q_len, const int32_t* tables,
                                    int max_blocks, const int32_t* lens, int B, int n_q_heads,
                                    float scale, void* out, void* stream) {
+    PKV_TRACE("paged_prefill_attention");
     if (!p || p->host_only || B < 0 || max_q_len < 0) return PKV_ERR_INVALID_ARG;
     if (B == 0 || max_q_len == 0) return PKV_OK;
     if (!q || !out || !q_starts || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
@@ -691,6 +719,7 @@ void pkv_step_destroy(pkv_step* s) {
 pkv_status pkv_decode_step_host(pkv_step* s, const int64_t* seq_ids, int B, const void* h_q,
                                 const void* h_k_new, const void* h_v_new, float scale,
                                 void* h_out, void* stream) {
+    PKV_TRACE("pkv_decode_step_host");
     if (!s || B < 0 || B > s->max_batch) return PKV_ERR_INVALID_ARG;
     if (B == 0) {
         s->last_launches = 0;
@@ -750,6 +779,7 @@ int pkv_step_last_kernel(const pkv_step* s) { return s ? s->last_kernel : 0; }
 pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const void* q,
                            const void* k_new, const void* v_new, float scale, void* out,
                            void* stream) {
+    PKV_TRACE("pkv_decode_step");
     if (!s || B < 0 || B > s->max_batch) return PKV_ERR_INVALID_ARG;
     s->last_launches = 0;
     s->last_kernel = 0;

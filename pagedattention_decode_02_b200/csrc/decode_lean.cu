@@ -28,6 +28,8 @@
 // records it).  Every wait is bounded.
 #include <cuda.h>
 
+#include <atomic>
+
 #include <algorithm>
 #include <cfloat>
 
@@ -526,23 +528,9 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
             (void)mbar_wait(&full[j % RG], (uint32_t)((j / RG) & 1));
 }
 
-int sm_count(int device) {
-    static int cached[64] = {};
-    if (device < 0 || device >= 64) return 0;
-    if (!cached[device]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
-            cudaGetLastError();
-            return 0;
-        }
-        cached[device] = n;
-    }
-    return cached[device];
-}
-
 template <typename T, int D, int MT>
 cudaError_t launch_lean_t(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                          int device, cudaStream_t st, cudaEvent_t mid) {
+                          int sms, cudaStream_t st, cudaEvent_t mid) {
     using S = LeanShape<D, MT>;
     constexpr int threads = S::TS * MT * 32;
     const int smem = (lean_fixed_smem<D, MT>() + (p.B + 1) * 4 + 15) & ~15;
@@ -550,16 +538,21 @@ cudaError_t launch_lean_t(const DecodeParams& p, const CUtensorMap* tk, const CU
     static unsigned long long attr_done = 0;
     cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
-    // one wave of persistent CTAs
-    static int last_smem = -1, last_per_sm = 0;
-    if (smem != last_smem) {
+    // one wave of persistent CTAs; the occupancy of the last shared-memory
+    // size is cached as one atomic word (size << 32 | CTAs per SM), so that
+    // calls from several host threads never see a half-written pair
+    static std::atomic<unsigned long long> occ_cache{~0ull};
+    unsigned long long occ = occ_cache.load(std::memory_order_acquire);
+    int per_sm = (int)(occ & 0xffffffffull);
+    if ((occ >> 32) != (unsigned long long)(unsigned)smem) {
         int n = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
         if (e != cudaSuccess) return e;
-        last_per_sm = std::max(1, std::min(n, kLeanMaxWorkersPerSm / S::TS));
-        last_smem = smem;
+        per_sm = std::max(1, std::min(n, kLeanMaxWorkersPerSm / S::TS));
+        occ_cache.store(((unsigned long long)(unsigned)smem << 32) | (unsigned)per_sm,
+                        std::memory_order_release);
     }
-    const int grid = std::max(1, sm_count(device)) * last_per_sm;
+    const int grid = std::max(1, sms) * per_sm;
     e = launch_kernel(kern, dim3(grid), dim3(threads), smem, st, p.pdl != 0, *tk, *tv, p);
     if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
     return e;
@@ -567,25 +560,25 @@ cudaError_t launch_lean_t(const DecodeParams& p, const CUtensorMap* tk, const CU
 
 template <typename T, int D>
 cudaError_t launch_lean_d(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                          int device, cudaStream_t st, cudaEvent_t mid) {
+                          int sms, cudaStream_t st, cudaEvent_t mid) {
     // warps of 8 query heads each
     switch ((p.G + 7) / 8) {
-        case 1: return launch_lean_t<T, D, 1>(p, tk, tv, device, st, mid);
-        case 2: return launch_lean_t<T, D, 2>(p, tk, tv, device, st, mid);
-        case 3: return launch_lean_t<T, D, 3>(p, tk, tv, device, st, mid);
-        case 4: return launch_lean_t<T, D, 4>(p, tk, tv, device, st, mid);
-        case 5: return launch_lean_t<T, D, 5>(p, tk, tv, device, st, mid);
-        case 6: return launch_lean_t<T, D, 6>(p, tk, tv, device, st, mid);
-        case 7: return launch_lean_t<T, D, 7>(p, tk, tv, device, st, mid);
-        case 8: return launch_lean_t<T, D, 8>(p, tk, tv, device, st, mid);
-        case 9: return launch_lean_t<T, D, 9>(p, tk, tv, device, st, mid);
-        case 10: return launch_lean_t<T, D, 10>(p, tk, tv, device, st, mid);
-        case 11: return launch_lean_t<T, D, 11>(p, tk, tv, device, st, mid);
-        case 12: return launch_lean_t<T, D, 12>(p, tk, tv, device, st, mid);
-        case 13: return launch_lean_t<T, D, 13>(p, tk, tv, device, st, mid);
-        case 14: return launch_lean_t<T, D, 14>(p, tk, tv, device, st, mid);
-        case 15: return launch_lean_t<T, D, 15>(p, tk, tv, device, st, mid);
-        case 16: return launch_lean_t<T, D, 16>(p, tk, tv, device, st, mid);
+        case 1: return launch_lean_t<T, D, 1>(p, tk, tv, sms, st, mid);
+        case 2: return launch_lean_t<T, D, 2>(p, tk, tv, sms, st, mid);
+        case 3: return launch_lean_t<T, D, 3>(p, tk, tv, sms, st, mid);
+        case 4: return launch_lean_t<T, D, 4>(p, tk, tv, sms, st, mid);
+        case 5: return launch_lean_t<T, D, 5>(p, tk, tv, sms, st, mid);
+        case 6: return launch_lean_t<T, D, 6>(p, tk, tv, sms, st, mid);
+        case 7: return launch_lean_t<T, D, 7>(p, tk, tv, sms, st, mid);
+        case 8: return launch_lean_t<T, D, 8>(p, tk, tv, sms, st, mid);
+        case 9: return launch_lean_t<T, D, 9>(p, tk, tv, sms, st, mid);
+        case 10: return launch_lean_t<T, D, 10>(p, tk, tv, sms, st, mid);
+        case 11: return launch_lean_t<T, D, 11>(p, tk, tv, sms, st, mid);
+        case 12: return launch_lean_t<T, D, 12>(p, tk, tv, sms, st, mid);
+        case 13: return launch_lean_t<T, D, 13>(p, tk, tv, sms, st, mid);
+        case 14: return launch_lean_t<T, D, 14>(p, tk, tv, sms, st, mid);
+        case 15: return launch_lean_t<T, D, 15>(p, tk, tv, sms, st, mid);
+        case 16: return launch_lean_t<T, D, 16>(p, tk, tv, sms, st, mid);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -601,13 +594,13 @@ bool lean_supported(const pkv_pool* pool, int q_dtype, int group, int B, int max
     // stage counts of the whole batch stay within int
     const long long stages = ((long long)max_blocks * pool->block_size + kStageTokens - 1) /
                              kStageTokens;
-    return (long long)B * stages < (1LL << 31) && sm_count(pool->device) > 0;
+    return (long long)B * stages < (1LL << 31) && pool->sm_count > 0;
 }
 
 // piece slots: pair + worker index
 size_t lean_slots(const pkv_pool* pool, int B) {
     const size_t pairs = (size_t)B * pool->n_kv_heads;
-    return pairs + (size_t)sm_count(pool->device) * kLeanMaxWorkersPerSm;
+    return pairs + (size_t)pool->sm_count * kLeanMaxWorkersPerSm;
 }
 
 size_t lean_workspace_bytes(const pkv_pool* pool, int B, int n_q_heads) {
@@ -635,12 +628,12 @@ cudaError_t launch_decode_lean(DecodeParams p, const pkv_pool* pool, void* ws, c
     const CUtensorMap* tk = reinterpret_cast<const CUtensorMap*>(pool->tmap_k);
     const CUtensorMap* tv = reinterpret_cast<const CUtensorMap*>(pool->tmap_v);
     if (pool->dtype == PKV_F16) {
-        if (pool->head_dim == 64) return launch_lean_d<__half, 64>(p, tk, tv, pool->device, st, mid);
-        if (pool->head_dim == 128) return launch_lean_d<__half, 128>(p, tk, tv, pool->device, st, mid);
+        if (pool->head_dim == 64) return launch_lean_d<__half, 64>(p, tk, tv, pool->sm_count, st, mid);
+        if (pool->head_dim == 128) return launch_lean_d<__half, 128>(p, tk, tv, pool->sm_count, st, mid);
     } else if (pool->dtype == PKV_BF16) {
-        if (pool->head_dim == 64) return launch_lean_d<__nv_bfloat16, 64>(p, tk, tv, pool->device, st, mid);
+        if (pool->head_dim == 64) return launch_lean_d<__nv_bfloat16, 64>(p, tk, tv, pool->sm_count, st, mid);
         if (pool->head_dim == 128)
-            return launch_lean_d<__nv_bfloat16, 128>(p, tk, tv, pool->device, st, mid);
+            return launch_lean_d<__nv_bfloat16, 128>(p, tk, tv, pool->sm_count, st, mid);
     }
     return cudaErrorInvalidValue;
 }

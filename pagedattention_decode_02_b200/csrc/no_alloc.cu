@@ -10,13 +10,21 @@
 //
 // What it does: the split-context scratch (per-partition max, sum and
 // accumulator) lives in one file-scope device array of kScratchBytes, part of
-// the library image: every GPU that loads the library holds it until the
-// process exits.  Its device address is looked up once per device with
-// cudaGetSymbolAddress (the array's name in host code is only a host-side
-// stand-in) and handed to the regular decode launch as its workspace.
+// the library image.  The array's name in host code is only a host-side
+// stand-in; its device address is looked up once per device with
+// cudaGetSymbolAddress and handed to the regular decode launch as its
+// workspace.  With CUDA's lazy module loading the array is placed on a device
+// only when its module is first touched there - and placing it is itself an
+// allocation.  kv_pool_create (which allocates anyway) therefore performs the
+// lookup for the pool's device, so the array is in place before a caller's
+// allocator takes the GPU; from then on the device holds it until the process
+// exits.  The lookup on the first static call is only a fallback for a device
+// no pool was created on.
 #include <mutex>
 
 #include "pagedkv.h"
+#include "pool.h"
+#include "trace.h"
 
 namespace {
 
@@ -28,21 +36,34 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 std::mutex g_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// device address of the scratch array on the current device (looked up on the
-// first call for that device); nullptr on failure
-void* scratch_for_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+// device address of the scratch array on device `dev`, which must be the
+// current device (looked up on first use for that device); nullptr on failure
+void* scratch_for_device(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_scratch_addr[dev]) {
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess) {
+            cudaGetLastError();   // leave no sticky error for the caller's next call
+            return nullptr;
+        }
         g_scratch_addr[dev] = ptr;
     }
     return g_scratch_addr[dev];
 }
 
+void* scratch_for_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    return scratch_for_device(dev);
+}
+
 }  // namespace
+
+namespace pkv {
+// called by kv_pool_create with the pool's device current
+bool static_scratch_prepare(int device) { return scratch_for_device(device) != nullptr; }
+}  // namespace pkv
 
 extern "C" {
 
@@ -53,22 +74,33 @@ pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dt
                                          const int32_t* d_context_lens, int B, int n_q_heads,
                                          float scale, void* d_out, int partition_tokens,
                                          void* stream) {
+    PKV_TRACE("paged_decode_attention_static");
     if (!pool || B < 0 || max_blocks < 1 || n_q_heads < 1) return PKV_ERR_INVALID_ARG;
     if (B == 0) return PKV_OK;
+    if (pool->host_only || n_q_heads % pool->n_kv_heads) return PKV_ERR_INVALID_ARG;
     int part = partition_tokens;
     size_t need = paged_decode_workspace_bytes_ex(pool, B, n_q_heads, max_blocks, part);
-    if (part == 0) {
-        // automatic: the library's own choice, or longer partitions (less
-        // scratch) until the scratch fits; an unsplit pass needs none
-        for (int p = 1024; need > kScratchBytes && p <= (1 << 29); p *= 2) {
-            part = p;
-            need = paged_decode_workspace_bytes_ex(pool, B, n_q_heads, max_blocks, part);
+    if (part == 0 && need > kScratchBytes) {
+        // automatic: the library's own choice as paged_decode_attention makes
+        // it - without the stage-balanced kernel when only its share does not
+        // fit (the automatic selection skips that kernel when the workspace
+        // is too small for it) - else partitions lengthened from the
+        // automatic length (less scratch) until the scratch fits; an unsplit
+        // pass needs none
+        need = pkv::decode_workspace_bytes_partitioned(pool, B, n_q_heads, max_blocks, 0);
+        if (need > kScratchBytes) {
+            const long long auto_p = pkv::decode_auto_partition(pool, B, n_q_heads, max_blocks);
+            for (long long p = 2 * auto_p; need > kScratchBytes && p <= (1 << 29); p *= 2) {
+                part = (int)p;
+                need = pkv::decode_workspace_bytes_partitioned(pool, B, n_q_heads, max_blocks,
+                                                               part);
+            }
         }
         if (need > kScratchBytes) {
             part = -1;
             need = 0;
         }
-    } else if (need > kScratchBytes) {
+    } else if (part != 0 && need > kScratchBytes) {
         return PKV_ERR_SCRATCH_LIMIT;
     }
     void* ws = nullptr;

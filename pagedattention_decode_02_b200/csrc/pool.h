@@ -36,4 +36,13 @@ struct pkv_pool {
 namespace pkv {
 // device-side extras set up after the buffers exist (tensor maps)
 void pool_init_device_extras(pkv_pool* p);
+// places the static decode scratch on `device` (the current device) and looks
+// up its address; false if that failed
+bool static_scratch_prepare(int device);
+// automatic partition length (tokens) for this batch shape, and the workspace
+// of the partitioned decode kernels for a partition request (0 = automatic),
+// not counting the stage-balanced kernel's
+int decode_auto_partition(const pkv_pool* pool, int B, int n_q_heads, int max_blocks);
+size_t decode_workspace_bytes_partitioned(const pkv_pool* pool, int B, int n_q_heads,
+                                          int max_blocks, int partition_tokens);
 }  // namespace pkv

@@ -20,6 +20,7 @@
 #include "decode_launch.h"
 #include "kernels_common.cuh"
 #include "pool.h"
+#include "trace.h"
 
 namespace pkv {
 namespace {
@@ -100,6 +101,7 @@ extern "C" {
 
 pkv_status kv_swap_out(pkv_pool* p, int64_t seq_id, void* h_k, void* h_v, size_t capacity_bytes,
                        int32_t* n_blocks_out, int64_t* n_tokens_out, void* stream) {
+    PKV_TRACE("kv_swap_out");
     if (!p || p->host_only || !h_k || !h_v) return PKV_ERR_INVALID_ARG;
     const pkv::Sequence* s = p->bm.find(seq_id);
     if (!s) return PKV_ERR_UNKNOWN_SEQ;
@@ -123,6 +125,7 @@ pkv_status kv_swap_out(pkv_pool* p, int64_t seq_id, void* h_k, void* h_v, size_t
 
 pkv_status kv_swap_in(pkv_pool* p, int64_t seq_id, const void* h_k, const void* h_v,
                       size_t capacity_bytes, int64_t n_tokens, void* stream) {
+    PKV_TRACE("kv_swap_in");
     if (!p || p->host_only || !h_k || !h_v || n_tokens < 0 || n_tokens > 0x7fffffff)
         return PKV_ERR_INVALID_ARG;
     const size_t block_bytes = (size_t)p->n_kv_heads * p->block_size * p->head_dim *
