@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--kernel", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-records", action="store_true",
+                    help="skip the Llama-2-70B GQA and FP8 records measured after the "
+                         "OPT-13B headline")
     ap.add_argument("--mode", choices=["decode", "prefill", "swap"], default="decode",
                     help="prefill: the prompt phase of the workload's batch (every history "
                          "attended causally as one prompt); swap: one sequence's blocks out to "
@@ -78,28 +81,28 @@ def config_of(args) -> wl.Config:
 
 # DRAM traffic of the decode kernel per launch, as a multiple of its
 # algorithmic KV bytes, from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum) of the same workload with one replica batch; the
-# summary and the command are under profiles/.  Valid only while the kernel's
-# sources hash to the recorded value, else the bench reports null.
+# dram__bytes_write.sum) of the same workload with one replica batch.  Valid
+# only while the kernel's sources hash to the recorded value, else the bench
+# reports null.
 TRAFFIC = {
     # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
-    # profiles/decode_tc_llama2_70b.md: 293.1 MB for 286.5 MB algorithmic
+    # 293.1 MB for 286.5 MB algorithmic
     ("llama2_70b", "decode_tc_kernel"):
         (1.0231, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # profiles/decode_tc_fp8_gqa.md: 149.0 MB for 143.3 MB
+    # 149.0 MB for 143.3 MB
     ("fp8_gqa", "decode_tc_kernel"):
         (1.0397, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # profiles/decode_tc_fp8.md: 1,358.7 MB for 1,343.5 MB
+    # 1,358.7 MB for 1,343.5 MB
     ("fp8", "decode_tc_kernel"):
         (1.0113, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # profiles/decode_simt2_opt13b.md: 612.2 MB for 604.1 MB
+    # 612.2 MB for 604.1 MB
     ("opt13b", "decode_simt2_kernel"):
         (1.0134, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
-    # profiles/decode_simt2_fp8.md: 1,358.7 MB for 1,343.5 MB
+    # 1,358.7 MB for 1,343.5 MB
     ("fp8", "decode_simt2_kernel"):
         (1.0113, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
-    # profiles/decode_lean_falcon7b.md: 2.98 MB for 8.31 MB (the samples of one
-    # prompt share its blocks; the re-reads within a launch hit L2)
+    # 2.98 MB for 8.31 MB (the samples of one prompt share its blocks; the
+    # re-reads within a launch hit L2)
     ("falcon7b", "decode_lean_kernel"):
         (0.3579, "b86acad210bccc586492a5dc87259763a1a6bc49bd327097f9d1f6005d917aba"),
 }
@@ -393,26 +396,27 @@ def build_batches(cfg: wl.Config, pk, torch, replicas: int, growth: int, seed: i
     return pool, groups, ctx
 
 
-def run_ours(args) -> None:
-    import torch
+def profile_stride(R: int) -> int:
+    """Every how many timed rounds one is profiled: the smallest stride >= 3
+    coprime with the number of replica batches, so that the profiled rounds
+    visit every batch in turn instead of a fixed subset."""
+    p = 3
+    while math.gcd(p, R) != 1:
+        p += 1
+    return p
 
-    import pagedattention_decode_02_b200 as pk
-    from pagedattention_decode_02_b200 import dist as pd
 
-    rank, world, local = pd.rank_world()
-    torch.cuda.set_device(local)
-    pd.init("nccl", timeout_s=120, device=torch.device("cuda", local))
-
-    cfg = config_of(args)
-    K, W = args.steps, args.warmup
-    E = args.e2e_steps or max(K // 3, 3)
-    R = args.replicas if args.replicas > 0 else auto_replicas(cfg)
+def measure_decode(cfg: wl.Config, pk, torch, pd, K: int, W: int, E: int, R: int,
+                   partition: int, kernel: int, rank: int, local: int) -> dict:
+    """One workload through the decode-step runtime: K timed rounds after R
+    priming and W warm-up rounds, then E end-to-end rounds through the
+    host-buffer call.  Returns this rank's raw measurements."""
     growth = -(-(R + K + W + E) // R) + 2
     pool, groups, ctx = build_batches(cfg, pk, torch, R, growth, seed=1000 * rank)
     B = cfg.batch
     max_ctx = max(int(c.max()) for c in ctx) + growth
     max_blocks = -(-max_ctx // cfg.block_size) + 2
-    step = pk.Step(pool, B, max_blocks, cfg.n_q_heads, cfg.q_dtype, args.partition, args.kernel,
+    step = pk.Step(pool, B, max_blocks, cfg.n_q_heads, cfg.q_dtype, partition, kernel,
                    max_seqs=B * R)
     dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[cfg.q_dtype]
     gen = torch.Generator(device="cuda")
@@ -449,7 +453,10 @@ def run_ours(args) -> None:
     torch.cuda.synchronize()
     pd.barrier()
 
-    prof_every = 4
+    # every prof_every-th timed round records CUDA events around its launches
+    # on the launch stream; prof_every is coprime with R, so the profiled
+    # rounds walk through all replica batches
+    prof_every = profile_stride(R)
     pk.pkv_step_profile(step, K, prof_every)
     clocks = ClockSampler(local)
     ev0 = torch.cuda.Event(enable_timing=True)
@@ -473,13 +480,15 @@ def run_ours(args) -> None:
     kernel_used = step.last_kernel
     pro_ms, dec_ms, merge_ms = pk.pkv_step_profile_read(step, K)
     pk.pkv_step_profile(step, 0)
-    prof_bytes = step_bytes[::prof_every][: len(dec_ms)]
+    prof_ks = list(range(0, K, prof_every))[: len(dec_ms)]
+    prof_bytes = [step_bytes[k] for k in prof_ks]
+    prof_batches = sorted({(R + W + k) % R for k in prof_ks})
 
     # end to end through the C ABI's host-buffer call (pkv_decode_step_host):
     # per round the new q/k/v come from pinned host memory and the output is
     # back in host memory when the call returns (a serving loop needs it
-    # before the next round)
-    # q | k | v packed in one pinned buffer: the call moves them in one copy
+    # before the next round); q | k | v packed in one pinned buffer, so the
+    # call moves them in one copy
     hqkv = torch.cat([t[0].flatten() for t in (q, kn, vn)]).cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=dt).pin_memory()
     esz = hqkv.element_size()
@@ -490,21 +499,22 @@ def run_ours(args) -> None:
     e1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e2e_bytes = 0
+    e2e_round_ms = []
     e0.record()
     for k in range(R + W + K, R + W + K + E):
         r = k % R
         ctx[r] += 1
+        t0 = time.perf_counter()
         step.run_host_raw(groups[r], hp[0], hp[1], hp[2], scale, hp[3], stream_ptr)
+        e2e_round_ms.append((time.perf_counter() - t0) * 1e3)
         e2e_bytes += int(ctx[r].sum()) * b_tok
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    h2d = hqkv.numel() * esz
-    d2h = hout.numel() * hout.element_size()
 
     bits = pk.pkv_device_error(pool)
     if bits:
-        raise SystemExit(f"device error bits {bits:#x}")
+        raise SystemExit(f"device error bits {bits:#x} on {cfg.name}")
     # KV memory actually storing tokens ("KV 缓存与分页注意力" §块表): slots
     # holding tokens over slots the blocks reserve, against reserving the
     # longest possible sequence up front (§先占好最长的位置)
@@ -517,18 +527,114 @@ def run_ours(args) -> None:
         "max_length_reservation": round(st["logical_tokens"] / max(1, n_seqs * max_len), 5),
         "max_length": int(max_len),
     }
+    res = {
+        "elapsed_ms": elapsed_ms, "tokens": tokens, "bytes": tokens * b_tok,
+        "launches": launches, "step_bytes": step_bytes,
+        "e2e_ms": e2e_ms, "e2e_bytes": e2e_bytes, "e2e_rounds": E,
+        "e2e_round_ms_median": float(statistics.median(e2e_round_ms)),
+        "h2d": hqkv.numel() * esz, "d2h": hout.numel() * hout.element_size(),
+        "kernel": pk.KERNEL_NAMES.get(kernel_used, "unknown"),
+        "prof_every": prof_every, "prof_bytes": [int(x) for x in prof_bytes],
+        "prof_batches": sorted(prof_batches),
+        "dec_ms": [float(x) for x in dec_ms], "merge_ms": [float(x) for x in merge_ms],
+        "pro_ms": [float(x) for x in pro_ms],
+        "utilisation": utilisation, "clocks": clocks.summary(), "R": R,
+        "pool_blocks": pool.num_blocks,
+    }
+    step.close()
+    pool.close()
+    del q, kn, vn, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def roofline_of(cfg: wl.Config, m: dict, peak: float, peak_kind: str) -> dict:
+    """The decode kernel against the HBM roofline, from the profiled rounds:
+    achieved = profiled_bytes / (profiled_launches x decode_ms_mean)."""
+    n = len(m["dec_ms"])
+    dec_total = float(np.sum(m["dec_ms"]))
+    pbytes = int(np.sum(m["prof_bytes"]))
+    achieved = pbytes / (dec_total / 1e3) / 1e9
+    return {
+        "bound": "hbm",
+        "kernel": m["kernel"],
+        "achieved": round(achieved, 2),
+        "peak": peak,
+        "peak_kind": peak_kind,
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": traffic_per_launch(cfg, m["kernel"], float(np.mean(m["step_bytes"]))),
+        "algorithmic_bytes_per_launch": int(np.mean(m["step_bytes"])),
+        "profiled_bytes": pbytes,
+        "profiled_launches": n,
+        "profiled_batches": m["prof_batches"],
+        "decode_ms_mean": round(dec_total / max(n, 1), 6),
+        "merge_ms_mean": round(float(np.mean(m["merge_ms"])), 6),
+        "prologue_ms_mean": round(float(np.mean(m["pro_ms"])), 6),
+        "profile_note": f"every {m['prof_every']}th timed round (a stride coprime with the "
+                        f"{m['R']} replica batches) records CUDA events on the launch stream "
+                        "around its kernels, which run without programmatic dependent launch "
+                        "in those rounds; achieved = profiled_bytes / profiled_launches / "
+                        "decode_ms_mean",
+    }
+
+
+def e2e_of(m: dict) -> dict:
+    return {
+        "value": round(m["e2e_bytes"] / (m["e2e_ms"] / 1e3) / 1e9, 2),
+        "unit": "GB/s",
+        "api": "pkv_decode_step_host (pinned host q/k/v in, output back in host memory)",
+        "h2d_bytes_per_step": int(m["h2d"]),
+        "d2h_bytes_per_step": int(m["d2h"]),
+        "steps": m["e2e_rounds"],
+        "ms_per_step": round(m["e2e_ms"] / m["e2e_rounds"], 5),
+        "host_ms_per_step_median": round(m["e2e_round_ms_median"], 5),
+    }
+
+
+# workloads measured after the headline in the same process (one GPU):
+# (record name, config, block size or 0 for the config's own)
+SUB_RECORDS = (("llama2_70b_gqa_bf16", "llama2_70b", 0),
+               ("fp8_bs16", "fp8", 16),
+               ("fp8_bs4", "fp8", 4))
+
+
+def run_ours(args) -> None:
+    import torch
+
+    import pagedattention_decode_02_b200 as pk
+    from pagedattention_decode_02_b200 import dist as pd
+
+    rank, world, local = pd.rank_world()
+    torch.cuda.set_device(local)
+    pd.init("nccl", timeout_s=120, device=torch.device("cuda", local))
+
+    cfg = config_of(args)
+    K, W = args.steps, args.warmup
+    E = args.e2e_steps or max(K // 3, 40)
+    R = args.replicas if args.replicas > 0 else auto_replicas(cfg)
+    m = measure_decode(cfg, pk, torch, pd, K, W, E, R, args.partition, args.kernel, rank, local)
+    tokens = m["tokens"]
 
     # time = max over ranks, work = sum over ranks (no data-path collective)
     (elapsed_ms, e2e_ms), (total_bytes, tokens_all, e2e_all, launches_all) = pd.reduce_run(
-        [elapsed_ms, e2e_ms], [tokens * b_tok, tokens, e2e_bytes, launches], device="cuda")
+        [m["elapsed_ms"], m["e2e_ms"]], [m["bytes"], tokens, m["e2e_bytes"], m["launches"]],
+        device="cuda")
+
+    subs = {}
+    if world == 1 and not args.no_sub_records and args.config == "opt13b" and not args.block_size:
+        Ks = max(K, 60)
+        for name, cname, bs in SUB_RECORDS:
+            c = wl.CONFIGS[cname]
+            if bs:
+                c = c.with_block_size(bs)
+            sm = measure_decode(c, pk, torch, pd, Ks, max(W, 3), max(Ks // 3, 40),
+                                auto_replicas(c), 0, 0, rank, local)
+            subs[name] = sm
 
     if rank == 0:
         value = total_bytes / (elapsed_ms / 1e3) / 1e9
         peak, peak_kind = peaks()
-        dec_total_ms = float(np.sum(dec_ms))
-        achieved = float(np.sum(prof_bytes)) / (dec_total_ms / 1e3) / 1e9
-        kernel_name = pk.KERNEL_NAMES.get(kernel_used, "unknown")
-        traffic = traffic_per_launch(cfg, kernel_name, float(np.mean(step_bytes)))
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -547,53 +653,52 @@ def run_ours(args) -> None:
                 "batch": cfg.batch, "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads,
                 "head_dim": cfg.head_dim, "block_size": cfg.block_size,
                 "mean_context": round(tokens / K / cfg.batch, 1),
-                "replica_batches_in_pool": R,
+                "replica_batches_in_pool": m["R"],
                 "priming": "one untimed round per replica batch before the warm-up (uploads "
                            "its block tables to the device)",
-                "pool_blocks": pool.num_blocks,
-                "l2": f"no flush: {R} replica batches cycled, {R * distinct_kv_bytes(cfg) / 1e6:.0f} MB "
-                      "of distinct KV between two reads of one batch (> 3 x 126 MB L2); attended "
-                      f"KV per step {np.mean(step_bytes) / 1e6:.0f} MB",
+                "pool_blocks": m["pool_blocks"],
+                "l2": f"no flush: {m['R']} replica batches cycled, "
+                      f"{m['R'] * distinct_kv_bytes(cfg) / 1e6:.0f} MB of distinct KV between "
+                      "two reads of one batch (> 3 x 126 MB L2); attended KV per step "
+                      f"{np.mean(m['step_bytes']) / 1e6:.0f} MB",
                 "parallelism": f"dp{world}",
             },
             "attended_tokens_per_s": round(tokens_all / (elapsed_ms / 1e3), 1),
             "seq_tokens_heads_per_s": round(tokens_all * cfg.n_q_heads / (elapsed_ms / 1e3), 1),
             "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS / world, 2),
-            "roofline": {
-                "bound": "hbm",
-                "kernel": kernel_name,
-                "achieved": round(achieved, 2),
-                "peak": peak,
-                "peak_kind": peak_kind,
-                "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "traffic": traffic,
-                "algorithmic_bytes_per_launch": int(np.mean(step_bytes)),
-                "decode_ms_mean": round(dec_total_ms / len(dec_ms), 5),
-                "merge_ms_mean": round(float(np.mean(merge_ms)), 5),
-                "prologue_ms_mean": round(float(np.mean(pro_ms)), 5),
-                "profiled_steps": int(len(dec_ms)),
-                "profile_note": f"every {prof_every}th timed step records events around its "
-                                "launches (those steps run without programmatic dependent launch)",
-            },
-            "e2e": {
-                "value": round(e2e_all / (e2e_ms / 1e3) / 1e9, 2),
-                "unit": "GB/s",
-                "api": "pkv_decode_step_host (pinned host q/k/v in, output back in host memory)",
-                "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h),
-                "steps": E,
-                "ms_per_step": round(e2e_ms / E, 5),
-            },
-            "kv_utilisation": utilisation,
+            "roofline": roofline_of(cfg, m, peak, peak_kind),
+            "e2e": dict(e2e_of(m), value=round(e2e_all / (e2e_ms / 1e3) / 1e9, 2),
+                        ms_per_step=round(e2e_ms / m["e2e_rounds"], 5)),
+            "kv_utilisation": m["utilisation"],
             "gpu_launches": int(launches_all),
-            "clocks": clocks.summary(),
+            "clocks": m["clocks"],
         }
+        if subs:
+            recs = {}
+            for name, sm in subs.items():
+                c = wl.CONFIGS[dict((n, cn) for n, cn, _ in SUB_RECORDS)[name]]
+                bs = dict((n, b) for n, _, b in SUB_RECORDS)[name]
+                if bs:
+                    c = c.with_block_size(bs)
+                v = sm["bytes"] / (sm["elapsed_ms"] / 1e3) / 1e9
+                recs[name] = {
+                    "workload": c.description + (f" (block size {bs})" if bs else ""),
+                    "value": round(v, 2), "unit": "GB/s",
+                    "steps": len(sm["step_bytes"]),
+                    "ms_per_step": round(sm["elapsed_ms"] / len(sm["step_bytes"]), 5),
+                    "pct_of_nominal_8tbs": round(100 * v / NOMINAL_HBM_GBS, 2),
+                    "attended_tokens_per_s": round(sm["tokens"] / (sm["elapsed_ms"] / 1e3), 1),
+                    "replica_batches_in_pool": sm["R"],
+                    "roofline": roofline_of(c, sm, peak, peak_kind),
+                    "e2e": e2e_of(sm),
+                    "kv_utilisation": sm["utilisation"],
+                    "gpu_launches": int(sm["launches"]),
+                    "clocks": sm["clocks"],
+                }
+            line["sub_records"] = recs
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_budget)
         print(json.dumps(line), flush=True)
-    step.close()
-    pool.close()
     pd.finish()
 
 
@@ -636,24 +741,31 @@ def run_prefill(args) -> None:
     flops = 4.0 * cfg.head_dim * cfg.n_q_heads * pairs
     kv_bytes = float(lens.sum()) * cfg.kv_bytes_per_token
 
-    def call():
+    def call(kernel=pk.PKV_PREFILL_AUTO):
         pk.paged_prefill_attention(pool, q, starts, t_tab, t_len, cfg.scale, max_q_len=max_q,
-                                   out=out)
+                                   out=out, kernel=kernel)
 
-    for _ in range(W):
-        call()
-    torch.cuda.synchronize()
+    def timed(kernel, sampler=None):
+        for _ in range(W):
+            call(kernel)
+        torch.cuda.synchronize()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        if sampler:
+            sampler.start()
+        ev0.record()
+        for _ in range(K):
+            call(kernel)
+        ev1.record()
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.stop()
+        return ev0.elapsed_time(ev1) / K
+
+    # the warp-level mma.sync kernel, timed first as the baseline
+    ms_legacy = timed(pk.PKV_PREFILL_MMA_SYNC)
     clocks = ClockSampler(0)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    clocks.start()
-    ev0.record()
-    for _ in range(K):
-        call()
-    ev1.record()
-    torch.cuda.synchronize()
-    clocks.stop()
-    ms = ev0.elapsed_time(ev1) / K
+    ms = timed(pk.PKV_PREFILL_AUTO, clocks)
     # end to end: the prompt's queries from pinned host memory, the output back
     hq = q.cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=dt).pin_memory()
@@ -694,8 +806,14 @@ def run_prefill(args) -> None:
                          "by its row tiles from L2"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": None, "kernel": "prefill_tc_kernel",
-                     "flops_per_launch": flops, "note": "mma.sync m16n8k16 tensor path"},
+                     "traffic": None, "kernel": "prefill_tc05_kernel",
+                     "flops_per_launch": flops,
+                     "note": "tcgen05.mma (M 128) with tensor-memory accumulators; FLOPs count "
+                             "4 d per unmasked (query, key) pair and query head"},
+        "baseline_mma_sync": {"kernel": "prefill_tc_kernel", "ms_per_step": round(ms_legacy, 5),
+                              "value": round(flops / (ms_legacy / 1e3) / 1e12, 2),
+                              "unit": "TFLOP/s",
+                              "frac": round(flops / (ms_legacy / 1e3) / 1e12 / peak, 4)},
         "e2e": {"value": round(flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(hq.numel() * hq.element_size()),
                 "d2h_bytes_per_step": int(hout.numel() * hout.element_size()),

@@ -495,13 +495,32 @@ pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dt
  *   grid).  n_i == 0 writes nothing.  A length outside [1, max_blocks * bs],
  *   n_i > c_i or n_i > max_q_len sets PKV_DEVERR_CONTEXT_LEN (that sequence's
  *   rows are zero where the grid covers them); a block id outside
- *   [0, num_blocks) sets PKV_DEVERR_BLOCK_ID and zeroes the affected 64-row
- *   tile.  No workspace.  Errors: INVALID_ARG, CUDA. */
+ *   [0, num_blocks) sets PKV_DEVERR_BLOCK_ID and zeroes the affected work
+ *   item's rows (128 rows with the tcgen05 kernel, 64 with mma.sync).  No
+ *   workspace.  Runs the tcgen05 kernel (see paged_prefill_attention_ex).
+ *   Errors: INVALID_ARG, CUDA. */
 pkv_status paged_prefill_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
                                    const int32_t* d_q_starts, int max_q_len,
                                    const int32_t* d_block_tables, int max_blocks,
                                    const int32_t* d_context_lens, int B, int n_q_heads,
                                    float scale, void* d_out, void* stream);
+
+/* Kernel selection for paged_prefill_attention_ex. */
+#define PKV_PREFILL_AUTO 0         /* PKV_PREFILL_TCGEN05 */
+#define PKV_PREFILL_TCGEN05 1      /* fifth-generation tensor cores: 128 query rows per work item,
+                                      S = Q K^T and O += P V by tcgen05.mma into tensor memory, one
+                                      persistent CTA per SM taking the heaviest items first */
+#define PKV_PREFILL_MMA_SYNC 2     /* warp-level mma.sync m16n8k16, register accumulators, one CTA
+                                      per 64 query rows */
+
+/* paged_prefill_attention_ex - paged_prefill_attention with an explicit kernel
+ *   (PKV_PREFILL_*); same arguments, results and errors.  Both kernels compute
+ *   the same attention. */
+pkv_status paged_prefill_attention_ex(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
+                                      const int32_t* d_q_starts, int max_q_len,
+                                      const int32_t* d_block_tables, int max_blocks,
+                                      const int32_t* d_context_lens, int B, int n_q_heads,
+                                      float scale, void* d_out, int kernel, void* stream);
 
 /* paged_decode_static_scratch_bytes - size of the static scratch array. */
 size_t paged_decode_static_scratch_bytes(void);
@@ -557,6 +576,26 @@ typedef struct {
 pkv_status pkv_simulate(const pkv_sim_request* requests, int n, int num_slots, int block_size,
                         int max_len, int max_rounds, pkv_sim_result* out,
                         int32_t* running_per_round);
+
+/* pkv_set_wait_budget - how long a kernel launched on this pool waits for
+ *   one copy (or one tensor-core result) in its main loop before it gives up:
+ *   it then sets PKV_DEVERR_TIMEOUT, stops issuing work, waits with the
+ *   default budget for its copies and tensor-core operations still in flight,
+ *   frees what it holds and returns (the affected outputs are zero or stale).
+ *   budget_ns: 1 .. 2e9 ns; 0 restores the default of 2 s, long enough that
+ *   only a wait that would otherwise never end gives up.  A short budget
+ *   makes waits give up while their copies are still on the way: it exists
+ *   to exercise that path.  The library has no counterpart in the pages: it
+ *   is this implementation's failure handling.  Errors: INVALID_ARG. */
+pkv_status pkv_set_wait_budget(pkv_pool* pool, uint64_t budget_ns);
+
+/* pkv_wait_probe - queues one small kernel on `stream` that waits, with the
+ *   pool's wait budget, on a barrier that nothing ever completes, and sets
+ *   PKV_DEVERR_TIMEOUT when that wait gives up (read it with
+ *   pkv_device_error): a check that the bounded wait and its error report
+ *   work on this device.  Takes about the budget to run.  Errors:
+ *   INVALID_ARG, CUDA. */
+pkv_status pkv_wait_probe(pkv_pool* pool, void* stream);
 
 /* pkv_device_error - synchronises the stream, returns the device error word's
  *   bits in *bits_out (may be NULL) and clears it.  Returns PKV_ERR_DEVICE if

@@ -37,6 +37,7 @@ PKV_DEVERR_CONTEXT_LEN, PKV_DEVERR_BLOCK_ID, PKV_DEVERR_SLOT, PKV_DEVERR_TIMEOUT
 PKV_POOL_HOST_ONLY = 0x1
 PKV_KERNEL_AUTO, PKV_KERNEL_SIMT, PKV_KERNEL_TENSOR, PKV_KERNEL_SIMT_BULK, PKV_KERNEL_SIMT_TMA = 0, 1, 2, 3, 4
 PKV_KERNEL_LEAN = 5
+PKV_PREFILL_AUTO, PKV_PREFILL_TCGEN05, PKV_PREFILL_MMA_SYNC = 0, 1, 2
 
 DTYPE_NAMES = {"f32": PKV_F32, "f16": PKV_F16, "bf16": PKV_BF16, "fp8": PKV_FP8_E4M3}
 ELEM_BYTES = {PKV_F32: 4, PKV_F16: 2, PKV_BF16: 2, PKV_FP8_E4M3: 1}
@@ -123,7 +124,11 @@ _sig("paged_decode_workspace_bytes_ex", ctypes.c_size_t, _P, ctypes.c_int, ctype
 _sig("pkv_device_error", _st, _P, _P, ctypes.POINTER(ctypes.c_uint32))
 _sig("paged_prefill_attention", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int, _P,
      ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, _P)
+_sig("paged_prefill_attention_ex", _st, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, ctypes.c_int, _P,
+     ctypes.c_int, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P)
 _sig("pkv_status_str", ctypes.c_char_p, ctypes.c_int)
+_sig("pkv_set_wait_budget", _st, _P, ctypes.c_uint64)
+_sig("pkv_wait_probe", _st, _P, _P)
 _sig("pkv_step_create", _st, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
      ctypes.c_int, ctypes.c_int, ctypes.POINTER(_P))
 _sig("pkv_step_destroy", None, _P)
@@ -149,7 +154,8 @@ EXPORTED = [
     "pkv_decode_step_host",
     "pkv_step_last_launches", "pkv_step_last_kernel", "pkv_step_profile", "pkv_step_profile_read",
     "paged_decode_attention_static", "paged_decode_static_scratch_bytes", "kv_swap_out", "kv_swap_in",
-    "paged_prefill_attention",
+    "paged_prefill_attention", "paged_prefill_attention_ex",
+    "pkv_set_wait_budget", "pkv_wait_probe",
     "bt_set_prefix_caching", "bt_alloc_prefix", "pkv_simulate",
 ]
 
@@ -436,11 +442,13 @@ def paged_decode_attention(pool: Pool, q, block_tables, context_lens, scale: flo
 
 
 def paged_prefill_attention(pool: Pool, q, q_starts, block_tables, context_lens, scale: float,
-                            max_q_len: Optional[int] = None, out=None, stream=None):
+                            max_q_len: Optional[int] = None, out=None, stream=None,
+                            kernel: int = 0):
     """Prompt-phase attention.  q: CUDA [rows][H_q][d]; q_starts: int32 CUDA [B+1]
     (row offsets per sequence); block_tables: int32 CUDA [B][max_blocks];
     context_lens: int32 CUDA [B] (cached tokens, the prompt's included).
-    max_q_len: the longest prompt (read from q_starts when None).  Returns out."""
+    max_q_len: the longest prompt (read from q_starts when None); kernel:
+    PKV_PREFILL_* (0 = automatic).  Returns out."""
     import torch
     B = int(context_lens.shape[0])
     H_q = int(q.shape[1])
@@ -448,11 +456,22 @@ def paged_prefill_attention(pool: Pool, q, q_starts, block_tables, context_lens,
         out = torch.empty_like(q)
     if max_q_len is None:
         max_q_len = int((q_starts[1:] - q_starts[:-1]).max().item()) if B else 0
-    _check(_lib.paged_prefill_attention(
+    _check(_lib.paged_prefill_attention_ex(
         pool.handle, _dev_ptr(q), torch_dtype_code(q.dtype), _dev_ptr(q_starts), int(max_q_len),
         _dev_ptr(block_tables), int(block_tables.shape[1]), _dev_ptr(context_lens), B, H_q,
-        float(scale), _dev_ptr(out), _stream_ptr(stream)), "paged_prefill_attention")
+        float(scale), _dev_ptr(out), int(kernel), _stream_ptr(stream)),
+        "paged_prefill_attention")
     return out
+
+
+def pkv_set_wait_budget(pool: Pool, budget_ns: int) -> None:
+    """Budget of the pool's kernels' main-loop waits in ns (0 = the default 2 s)."""
+    _check(_lib.pkv_set_wait_budget(pool.handle, int(budget_ns)), "pkv_set_wait_budget")
+
+
+def pkv_wait_probe(pool: Pool, stream=None) -> None:
+    """Queue the probe kernel: a wait that nothing completes, with the pool's budget."""
+    _check(_lib.pkv_wait_probe(pool.handle, _stream_ptr(stream)), "pkv_wait_probe")
 
 
 def pkv_device_error(pool: Pool, stream=None) -> int:

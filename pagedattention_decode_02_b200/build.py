@@ -31,6 +31,7 @@ SOURCES = [
     "decode_simt2.cu",
     "decode_lean.cu",
     "prefill.cu",
+    "prefill_tc05.cu",
     "decode_tc.cu",
     "api.cu",
     "no_alloc.cu",

@@ -444,6 +444,7 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     dp.v_scale = p->v_scale;
     dp.head_stride = (long long)p->block_size * p->head_dim * elem_bytes(p->dtype);
     dp.block_stride = dp.head_stride * p->n_kv_heads;
+    dp.wait_ns = p->wait_ns;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = ev_begin ? cudaEventRecord(ev_begin, st) : cudaSuccess;
@@ -491,12 +492,14 @@ pkv_status paged_decode_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                      out, ws, ws_bytes, 0, PKV_KERNEL_AUTO, stream);
 }
 
-pkv_status paged_prefill_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
-                                   const int32_t* q_starts, int max_q_len, const int32_t* tables,
-                                   int max_blocks, const int32_t* lens, int B, int n_q_heads,
-                                   float scale, void* out, void* stream) {
-    PKV_TRACE("paged_prefill_attention");
+pkv_status paged_prefill_attention_ex(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                      const int32_t* q_starts, int max_q_len,
+                                      const int32_t* tables, int max_blocks, const int32_t* lens,
+                                      int B, int n_q_heads, float scale, void* out, int kernel,
+                                      void* stream) {
+    PKV_TRACE("paged_prefill_attention_ex");
     if (!p || p->host_only || B < 0 || max_q_len < 0) return PKV_ERR_INVALID_ARG;
+    if (kernel < PKV_PREFILL_AUTO || kernel > PKV_PREFILL_MMA_SYNC) return PKV_ERR_INVALID_ARG;
     if (B == 0 || max_q_len == 0) return PKV_OK;
     if (!q || !out || !q_starts || !tables || !lens || max_blocks < 1) return PKV_ERR_INVALID_ARG;
     if (n_q_heads < p->n_kv_heads || n_q_heads % p->n_kv_heads) return PKV_ERR_INVALID_ARG;
@@ -521,7 +524,32 @@ pkv_status paged_prefill_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype
     pp.num_blocks = p->num_blocks;
     pp.max_q_len = max_q_len;
     pp.q_scale = scale * 1.4426950408889634f;
-    return pkv::launch_prefill(pp, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    pp.wait_ns = p->wait_ns;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = kernel == PKV_PREFILL_MMA_SYNC ? pkv::launch_prefill(pp, p, st)
+                                                         : pkv::launch_prefill_tc05(pp, p, st);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status paged_prefill_attention(pkv_pool* p, const void* q, pkv_dtype q_dtype,
+                                   const int32_t* q_starts, int max_q_len, const int32_t* tables,
+                                   int max_blocks, const int32_t* lens, int B, int n_q_heads,
+                                   float scale, void* out, void* stream) {
+    return paged_prefill_attention_ex(p, q, q_dtype, q_starts, max_q_len, tables, max_blocks, lens,
+                                      B, n_q_heads, scale, out, PKV_PREFILL_AUTO, stream);
+}
+
+pkv_status pkv_set_wait_budget(pkv_pool* p, uint64_t budget_ns) {
+    if (!p || budget_ns > pkv::kWaitBudgetNs) return PKV_ERR_INVALID_ARG;
+    p->wait_ns = budget_ns == 0 ? pkv::kWaitBudgetNs : budget_ns;
+    return PKV_OK;
+}
+
+pkv_status pkv_wait_probe(pkv_pool* p, void* stream) {
+    PKV_TRACE("pkv_wait_probe");
+    if (!p || p->host_only || !same_device(p)) return PKV_ERR_INVALID_ARG;
+    return pkv::launch_wait_probe(p->d_err, p->wait_ns, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
                ? PKV_OK
                : PKV_ERR_CUDA;
 }

@@ -356,4 +356,24 @@ cudaError_t launch_scatter_rows(const int32_t* staged, const int32_t* rows, int 
     return cudaGetLastError();
 }
 
+namespace {
+// One thread waits, with the given budget, on a barrier phase that nothing
+// completes (no arrival, no copy), the same bounded wait the decode and
+// prompt kernels use; when it gives up it reports PKV_DEVERR_TIMEOUT.
+__global__ void wait_probe_kernel(uint32_t* err, unsigned long long budget_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, budget_ns)) report_error(err, PKV_DEVERR_TIMEOUT);
+}
+}  // namespace
+
+cudaError_t launch_wait_probe(uint32_t* err, unsigned long long budget_ns, cudaStream_t st) {
+    wait_probe_kernel<<<1, 32, 0, st>>>(err, budget_ns);
+    return cudaGetLastError();
+}
+
 }  // namespace pkv

@@ -62,9 +62,13 @@ struct PrefillParams {
     int max_blocks, block_size, num_blocks;
     int max_q_len;             // >= every n_i (sizes the grid)
     float q_scale;             // scale * log2(e)
+    unsigned long long wait_ns;// budget of the main loops' waits (the pool's)
 };
 bool prefill_supported(const pkv_pool* pool, int q_dtype);
+// the mma.sync kernel (m16n8k16, register accumulators)
 cudaError_t launch_prefill(const PrefillParams& p, const pkv_pool* pool, cudaStream_t st);
+// the tcgen05 kernel (tensor-memory accumulators, persistent heaviest-first schedule)
+cudaError_t launch_prefill_tc05(const PrefillParams& p, const pkv_pool* pool, cudaStream_t st);
 
 // One decode round's small host-side results, passed by value as kernel
 // parameters (no separate host-to-device copy):
@@ -100,6 +104,10 @@ cudaError_t launch_kv_append(uint8_t* k_pool, uint8_t* v_pool, const int32_t* sl
                              const void* k, const void* v, int in_dtype, int kv_dtype,
                              int n_kv_heads, int head_dim, int block_size, int num_blocks,
                              float k_scale, float v_scale, uint32_t* err, cudaStream_t st);
+
+// One CTA waiting, with budget_ns, on a barrier that nothing completes; sets
+// PKV_DEVERR_TIMEOUT in *err when the wait gives up.
+cudaError_t launch_wait_probe(uint32_t* err, unsigned long long budget_ns, cudaStream_t st);
 
 // Whole-block copies src[i] -> dst[i] of K and V.
 cudaError_t launch_block_copy(uint8_t* k_pool, uint8_t* v_pool, const int32_t* src,

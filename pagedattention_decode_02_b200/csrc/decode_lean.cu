@@ -412,7 +412,7 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int slot = it % RG;
             const uint32_t par = (uint32_t)((it / RG) & 1);
             if (!abort) {
-                const bool ok = mbar_wait(&full[slot], par);
+                const bool ok = mbar_wait(&full[slot], par, p.wait_ns);
                 if (!__all_sync(kFull, ok)) {
                     abort = true;
                     if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -432,7 +432,7 @@ decode_lean_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (issuer && it + RG < n_stages) {
                 bool ok = !abort;
-                if constexpr (MT > 1) ok = ok && mbar_wait(&empty[slot], par);
+                if constexpr (MT > 1) ok = ok && mbar_wait(&empty[slot], par, p.wait_ns);
                 if (__all_sync(kFull, ok)) {
                     issue_stage<D>(is, hi, sc, p, &tmap_k, &tmap_v, ring + slot * SLOT, &full[slot],
                                    &slot_n[slot], policy, lane);

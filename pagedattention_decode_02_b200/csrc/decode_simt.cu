@@ -242,7 +242,7 @@ decode_simt_kernel(const DecodeParams p, int table_entries) {
     bool timed_out = false;
     for (; k < my_n; ++k) {
         const int slot = k % kStages;
-        if (!mbar_wait(&my_bars[slot], (uint32_t)((k / kStages) & 1))) {
+        if (!mbar_wait(&my_bars[slot], (uint32_t)((k / kStages) & 1), p.wait_ns)) {
             timed_out = true;
             break;
         }

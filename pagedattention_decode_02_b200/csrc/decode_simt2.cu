@@ -251,7 +251,7 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
     bool timed_out = false;
     for (; k < my_n; ++k) {
         const int slot = k % S;
-        if (!mbar_wait(&my_bars[slot], (uint32_t)((k / S) & 1))) {
+        if (!mbar_wait(&my_bars[slot], (uint32_t)((k / S) & 1), p.wait_ns)) {
             timed_out = true;
             break;
         }

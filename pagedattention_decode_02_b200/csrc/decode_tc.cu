@@ -212,7 +212,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     bool timed_out = false;
     for (; k < my_n; ++k) {
         const int slot = k % kStages;
-        if (!mbar_wait(&my_full[slot], (uint32_t)((k / kStages) & 1))) {
+        if (!mbar_wait(&my_full[slot], (uint32_t)((k / kStages) & 1), p.wait_ns)) {
             timed_out = true;
             break;
         }
@@ -230,7 +230,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (producer && k + kStages < my_n) {
                 if constexpr (MT > 1) {
-                    if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1))) return false;
+                    if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1), p.wait_ns)) return false;
                 }
                 issue(k + kStages, slot);
             }

@@ -193,18 +193,37 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// non-blocking test of the phase with the given parity
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the barrier phase with the given parity.  Gives up after
-// kWaitBudgetNs of wall-clock time and returns false.  A healthy copy of a
-// few KB completes in microseconds; the budget only ends a wait that would
-// otherwise never end.
+// budget_ns of wall-clock time and returns false.  A healthy copy of a few KB
+// completes in microseconds; the default budget only ends a wait that would
+// otherwise never end.  Kernels pass their pool's budget (pkv_set_wait_budget)
+// for the waits of their main loops, and keep the default for the waits that
+// make sure no copy is still in flight when they give up.  With a shortened
+// budget the first probe does not block, so that the wait can give up while
+// the copy is still on its way.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t budget_ns = kWaitBudgetNs) {
+    if (budget_ns >= kWaitBudgetNs ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity))
+        return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitBudgetNs) return false;
+        if (global_timer_ns() - t0 > budget_ns) return false;
     }
 }
 
@@ -269,6 +288,7 @@ struct DecodeParams {
     float v_scale;    // FP8 V dequantisation (1 otherwise)
     long long head_stride;   // bytes of one (block, kv head) tile: bs * D * elem
     long long block_stride;  // bytes of one block: H_kv * head_stride
+    unsigned long long wait_ns;  // budget of the main loops' waits (the pool's)
 };
 
 }  // namespace pkv

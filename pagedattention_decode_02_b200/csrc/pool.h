@@ -25,6 +25,8 @@ struct pkv_pool {
     uint8_t* v = nullptr;
     size_t bytes = 0;       // bytes of one of the two buffers
     uint32_t* d_err = nullptr;
+    // budget of the kernels' main-loop waits on a copy (pkv_set_wait_budget)
+    unsigned long long wait_ns = 2000000000ull;
     pkv::BlockManager bm;
     // TMA descriptors of the K and V pools (CUtensorMap, 128 bytes each) for
     // the tensor-core decode path; valid when has_tmaps.

@@ -122,7 +122,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (; kt < n_kt; ++kt) {
             const int b = kt % kBufs;
             if (kt >= kBufs) {
-                const bool ok = mbar_wait(&empty[b], (uint32_t)(((kt / kBufs) - 1) & 1));
+                const bool ok = mbar_wait(&empty[b], (uint32_t)(((kt / kBufs) - 1) & 1), p.wait_ns);
                 if (!__all_sync(kFull, ok)) {
                     if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
                     break;
@@ -236,7 +236,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int kt = 0; kt < n_kt; ++kt) {
         const int b = kt % kBufs;
         if (!abort) {
-            const bool ok = mbar_wait(&full[b], (uint32_t)((kt / kBufs) & 1));
+            const bool ok = mbar_wait(&full[b], (uint32_t)((kt / kBufs) & 1), p.wait_ns);
             if (!__all_sync(kFull, ok)) {
                 abort = true;
                 if (lane == 0) report_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -340,7 +340,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
         }
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&empty[b]);
+        // a warp that gave up hands no buffer back: its copy may still be in
+        // flight, so the producer must not refill it (the producer's own wait
+        // for the buffer then gives up too, and it waits for its last copies)
+        if (lane == 0 && !abort) tc::mbar_arrive(&empty[b]);
     }
 
 #pragma unroll

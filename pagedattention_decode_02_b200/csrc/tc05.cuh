@@ -1,0 +1,135 @@
+// Fifth-generation tensor-core building blocks (sm_100a): tensor-memory
+// allocation, the tcgen05.mma instruction for f16/bf16 inputs with fp32
+// accumulation, its commit to an mbarrier, tensor-memory loads and stores, and
+// the shared-memory matrix descriptors of 128-byte swizzled tiles.
+//
+// Shared-memory tiles used with these descriptors are 1024-byte aligned and
+// stored as 128-byte rows whose 16-byte chunks are XOR-swizzled by (row % 8),
+// i.e. the layout a 128-byte-swizzled TMA box writes:
+//   K-major operand (rows = M or N, the contraction dimension K contiguous):
+//     rows 128 B apart, groups of 8 rows 1024 B apart (stride byte offset);
+//     a 16-element K step inside the 64-element row advances the start
+//     address by 32 B; the next 64 elements of K live in another region.
+//   MN-major operand (the M/N dimension contiguous, K strided):
+//     64 elements of N per 128-byte row, one row per K index, 8 K rows per
+//     1024 B (stride byte offset), further 64-element N blocks a leading byte
+//     offset apart; a 16-element K step advances the start address by 2 KB.
+#pragma once
+
+#include <stdint.h>
+
+#include "kernels_common.cuh"
+
+namespace pkv {
+namespace tc05 {
+
+// ---------------------------------------------------------------------------
+// tensor memory
+// ---------------------------------------------------------------------------
+// Allocate ncols columns (a power of two >= 32) of this CTA's tensor memory;
+// the base address is written to *dst (shared memory).  Whole warp.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+// Whole warp (the one that allocated).
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+// Order tensor-core operations around a thread synchronisation (barrier or
+// mbarrier): "before" on the signalling side, "after" on the waiting side.
+__device__ __forceinline__ void fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane (lane = 32 * (warp % 4)
+// + lane id, encoded in taddr's upper half), loaded and waited for in one
+// statement so that no use of r can be scheduled before the data arrived.
+#define PKV_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                  "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : PKV_R8(0), PKV_R8(8), PKV_R8(16), PKV_R8(24)
+        : "r"(taddr)
+        : "memory");
+}
+#undef PKV_R8
+
+#define PKV_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
+                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+// Store 32 columns of this thread's lane and wait until the store is done.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        PKV_W8(0), PKV_W8(8), PKV_W8(16), PKV_W8(24)
+        : "memory");
+}
+#undef PKV_W8
+
+// ---------------------------------------------------------------------------
+// matrix multiply-accumulate
+// ---------------------------------------------------------------------------
+// Instruction descriptor of kind::f16 with fp32 accumulation: A and B both
+// f16 (bf16 = false) or both bf16; K-major A; B K-major or MN-major; M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major, int M, int N) {
+    return (1u << 4)                               // D format: fp32
+           | ((bf16 ? 1u : 0u) << 7)               // A format
+           | ((bf16 ? 1u : 0u) << 10)              // B format
+           | ((b_mn_major ? 1u : 0u) << 16)        // B major
+           | ((uint32_t)(N >> 3) << 17)            // N / 8
+           | ((uint32_t)(M >> 4) << 24);           // M / 16
+}
+
+// Shared-memory matrix descriptor: start address, leading and stride byte
+// offsets (bytes, multiples of 16), descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one instruction (K = 16); issued by one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tensor-core operation this thread issued
+// so far has completed.
+__device__ __forceinline__ void commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+// 2^x on the special-function unit (approximate, subnormal results flushed to
+// zero; 2^-inf = +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+}  // namespace tc05
+}  // namespace pkv

@@ -1,7 +1,9 @@
 """GPU parity of the prompt-phase attention over the paged cache against the
 CPU oracle: prompts with and without a cached prefix, grouped heads, block
-sizes, ragged prompt lengths spanning several 64-row tiles, prompts admitted
-through the prefix cache, and invalid inputs."""
+sizes, ragged prompt lengths spanning several row tiles and key tiles, prompts
+admitted through the prefix cache, and invalid inputs - for both kernels (the
+tcgen05 kernel with tensor-memory accumulators, which the library runs by
+default, and the mma.sync kernel)."""
 
 import dataclasses
 
@@ -21,7 +23,10 @@ def small(base: str, **kw) -> wl.Config:
     return dataclasses.replace(wl.CONFIGS[base], **kw)
 
 
-def run_prefill(side, prompt_lens, seed=0):
+KERNELS = [pk.PKV_PREFILL_TCGEN05, pk.PKV_PREFILL_MMA_SYNC]
+
+
+def run_prefill(side, prompt_lens, seed=0, kernel=0):
     """Prefill the last n_i tokens of every admitted sequence; -> (gpu, ref)
     lists of float64 [n_i][H_q][d]."""
     cfg = side.cfg
@@ -36,7 +41,7 @@ def run_prefill(side, prompt_lens, seed=0):
     out = pk.paged_prefill_attention(side.pool, to_torch(q_all, cfg.q_dtype),
                                      torch.from_numpy(starts).cuda(),
                                      torch.from_numpy(tables).cuda(),
-                                     torch.from_numpy(lens).cuda(), cfg.scale)
+                                     torch.from_numpy(lens).cuda(), cfg.scale, kernel=kernel)
     torch.cuda.synchronize()
     assert pk.pkv_device_error(side.pool) == 0
     gpu = to_f64(from_torch(out, cfg.q_dtype), cfg.q_dtype)
@@ -55,8 +60,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("dt,d,bs,hq,hkv", CASES)
-def test_prefill_small(dt, d, bs, hq, hkv):
+def test_prefill_small(dt, d, bs, hq, hkv, kernel):
     cfg = small("llama2_70b", n_q_heads=hq, n_kv_heads=hkv, head_dim=d, kv_dtype=dt, q_dtype=dt,
                 block_size=bs, batch=4, lengths=("uniform", 1, 200))
     side = setup_config(cfg, seed=d + bs + hq)
@@ -64,36 +70,39 @@ def test_prefill_small(dt, d, bs, hq, hkv):
     rng = np.random.default_rng(bs + hq)
     # prompts from a single token to the whole history (no prefix)
     n = [int(h) if i == 0 else int(rng.integers(1, h + 1)) for i, h in enumerate(hist)]
-    gpu, ref = run_prefill(side, n)
+    gpu, ref = run_prefill(side, n, kernel=kernel)
     for g, r in zip(gpu, ref):
         compare_out(g, r, dt)
 
 
-@pytest.mark.parametrize("hq,hkv,d", [(64, 8, 128), (71, 1, 64), (40, 40, 128)])
-def test_prefill_long_prompts(hq, hkv, d):
-    # several 64-row tiles per (sequence, KV head) and several 64-key tiles
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("hq,hkv,d", [(64, 8, 128), (71, 1, 64), (40, 40, 128), (8, 2, 64)])
+def test_prefill_long_prompts(hq, hkv, d, kernel):
+    # several row tiles per (sequence, KV head) and several key tiles
     dt = "bf16" if d == 128 else "f16"
     cfg = small("llama2_70b", n_q_heads=hq, n_kv_heads=hkv, head_dim=d, kv_dtype=dt, q_dtype=dt,
                 block_size=16, batch=3, lengths=("uniform", 300, 700))
     side = setup_config(cfg, seed=hq)
     hist = [side.orc.bm.lengths[s] for s in side.seqs]
     n = [hist[0], hist[1] // 2, 37]
-    gpu, ref = run_prefill(side, n)
+    gpu, ref = run_prefill(side, n, kernel=kernel)
     for g, r in zip(gpu, ref):
         compare_out(g, r, dt)
 
 
-def test_prefill_zero_length_prompt_writes_nothing():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_zero_length_prompt_writes_nothing(kernel):
     cfg = small("llama2_70b", n_q_heads=4, n_kv_heads=2, head_dim=64, kv_dtype="f16",
                 q_dtype="f16", block_size=16, batch=3, lengths=("uniform", 5, 40))
     side = setup_config(cfg, seed=1)
-    gpu, ref = run_prefill(side, [3, 0, 5])
+    gpu, ref = run_prefill(side, [3, 0, 5], kernel=kernel)
     assert gpu[1].shape[0] == 0
     compare_out(gpu[0], ref[0], "f16")
     compare_out(gpu[2], ref[2], "f16")
 
 
-def test_prefill_after_prefix_cache_hit():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_after_prefix_cache_hit(kernel):
     # the second prompt shares its first two blocks with the first; only its
     # tail is prefilled, attending to the shared cached blocks
     cfg = small("llama2_70b", n_q_heads=8, n_kv_heads=2, head_dim=128, kv_dtype="bf16",
@@ -118,7 +127,7 @@ def test_prefill_after_prefix_cache_hit():
     out = pk.paged_prefill_attention(pool, to_torch(q, "bf16"),
                                      torch.tensor([0, 3], dtype=torch.int32, device="cuda"),
                                      torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(),
-                                     cfg.scale)
+                                     cfg.scale, kernel=kernel)
     torch.cuda.synchronize()
     from oracle.attention import prefill_attention
     kh = np.concatenate([to_f64(k[:32], "bf16"), to_f64(kb, "bf16")])
@@ -127,19 +136,21 @@ def test_prefill_after_prefix_cache_hit():
     compare_out(to_f64(from_torch(out, "bf16"), "bf16"), ref, "bf16")
 
 
-def test_prefill_invalid_inputs():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_invalid_inputs(kernel):
     pool = pk.kv_pool_create(8, 16, 2, 64, "f16")
     q = torch.randn(6, 4, 64, device="cuda", dtype=torch.float16)
     tables = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device="cuda")
     starts = torch.tensor([0, 3, 6], dtype=torch.int32, device="cuda")
     lens = torch.tensor([2, 20], dtype=torch.int32, device="cuda")        # 3 prompt rows > 2 cached
-    out = pk.paged_prefill_attention(pool, q, starts, tables, lens, 0.1)
+    out = pk.paged_prefill_attention(pool, q, starts, tables, lens, 0.1, kernel=kernel)
     assert pk.pkv_device_error(pool) & pk.PKV_DEVERR_CONTEXT_LEN
     assert torch.all(out[:3] == 0)
     tables = torch.tensor([[0, 1], [2, 77]], dtype=torch.int32, device="cuda")
     lens = torch.tensor([3, 20], dtype=torch.int32, device="cuda")
-    pk.paged_prefill_attention(pool, q, starts, tables, lens, 0.1)
+    out = pk.paged_prefill_attention(pool, q, starts, tables, lens, 0.1, kernel=kernel)
     assert pk.pkv_device_error(pool) & pk.PKV_DEVERR_BLOCK_ID
+    assert torch.all(out[3:] == 0)
     with pytest.raises(pk.PagedKVError):                                 # f32 pool
         p32 = pk.kv_pool_create(8, 16, 2, 64, "f32")
         pk.paged_prefill_attention(p32, q.float(), starts, tables, lens, 0.1)

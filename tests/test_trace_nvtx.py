@@ -82,7 +82,7 @@ def test_device_calls_open_named_ranges(tmp_path):
     lines = log.read_text().splitlines()
     pushed = [ln[5:] for ln in lines if ln.startswith("push ")]
     for want in ("kv_append", "block_copy", "paged_decode_attention_ex",
-                 "paged_decode_attention_static", "paged_prefill_attention", "kv_swap_out",
+                 "paged_decode_attention_static", "paged_prefill_attention_ex", "kv_swap_out",
                  "kv_swap_in"):
         assert "pkv:" + want in pushed, (want, pushed)
     # every range that opened was closed, in nesting order
