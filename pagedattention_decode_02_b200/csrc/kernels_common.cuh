@@ -211,15 +211,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // completes in microseconds; the default budget only ends a wait that would
 // otherwise never end.  Kernels pass their pool's budget (pkv_set_wait_budget)
 // for the waits of their main loops, and keep the default for the waits that
-// make sure no copy is still in flight when they give up.  With a shortened
-// budget the first probe does not block, so that the wait can give up while
-// the copy is still on its way.
+// make sure no copy is still in flight when they give up.  A shortened budget
+// polls without blocking (try_wait may suspend the thread until the phase
+// completes), so that the wait can give up while the copy is still on its way.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t budget_ns = kWaitBudgetNs) {
-    if (budget_ns >= kWaitBudgetNs ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity))
-        return true;
+    if (budget_ns < kWaitBudgetNs) {
+        const uint64_t t0 = global_timer_ns();
+        while (true) {
+            if (mbar_test_wait(bar, parity)) return true;
+            if (global_timer_ns() - t0 > budget_ns) return false;
+        }
+    }
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;

@@ -8,30 +8,34 @@
 // §放不下的时候); token t, at position c_i - n_i + t, attends causally to
 // positions 0 .. c_i - n_i + t through the block table.
 //
-// Work item = 128 query rows of one (sequence, KV head g): the rows of a
-// (sequence, g) are its (token, query head of the group) pairs in token-major
-// order, so all 128 rows share one stream of K/V tiles.  A persistent CTA per
-// SM walks the items heaviest first (the last rows of the longest prompts see
-// the most keys) in a grid-stride order.  Per CTA:
-//   warps 0-3  softmax: load the item's Q tile into shared memory, read each
-//              score tile S = Q K^T from tensor memory (one row per thread),
-//              mask causally, online softmax in base 2, write P (f16/bf16) to
-//              shared memory and rescale the O accumulator in tensor memory
-//              when the running maximum grew by more than 2^8; finally
-//              O / l to global memory;
-//   warp 4     producer: 128-key K and V tiles through two-deep rings, each
+// Work item = 256 query rows of one (sequence, KV head g), as two 128-row
+// tiles that share every K/V tile: the rows of a (sequence, g) are its
+// (token, query head of the group) pairs in token-major order.  Items are
+// ordered group by group - all items of one (sequence, g) next to each other,
+// its last rows (the most keys) first - so that the CTAs working at the same
+// time re-read the same K/V from L2; one persistent CTA per SM takes them in a
+// snake order (forward in even rounds, backward in odd ones), which evens out
+// the decreasing item sizes.  Per CTA:
+//   warps 0-3, 4-7  softmax of tile 0 and tile 1: load the tile's Q rows into
+//              shared memory, read each score tile S = Q K^T from tensor
+//              memory (one row per thread), mask causally, online softmax in
+//              base 2, write P (f16/bf16) back over S in tensor memory, and
+//              rescale the O accumulator there when the running maximum grew
+//              by more than 2^8; finally O / l to global memory;
+//   warp 8     producer: 128-key K and V tiles through two-deep rings, each
 //              tile 16-key stages of 2-D TMA boxes (128-byte swizzle) read
 //              through the block table from this GPU's own pool;
-//   warp 5     MMA: one thread issues S_j = Q K_j^T (M 128, N 128, K = d)
-//              into one of two tensor-memory score buffers and O += P_j V_j
-//              (M 128, N = d, K 128) with tcgen05.mma, completion signalled
-//              by tcgen05.commit; S_{j+1} is issued before P_j is ready so
-//              the tensor pipe computes it while the softmax warps work.
-// Tensor memory: S buffers in columns [0, 128) and [128, 256), O in [256,
-// 256 + d).  Every wait is bounded; a wait that gives up sets
-// PKV_DEVERR_TIMEOUT, the CTA stops issuing work, waits (with the normal
-// budget) for its copies and tensor-core operations in flight, frees its
-// tensor memory and exits.
+//   warp 9     MMA: one thread issues, per tile x, S_x = Q_x K^T (M 128,
+//              N 128, K = d; both operands in shared memory) and O_x += P_x V
+//              (M 128, N = d, K 128; P from tensor memory, V from shared memory
+//              as an MN-major operand), completion by tcgen05.commit.  The
+//              order S_0 S_1 | P_0 V, S_0', P_1 V, S_1' | ... keeps the tensor
+//              pipe on one tile while the softmax warps of the other work.
+// Tensor memory: tile x owns columns [256 x, 256 x + 128) for S (P packed
+// into the first 64 of them) and [256 x + 128, 256 x + 128 + d) for O.
+// Every wait is bounded; a wait that gives up sets PKV_DEVERR_TIMEOUT, the CTA
+// stops issuing work, waits (with the default budget) for its copies and
+// tensor-core operations in flight, frees its tensor memory and exits.
 #include <cuda.h>
 
 #include <type_traits>
@@ -46,30 +50,30 @@ namespace pkv {
 
 namespace {
 
-constexpr int kM = 128;             // query rows per item (tensor-memory lanes)
-constexpr int kN = 128;             // keys per K/V tile
-constexpr int kRing = 2;            // K ring and V ring depth
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
+constexpr int kM = 128;              // rows per query tile (tensor-memory lanes)
+constexpr int kTiles = 2;            // query tiles per work item
+constexpr int kRows = kTiles * kM;   // rows per work item
+constexpr int kN = 128;              // keys per K/V tile
+constexpr int kRing = 2;             // K ring and V ring depth
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;       // two score buffers of kN columns
-constexpr uint32_t kColO = 2 * kN;  // the output accumulator
-constexpr float kRescaleLog2 = 8.f; // keep a stale maximum while the new one is within 2^8
+constexpr uint32_t kTileCols = 256;  // per query tile: S (P) then O
+constexpr float kRescaleLog2 = 8.f;  // keep a stale maximum while the new one is within 2^8
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kMaxSchedSeqs = 4096;  // sequences the group-major order handles (prefix in smem)
 
 enum Bar {
     kKFull = 0,
     kKEmpty = kKFull + kRing,
     kVFull = kKEmpty + kRing,
     kVEmpty = kVFull + kRing,
-    kSFull = kVEmpty + kRing,
-    kSEmpty = kSFull + 2,
-    kPFull = kSEmpty + 2,
-    kPvDone = kPFull + 1,
-    kQFull = kPvDone + 1,
-    kDrain = kQFull + 1,
+    kSFull = kVEmpty + kRing,        // per tile: S_x computed
+    kPFull = kSFull + kTiles,        // per tile: P_x written, O_x rescaled (4 warps)
+    kPvDone = kPFull + kTiles,       // per tile: O_x += P_x V done
+    kQFull = kPvDone + kTiles,       // per tile: Q_x rows written (4 warps)
+    kDrain = kQFull + kTiles,
     kNumBars = kDrain + 1
 };
 
@@ -77,14 +81,13 @@ template <int D>
 struct Layout5 {
     static constexpr int kHalves = D / 64;
     static constexpr int kQBytes = kHalves * kM * 128;   // Q tile [half][row][128 B]
-    static constexpr int kPBytes = 2 * kM * 128;         // P tile [key half][row][128 B]
     static constexpr int kTileBytes = kHalves * kN * 128;// K or V tile [half][key][128 B]
-    static constexpr int kQ = 0;
-    static constexpr int kP = kQ + kQBytes;
-    static constexpr int kK = kP + kPBytes;
+    static constexpr int kQ = 0;                          // [kTiles][kQBytes]
+    static constexpr int kK = kQ + kTiles * kQBytes;
     static constexpr int kV = kK + kRing * kTileBytes;
     static constexpr int kBars = kV + kRing * kTileBytes;
-    static constexpr int kEnd = kBars + kNumBars * 8 + 16;
+    static constexpr int kPrefix = kBars + kNumBars * 8 + 16;   // int [kMaxSchedSeqs + 1]
+    static constexpr int kEnd = kPrefix + (kMaxSchedSeqs + 1) * 4 + kThreads * 4;
     // at least 116 KB, so that a second CTA never shares an SM (each CTA
     // takes all 512 tensor-memory columns)
     static constexpr int kSmem = (1024 + kEnd) > 118784 ? (1024 + kEnd) : 118784;
@@ -92,31 +95,75 @@ struct Layout5 {
 
 // Item parameters, computed identically by every role.
 struct Item {
-    int seq, g, q0, n, c, row0, row_end, base, kv_end, n_kt;
+    int seq, g, q0, n, c, row0, base;
+    int row_end[kTiles];             // exclusive row end of each query tile
+    int n_kt[kTiles];                // key tiles each query tile sees (0: empty tile)
+    int n_kt_all, kv_end;
     bool valid;
 };
 
-__device__ __forceinline__ bool load_item(const PrefillParams& p, long long it,
-                                          long long per_rank, Item& x) {
-    const int rank = (int)(it / per_rank);
-    const int sg = (int)(it % per_rank);
-    x.seq = sg / p.H_kv;
-    x.g = sg % p.H_kv;
+// Work items of sequence s: H_kv groups of ceil(n_s G / 256) items.
+__device__ __forceinline__ int items_of(const PrefillParams& p, int s) {
+    const int n = p.q_starts[s + 1] - p.q_starts[s];
+    if (n <= 0) return 0;
+    const long long rows = (long long)n * p.G;
+    return (int)((rows + kRows - 1) / kRows) * p.H_kv;
+}
+
+// Item `it` -> (sequence, g, tile), the tile counted from the last rows.
+// With `prefix` (items of the sequences before s, shared memory): group-major
+// order; without: rank-major over max_tiles per (sequence, g).
+__device__ __forceinline__ bool load_item(const PrefillParams& p, long long it, const int* prefix,
+                                          long long max_tiles, Item& x) {
+    int rank;
+    if (prefix) {
+        int lo = 0, hi = p.B - 1;          // the last s with prefix[s] <= it
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= it) lo = mid; else hi = mid - 1;
+        }
+        x.seq = lo;
+        const int local = (int)(it - prefix[lo]);
+        const int per_g = (prefix[lo + 1] - prefix[lo]) / p.H_kv;
+        if (per_g <= 0) return false;
+        x.g = local / per_g;
+        rank = local % per_g;
+    } else {
+        const long long per_rank = (long long)p.B * p.H_kv;
+        rank = (int)(it / per_rank);
+        const int sg = (int)(it % per_rank);
+        x.seq = sg / p.H_kv;
+        x.g = sg % p.H_kv;
+        if (rank >= max_tiles) return false;
+    }
     x.q0 = p.q_starts[x.seq];
     x.n = p.q_starts[x.seq + 1] - x.q0;
     x.c = p.lens[x.seq];
     if (x.n <= 0) return false;
     const long long rows = (long long)x.n * p.G;
-    const int n_tiles = (int)((rows + kM - 1) / kM);
+    const int n_tiles = (int)((rows + kRows - 1) / kRows);
     if (rank >= n_tiles) return false;
-    const int tile = n_tiles - 1 - rank;          // heaviest (last rows) first
-    x.row0 = tile * kM;
-    x.row_end = (int)min(rows, (long long)x.row0 + kM);
+    const int tile = n_tiles - 1 - rank;          // last rows (most keys) first
+    x.row0 = tile * kRows;
     x.valid = x.c >= 1 && (long long)x.c <= (long long)p.max_blocks * p.block_size &&
               x.n <= x.c && x.n <= p.max_q_len;
     x.base = x.c - x.n;
-    x.kv_end = x.base + (x.row_end - 1) / p.G + 1;
-    x.n_kt = (x.kv_end + kN - 1) / kN;
+    x.n_kt_all = 0;
+    x.kv_end = 0;
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+        const long long r0 = (long long)x.row0 + t * kM;
+        if (r0 >= rows) {
+            x.row_end[t] = (int)rows;
+            x.n_kt[t] = 0;
+            continue;
+        }
+        x.row_end[t] = (int)min(rows, r0 + kM);
+        const int kv_end = x.base + (x.row_end[t] - 1) / p.G + 1;
+        x.n_kt[t] = (kv_end + kN - 1) / kN;
+        x.kv_end = max(x.kv_end, kv_end);
+        x.n_kt_all = max(x.n_kt_all, x.n_kt[t]);
+    }
     return true;
 }
 
@@ -124,19 +171,20 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const PrefillParams p,
-                    long long n_items) {
+                    long long max_tiles, int allow_grouped) {
     using L = Layout5<D>;
     constexpr int HALVES = L::kHalves;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     uint8_t* sQ = sm + L::kQ;
-    uint8_t* sP = sm + L::kP;
     uint8_t* sK = sm + L::kK;
     uint8_t* sV = sm + L::kV;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* prefix = reinterpret_cast<int*>(sm + L::kPrefix);
+    int* partial = prefix + kMaxSchedSeqs + 1;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -149,13 +197,12 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_init(&bar[kVFull + i], 1);
             mbar_init(&bar[kVEmpty + i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar[kSFull + i], 1);
-            mbar_init(&bar[kSEmpty + i], kSoftmaxWarps);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&bar[kSFull + t], 1);
+            mbar_init(&bar[kPFull + t], 4);
+            mbar_init(&bar[kPvDone + t], 1);
+            mbar_init(&bar[kQFull + t], 4);
         }
-        mbar_init(&bar[kPFull], kSoftmaxWarps);
-        mbar_init(&bar[kPvDone], 1);
-        mbar_init(&bar[kQFull], kSoftmaxWarps);
         mbar_init(&bar[kDrain], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -164,13 +211,48 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tc05::tmem_alloc(tmem_slot, kTmemCols);
         tc05::tmem_relinquish();
     }
+    grid_dependency_wait();
+    // the work order: items per sequence and their prefix sums (every CTA
+    // computes the same)
+    const bool grouped = allow_grouped && p.B <= kMaxSchedSeqs;
+    int s0 = 0, s1 = 0;
+    if (grouped) {
+        const int per = (p.B + kThreads - 1) / kThreads;
+        s0 = min(p.B, tid * per);
+        s1 = min(p.B, s0 + per);
+        int sum = 0;
+        for (int s = s0; s < s1; ++s) sum += items_of(p, s);
+        partial[tid] = sum;
+    }
+    __syncthreads();
+    if (grouped && tid == 0) {
+        int run = 0;
+        for (int i = 0; i < kThreads; ++i) {
+            const int v = partial[i];
+            partial[i] = run;
+            run += v;
+        }
+        prefix[p.B] = run;
+    }
+    __syncthreads();
+    if (grouped) {
+        int run = partial[tid];
+        for (int s = s0; s < s1; ++s) {
+            prefix[s] = run;
+            run += items_of(p, s);
+        }
+    }
     tc05::fence_before();
     __syncthreads();
     tc05::fence_after();
+    const long long n_items = grouped ? (long long)prefix[p.B] : max_tiles * p.B * p.H_kv;
+    const int* pre = grouped ? prefix : nullptr;
     const uint32_t tmem = *tmem_slot;
-
-    grid_dependency_wait();
-    const long long per_rank = (long long)p.B * p.H_kv;
+    // snake order over the persistent CTAs
+    const long long G0 = gridDim.x;
+    auto item_at = [&](long long round) -> long long {
+        return round * G0 + ((round & 1) ? (G0 - 1 - blockIdx.x) : blockIdx.x);
+    };
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
@@ -178,16 +260,18 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int bs = p.block_size;
         const int rpb = bs < 16 ? bs : 16;          // rows per TMA box
         const int boxes = kN / rpb;                  // boxes per half-tile
-        long long armed[2] = {0, 0};                 // K, V tiles whose barrier was armed
+        long long armed_k = 0, armed_v = 0;          // K, V tiles whose barrier was armed
         bool ok = true;
-        for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        for (long long rd = 0; ok; ++rd) {
+            const long long it = item_at(rd);
+            if (it >= n_items) break;
             Item x;
-            if (!load_item(p, it, per_rank, x) || !x.valid) continue;
+            if (!load_item(p, it, pre, max_tiles, x) || !x.valid) continue;
             const int32_t* table = p.tables + (long long)x.seq * p.max_blocks;
-            for (int kt = 0; kt < x.n_kt && ok; ++kt) {
+            for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
                 const int a0 = kt * kN;
                 for (int kv = 0; kv < 2; ++kv) {
-                    const long long j = armed[kv];
+                    const long long j = kv ? armed_v : armed_k;
                     const int st = (int)(j % kRing);
                     if (j >= kRing) {
                         const bool w = mbar_wait(&bar[(kv ? kVEmpty : kKEmpty) + st],
@@ -213,7 +297,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     if (lane == 0)
                         mbar_arrive_expect_tx(full, good * (uint32_t)(rpb * 128 * HALVES));
                     __syncwarp();
-                    armed[kv] = j + 1;
+                    (kv ? armed_v : armed_k) = j + 1;
                     uint8_t* dst = (kv ? sV : sK) + st * L::kTileBytes;
                     const CUtensorMap* map = kv ? &tmap_v : &tmap_k;
                     for (int b = lane; b < boxes; b += 32) {
@@ -234,17 +318,22 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // no copy may outlive the CTA: the last armed tiles of each ring may
         // still be in flight (an earlier tile's slot was reused only after the
         // MMA warp had waited for it to land)
-        for (int kv = 0; kv < 2; ++kv)
-            for (long long j = armed[kv] - kRing < 0 ? 0 : armed[kv] - kRing; j < armed[kv]; ++j)
+        for (int kv = 0; kv < 2; ++kv) {
+            const long long n = kv ? armed_v : armed_k;
+            for (long long j = n - kRing < 0 ? 0 : n - kRing; j < n; ++j)
                 (void)mbar_wait(&bar[(kv ? kVFull : kKFull) + (int)(j % kRing)],
                                 (uint32_t)((j / kRing) & 1));
+        }
     } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------------- MMA
-        constexpr uint32_t idS = tc05::idesc_f16(std::is_same<T, __nv_bfloat16>::value, false, kM, kN);
-        constexpr uint32_t idPV = tc05::idesc_f16(std::is_same<T, __nv_bfloat16>::value, true, kM, D);
-        const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP);
+        constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+        constexpr uint32_t idS = tc05::idesc_f16(kBf16, false, kM, kN);
+        constexpr uint32_t idPV = tc05::idesc_f16(kBf16, true, kM, D);
+        const uint32_t aQ = smem_addr(sQ);
         const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
-        long long sc = 0, pc = 0, ic = 0;   // S issued, PV issued, items started
+        long long kc = 0;                  // K/V tiles consumed
+        long long cnt0 = 0, cnt1 = 0;      // P.V issued per query tile
+        long long qc0 = 0, qc1 = 0;        // items started per query tile
         bool ok = true;
         auto wait_ok = [&](uint64_t* b, uint32_t ph) {
             const bool w = mbar_wait(b, ph, p.wait_ns);
@@ -255,52 +344,76 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             return ok;
         };
-        auto issue_s = [&]() {
-            const int sb = (int)(sc & 1);
-            const int st = (int)(sc % kRing);
-            if (sc >= 2 && !wait_ok(&bar[kSEmpty + sb], (uint32_t)(((sc >> 1) - 1) & 1))) return;
-            if (!wait_ok(&bar[kKFull + st], (uint32_t)((sc / kRing) & 1))) return;
+        // S_x of a key tile whose K sits in ring slot st (issued after this
+        // tile's P.V of the previous key tile)
+        auto issue_s = [&](int x, int st, bool first) {
+            // this tile's previous P.V is done: its P (in S_x's columns) was read
+            const long long c = x ? cnt1 : cnt0;
+            if (!first && !wait_ok(&bar[kPvDone + x], (uint32_t)((c - 1) & 1))) return;
             tc05::fence_after();
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk & 3) * 32);
-                    const uint64_t a = tc05::sdesc_sw128(aQ + (kk >> 2) * (kM * 128) + off, 16, 1024);
-                    const uint64_t b = tc05::sdesc_sw128(aK + st * L::kTileBytes +
-                                                             (kk >> 2) * (kN * 128) + off, 16, 1024);
-                    tc05::mma_ss(tmem + kColS + sb * kN, a, b, idS, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (uint32_t)((kk >> 2) * (kM * 128) + (kk & 3) * 32);
+                    const uint64_t a = tc05::sdesc_sw128(aQ + x * L::kQBytes + off, 16, 1024);
+                    const uint64_t b = tc05::sdesc_sw128(
+                        aK + st * L::kTileBytes + (uint32_t)((kk >> 2) * (kN * 128) + (kk & 3) * 32),
+                        16, 1024);
+                    tc05::mma_ss(tmem + x * kTileCols, a, b, idS, kk > 0 ? 1u : 0u);
                 }
-                tc05::commit(&bar[kSFull + sb]);
-                tc05::commit(&bar[kKEmpty + st]);
+                tc05::commit(&bar[kSFull + x]);
             }
             __syncwarp();
-            ++sc;
         };
-        for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            Item x;
-            if (!load_item(p, it, per_rank, x) || !x.valid) continue;
-            if (!wait_ok(&bar[kQFull], (uint32_t)(ic & 1))) break;
-            ++ic;
+        // O_x += P_x V of a key tile whose V sits in ring slot st
+        auto issue_pv = [&](int x, int st, int ksteps, bool first) {
+            long long& c = x ? cnt1 : cnt0;
+            if (!wait_ok(&bar[kPFull + x], (uint32_t)(c & 1))) return;
             tc05::fence_after();
-            issue_s();
-            for (int kt = 0; kt < x.n_kt && ok; ++kt) {
-                if (kt + 1 < x.n_kt) {
-                    issue_s();
-                    if (!ok) break;
+            if (lane == 0) {
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    const uint64_t b = tc05::sdesc_sw128(
+                        aV + st * L::kTileBytes + (uint32_t)(kk * 16 * 128), kN * 128, 1024);
+                    tc05::mma_ts(tmem + x * kTileCols + kM, tmem + x * kTileCols + kk * 8, b, idPV,
+                                 (!first || kk > 0) ? 1u : 0u);
                 }
-                // O += P_kt V_kt
-                const int st = (int)(pc % kRing);
-                if (!wait_ok(&bar[kPFull], (uint32_t)(pc & 1))) break;
-                if (!wait_ok(&bar[kVFull + st], (uint32_t)((pc / kRing) & 1))) break;
+                tc05::commit(&bar[kPvDone + x]);
+            }
+            __syncwarp();
+            ++c;
+        };
+        for (long long rd = 0; ok; ++rd) {
+            const long long it = item_at(rd);
+            if (it >= n_items) break;
+            Item x;
+            if (!load_item(p, it, pre, max_tiles, x) || !x.valid) continue;
+            if (x.n_kt[0] > 0 && wait_ok(&bar[kQFull + 0], (uint32_t)(qc0 & 1))) ++qc0;
+            if (ok && x.n_kt[1] > 0 && wait_ok(&bar[kQFull + 1], (uint32_t)(qc1 & 1))) ++qc1;
+            if (!ok) break;
+            // key tile 0: S_0, S_1
+            {
+                const int st = (int)(kc % kRing);
+                if (!wait_ok(&bar[kKFull + st], (uint32_t)((kc / kRing) & 1))) break;
+                if (x.n_kt[0] > 0) issue_s(0, st, true);
+                if (ok && x.n_kt[1] > 0) issue_s(1, st, true);
+                if (!ok) break;
+                if (lane == 0) tc05::commit(&bar[kKEmpty + st]);
+                __syncwarp();
+            }
+            for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
+                const int st = (int)(kc % kRing);
+                const int st1 = (int)((kc + 1) % kRing);
+                const bool more = kt + 1 < x.n_kt_all;
+                if (!wait_ok(&bar[kVFull + st], (uint32_t)((kc / kRing) & 1))) break;
+                if (more && !wait_ok(&bar[kKFull + st1], (uint32_t)(((kc + 1) / kRing) & 1))) break;
                 tc05::fence_after();
-                const int a0 = kt * kN;
-                const int keys = min(kN, x.kv_end - a0);
+                const int keys = min(kN, x.kv_end - kt * kN);
                 const int ksteps = (keys + 15) >> 4;
-                uint8_t* vt = sV + st * L::kTileBytes;
                 if (keys < ksteps * 16) {
                     // keys past the end inside the last 16-key step carry P = 0;
                     // their V rows may hold anything, so make them 0 (0 * NaN
                     // would poison the sum)
+                    uint8_t* vt = sV + st * L::kTileBytes;
                     const int rows = ksteps * 16 - keys;
                     for (int i = lane; i < rows * HALVES * 8; i += 32) {
                         const int r = keys + i / (HALVES * 8);
@@ -312,19 +425,25 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                if (lane == 0) {
-                    for (int kk = 0; kk < ksteps; ++kk) {
-                        const uint64_t a = tc05::sdesc_sw128(
-                            aP + (kk >> 2) * (kM * 128) + (uint32_t)((kk & 3) * 32), 16, 1024);
-                        const uint64_t b = tc05::sdesc_sw128(
-                            aV + st * L::kTileBytes + (uint32_t)(kk * 16 * 128), kN * 128, 1024);
-                        tc05::mma_ss(tmem + kColO, a, b, idPV, (kt > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc05::commit(&bar[kVEmpty + st]);
-                    tc05::commit(&bar[kPvDone]);
-                }
+                // per tile: P.V of this key tile, then S of the next one
+                // both tiles' P.V of this key tile first, then (each once its
+                // own P.V has completed, so that its P is read before S
+                // overwrites it) both tiles' S of the next one: the second P.V
+                // and the first S queue behind running work, so the tensor pipe
+                // does not wait for the issuing thread
+                if (kt < x.n_kt[0]) issue_pv(0, st, ksteps, kt == 0);
+                if (ok && kt < x.n_kt[1]) issue_pv(1, st, ksteps, kt == 0);
+                if (!ok) break;
+                if (lane == 0) tc05::commit(&bar[kVEmpty + st]);
                 __syncwarp();
-                ++pc;
+                if (more) {
+                    if (kt + 1 < x.n_kt[0]) issue_s(0, st1, false);
+                    if (ok && kt + 1 < x.n_kt[1]) issue_s(1, st1, false);
+                    if (!ok) break;
+                    if (lane == 0) tc05::commit(&bar[kKEmpty + st1]);
+                    __syncwarp();
+                }
+                ++kc;
             }
         }
         // every tensor-core operation issued has completed before the CTA
@@ -334,9 +453,11 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         (void)mbar_wait(&bar[kDrain], 0);
     } else {
         // ------------------------------------------------------------- softmax
-        const int r = tid;                         // tensor-memory lane = tile row
-        const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
-        long long sc = 0, pc = 0;
+        const int t = warp >> 2;                   // query tile of this warp
+        const int r = tid & (kM - 1);              // tensor-memory lane = tile row
+        const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16) + t * kTileCols;
+        uint8_t* sQt = sQ + t * L::kQBytes;
+        long long cnt = 0;
         bool ok = true;
         auto wait_ok = [&](uint64_t* b, uint32_t ph) {
             const bool w = mbar_wait(b, ph, p.wait_ns);
@@ -349,23 +470,31 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         T* out = reinterpret_cast<T*>(p.out);
         const T* qg = reinterpret_cast<const T*>(p.q);
-        for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        for (long long rd = 0; ok; ++rd) {
+            const long long it = item_at(rd);
+            if (it >= n_items) break;
             Item x;
-            if (!load_item(p, it, per_rank, x)) continue;
-            const int gr = x.row0 + r;             // this thread's row of (seq, g)
-            const bool row_ok = gr < x.row_end;
-            const int tok = (row_ok ? gr : x.row_end - 1) / p.G;
-            const int head = x.g * p.G + (row_ok ? gr : x.row_end - 1) % p.G;
+            if (!load_item(p, it, pre, max_tiles, x)) continue;
+            // this warp's tile (plain values: no run-time index into x)
+            const int my_n_kt = t ? x.n_kt[1] : x.n_kt[0];
+            const int my_row_end = t ? x.row_end[1] : x.row_end[0];
+            if (my_n_kt == 0) continue;                    // this tile is past the rows
+            const int row0 = x.row0 + t * kM;
+            const int gr = row0 + r;                       // this thread's row of (seq, g)
+            const bool row_ok = gr < my_row_end;
+            const int last = row_ok ? gr : my_row_end - 1;
+            const int tok = last / p.G;
+            const int head = x.g * p.G + last % p.G;
             T* orow = out + ((size_t)(x.q0 + tok) * p.H_q + head) * D;
             if (!x.valid) {
-                if (r == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
+                if (r == 0 && t == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
                 if (x.n <= p.max_q_len && row_ok)
                     for (int i = 0; i < D; i += 8)
                         *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
                 continue;
             }
-            // block ids of the item in range? (the producer skipped bad ones)
-            // (each warp checks on its own: no CTA-wide barrier inside the
+            // block ids of the item in range? (the producer skipped bad ones;
+            // each warp checks on its own: no CTA-wide barrier inside the
             // roles, which a warp that gave up could leave unreached)
             bool bad = false;
             const int n_blk = (x.kv_end + p.block_size - 1) / p.block_size;
@@ -375,7 +504,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 bad |= id < 0 || id >= p.num_blocks;
             }
             bad = __any_sync(kFull, bad);
-            if (bad && r == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
+            if (bad && r == 0 && t == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
             // Q row -> shared memory, 128-byte swizzle
             {
                 const T* qrow = qg + ((size_t)(x.q0 + tok) * p.H_q + head) * D;
@@ -383,113 +512,136 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 for (int c = 0; c < D / 8; ++c) {
                     uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + c * 8)
                                      : make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(sQ + (c >> 3) * (kM * 128) + (r >> 3) * 1024 +
+                    *reinterpret_cast<uint4*>(sQt + (c >> 3) * (kM * 128) + (r >> 3) * 1024 +
                                               (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
                 }
             }
             fence_proxy_async_smem();
             tc05::fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bar[kQFull]);
+            if (lane == 0) tc::mbar_arrive(&bar[kQFull + t]);
 
-            const int lim = x.base + tok;          // last visible key of this row
-            const int min_lim = x.base + x.row0 / p.G;
+            const int lim = x.base + tok;                  // last visible key of this row
+            const int min_lim = x.base + row0 / p.G;
             float m_run = -INFINITY, l_run = 0.f;
-            for (int kt = 0; kt < x.n_kt; ++kt) {
-                const int sb = (int)(sc & 1);
-                if (!wait_ok(&bar[kSFull + sb], (uint32_t)((sc >> 1) & 1))) break;
+            for (int kt = 0; kt < my_n_kt; ++kt) {
+                if (!wait_ok(&bar[kSFull + t], (uint32_t)(cnt & 1))) break;
                 tc05::fence_after();
-                float s[kN];
-#pragma unroll
-                for (int c = 0; c < kN / 32; ++c) {
-                    uint32_t u[32];
-                    tc05::tmem_ld32(t_lane + kColS + sb * kN + c * 32, u);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) s[c * 32 + j] = __uint_as_float(u[j]);
-                }
-                tc05::fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bar[kSEmpty + sb]);
-                ++sc;
-                // scale into the base-2 domain, causal mask, tile maximum
+                // pass 1 over S: the largest scaled score of each row (32 columns
+                // at a time: few live registers).  Keys past the row's position
+                // are masked, which only the tile on the diagonal needs; the
+                // scale may be negative, then the smallest raw score counts.
                 const int k0 = kt * kN;
-                float mt = -INFINITY;
-                if (k0 + kN - 1 <= min_lim) {
+                const bool full_tile = k0 + kN - 1 <= min_lim;
+                const bool up = p.q_scale >= 0.f;
+                float ext = up ? -INFINITY : INFINITY;
 #pragma unroll
-                    for (int j = 0; j < kN; ++j) {
-                        s[j] *= p.q_scale;
-                        mt = fmaxf(mt, s[j]);
-                    }
-                } else {
+                for (int c = 0; c < kN / 64; ++c) {
+                    uint32_t u[64];
+                    tc05::tmem_ld64(t_lane + c * 64, u);
+                    const int vis = lim - k0 - c * 64;     // columns j <= vis are visible
+                    if (full_tile) {
+                        if (up) {
 #pragma unroll
-                    for (int j = 0; j < kN; ++j) {
-                        s[j] = (k0 + j <= lim) ? s[j] * p.q_scale : -INFINITY;
-                        mt = fmaxf(mt, s[j]);
+                            for (int j = 0; j < 64; ++j) ext = fmaxf(ext, __uint_as_float(u[j]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) ext = fminf(ext, __uint_as_float(u[j]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            const float v = __uint_as_float(u[j]);
+                            if (j <= vis) ext = up ? fmaxf(ext, v) : fminf(ext, v);
+                        }
                     }
                 }
+                const float mt = fabsf(ext) == INFINITY ? -INFINITY : ext * p.q_scale;
                 const float m_new = (mt > m_run + kRescaleLog2) ? mt : m_run;
                 const float alpha = tc05::ex2(m_run - m_new);   // 0 on the first tile
-                // probabilities, row sum, P row (f16/bf16 pairs) in registers
-                uint32_t pk[kN / 2];
-                float rs = 0.f;
-#pragma unroll
-                for (int j = 0; j < kN; j += 2) {
-                    const float a = tc05::ex2(s[j] - m_new);
-                    const float b = tc05::ex2(s[j + 1] - m_new);
-                    rs += a + b;
-                    pk[j / 2] = tc::MmaType<T>::pack(a, b);
-                }
-                l_run = l_run * alpha + rs;
-                // the previous P.V must be done: P's buffer is reused and O is
-                // rescaled below
-                if (pc > 0 && !wait_ok(&bar[kPvDone], (uint32_t)((pc - 1) & 1))) break;
-                tc05::fence_after();
+                // O of this tile is idle: the MMA warp issued this S only after
+                // the previous P.V had completed
                 if (kt > 0 && __any_sync(kFull, m_new != m_run)) {
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
-                        uint32_t u[32];
-                        tc05::tmem_ld32(t_lane + kColO + c * 32, u);
+                        uint32_t o[32];
+                        tc05::tmem_ld32(t_lane + kM + c * 32, o);
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
-                        tc05::tmem_st32(t_lane + kColO + c * 32, u);
+                            o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tc05::tmem_st32(t_lane + kM + c * 32, o);
                     }
                 }
                 m_run = m_new;
+                // pass 2: probabilities -> P (f16/bf16 pairs) over S's first 64
+                // columns; chunk c's P lands in columns 32 c .. 32 c + 31, all
+                // of them S values already read
+                const float neg_m = -m_new;
+                float rs = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < kN / 64; ++c) {
+                    uint32_t u[64];
+                    tc05::tmem_ld64(t_lane + c * 64, u);
+                    if (full_tile) {
 #pragma unroll
-                for (int c = 0; c < kN / 8; ++c) {
-                    // keys 8c .. 8c + 7: half c / 8 of the P tile, chunk c % 8
-                    *reinterpret_cast<uint4*>(sP + (c >> 3) * (kM * 128) + (r >> 3) * 1024 +
-                                              (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2) {
+                                const float a = tc05::ex2(fmaf(__uint_as_float(u[h * 32 + j]), p.q_scale, neg_m));
+                                const float b = tc05::ex2(fmaf(__uint_as_float(u[h * 32 + j + 1]), p.q_scale, neg_m));
+                                rs += a + b;
+                                pk[j / 2] = tc::MmaType<T>::pack(a, b);
+                            }
+                            tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
+                        }
+                    } else {
+                        const int vis = lim - k0 - c * 64;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2) {
+                                const int jj = h * 32 + j;
+                                const float a = jj <= vis
+                                    ? tc05::ex2(fmaf(__uint_as_float(u[jj]), p.q_scale, neg_m)) : 0.f;
+                                const float b = jj + 1 <= vis
+                                    ? tc05::ex2(fmaf(__uint_as_float(u[jj + 1]), p.q_scale, neg_m)) : 0.f;
+                                rs += a + b;
+                                pk[j / 2] = tc::MmaType<T>::pack(a, b);
+                            }
+                            tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
+                        }
+                    }
                 }
-                fence_proxy_async_smem();
+                tc05::tmem_st_wait();
+                l_run = l_run * alpha + rs;
                 tc05::fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&bar[kPFull]);
-                ++pc;
+                if (lane == 0) tc::mbar_arrive(&bar[kPFull + t]);
+                ++cnt;
             }
             if (!ok) break;
             // epilogue: O / l of the item's last P.V
-            if (!wait_ok(&bar[kPvDone], (uint32_t)((pc - 1) & 1))) break;
+            if (!wait_ok(&bar[kPvDone + t], (uint32_t)((cnt - 1) & 1))) break;
             tc05::fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t u[32];
-                tc05::tmem_ld32(t_lane + kColO + c * 32, u);
+                uint32_t o[32];
+                tc05::tmem_ld32(t_lane + kM + c * 32, o);
                 if (bad) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) u[j] = 0u;   // the item's keys were not read
+                    for (int j = 0; j < 32; ++j) o[j] = 0u;   // the item's keys were not read
                 }
                 if (row_ok) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         uint4 v;
-                        v.x = tc::MmaType<T>::pack(__uint_as_float(u[j]) * inv, __uint_as_float(u[j + 1]) * inv);
-                        v.y = tc::MmaType<T>::pack(__uint_as_float(u[j + 2]) * inv, __uint_as_float(u[j + 3]) * inv);
-                        v.z = tc::MmaType<T>::pack(__uint_as_float(u[j + 4]) * inv, __uint_as_float(u[j + 5]) * inv);
-                        v.w = tc::MmaType<T>::pack(__uint_as_float(u[j + 6]) * inv, __uint_as_float(u[j + 7]) * inv);
+                        v.x = tc::MmaType<T>::pack(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv);
+                        v.y = tc::MmaType<T>::pack(__uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+                        v.z = tc::MmaType<T>::pack(__uint_as_float(o[j + 4]) * inv, __uint_as_float(o[j + 5]) * inv);
+                        v.w = tc::MmaType<T>::pack(__uint_as_float(o[j + 6]) * inv, __uint_as_float(o[j + 7]) * inv);
                         *reinterpret_cast<uint4*>(orow + c * 32 + j) = v;
                     }
                 }
@@ -515,14 +667,17 @@ cudaError_t launch_t(const PrefillParams& p, const pkv_pool* pool, cudaStream_t 
     static unsigned long long attr_done = 0;
     cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
-    const long long max_tiles = ((long long)p.max_q_len * p.G + kM - 1) / kM;
-    const long long n_items = max_tiles * p.B * p.H_kv;
+    const long long max_tiles = ((long long)p.max_q_len * p.G + kRows - 1) / kRows;
+    const long long n_items = max_tiles * p.B * p.H_kv;   // an upper bound
     if (n_items <= 0) return cudaSuccess;
     const int sms = pool->sm_count > 0 ? pool->sm_count : 148;
     const int grid = (int)(n_items < sms ? n_items : sms);
+    // the group-major order counts items in 32-bit prefix sums
+    const int allow_grouped = n_items < (1LL << 31) ? 1 : 0;
     return launch_kernel(kern, dim3(grid), dim3(kThreads), L::kSmem, st, false,
                          *reinterpret_cast<const CUtensorMap*>(pool->tmap_k),
-                         *reinterpret_cast<const CUtensorMap*>(pool->tmap_v), p, n_items);
+                         *reinterpret_cast<const CUtensorMap*>(pool->tmap_v), p, max_tiles,
+                         allow_grouped);
 }
 
 }  // namespace

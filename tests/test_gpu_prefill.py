@@ -156,3 +156,29 @@ def test_prefill_invalid_inputs(kernel):
         pk.paged_prefill_attention(p32, q.float(), starts, tables, lens, 0.1)
     with pytest.raises(pk.PagedKVError):                                 # q dtype mismatch
         pk.paged_prefill_attention(pool, q.bfloat16(), starts, tables, lens, 0.1)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_negative_scale(kernel):
+    # the scale is a parameter (any finite value): with a negative one the
+    # largest scaled score comes from the smallest raw score
+    cfg = small("llama2_70b", n_q_heads=8, n_kv_heads=2, head_dim=128, kv_dtype="bf16",
+                q_dtype="bf16", block_size=16, batch=3, lengths=("uniform", 150, 400))
+    cfg = dataclasses.replace(cfg)
+    side = setup_config(cfg, seed=21)
+    hist = [side.orc.bm.lengths[s] for s in side.seqs]
+    seqs = side.seqs
+    qs = [wl.round_to(wl.prompt_queries(cfg, 0, s, int(n)), "bf16") for s, n in zip(seqs, hist)]
+    starts = np.concatenate([[0], np.cumsum(hist)]).astype(np.int32)
+    max_blocks = max(pk.bt_num_blocks(side.pool, s) for s in seqs)
+    tables, lens, _ = pk.bt_export(side.pool, seqs, max_blocks)
+    out = pk.paged_prefill_attention(side.pool, to_torch(np.concatenate(qs), "bf16"),
+                                     torch.from_numpy(starts).cuda(),
+                                     torch.from_numpy(tables).cuda(),
+                                     torch.from_numpy(lens).cuda(), -cfg.scale, kernel=kernel)
+    torch.cuda.synchronize()
+    assert pk.pkv_device_error(side.pool) == 0
+    got = to_f64(from_torch(out, "bf16"), "bf16")
+    for i, (s, q) in enumerate(zip(seqs, qs)):
+        ref = side.orc.prefill(s, q, "bf16", -cfg.scale)
+        compare_out(got[starts[i]:starts[i + 1]], ref, "bf16")
