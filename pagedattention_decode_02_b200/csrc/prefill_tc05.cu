@@ -16,21 +16,25 @@
 // time re-read the same K/V from L2; one persistent CTA per SM takes them in a
 // snake order (forward in even rounds, backward in odd ones), which evens out
 // the decreasing item sizes.  Per CTA:
-//   warps 0-3, 4-7  softmax of tile 0 and tile 1: load the tile's Q rows into
-//              shared memory, read each score tile S = Q K^T from tensor
-//              memory (one row per thread), mask causally, online softmax in
-//              base 2, write P (f16/bf16) back over S in tensor memory, and
-//              rescale the O accumulator there when the running maximum grew
-//              by more than 2^8; finally O / l to global memory;
+//   warps 0-3, 4-7  softmax of tile 0 and tile 1: read each score tile
+//              S = Q K^T from tensor memory (one row per thread), mask
+//              causally, online softmax in base 2, write P (f16/bf16) back
+//              over S in tensor memory, and rescale the O accumulator there
+//              when the running maximum grew by more than 2^8; finally O / l
+//              to global memory.  The next item's Q rows are copied into
+//              shared memory (cp.async) as soon as the tile's last S of the
+//              current item is done, and handed to the tensor cores before
+//              the current item's output is written, so that the next S runs
+//              under that epilogue;
 //   warp 8     producer: 128-key K and V tiles through two-deep rings, each
 //              tile 16-key stages of 2-D TMA boxes (128-byte swizzle) read
 //              through the block table from this GPU's own pool;
 //   warp 9     MMA: one thread issues, per tile x, S_x = Q_x K^T (M 128,
 //              N 128, K = d; both operands in shared memory) and O_x += P_x V
 //              (M 128, N = d, K 128; P from tensor memory, V from shared memory
-//              as an MN-major operand), completion by tcgen05.commit.  The
-//              order S_0 S_1 | P_0 V, S_0', P_1 V, S_1' | ... keeps the tensor
-//              pipe on one tile while the softmax warps of the other work.
+//              as an MN-major operand), completion by tcgen05.commit.  Per key
+//              tile: P_0 V, P_1 V, then S_0 and S_1 of the next key tile (each
+//              after its tile's P.V completed: S overwrites P).
 // Tensor memory: tile x owns columns [256 x, 256 x + 128) for S (P packed
 // into the first 64 of them) and [256 x + 128, 256 x + 128 + d) for O.
 // Every wait is bounded; a wait that gives up sets PKV_DEVERR_TIMEOUT, the CTA
@@ -62,7 +66,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTileCols = 256;  // per query tile: S (P) then O
 constexpr float kRescaleLog2 = 8.f;  // keep a stale maximum while the new one is within 2^8
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kMaxSchedSeqs = 4096;  // sequences the group-major order handles (prefix in smem)
+// sequences for which the group-major order and shared copies of q_starts
+// and context lengths are kept in shared memory
+constexpr int kMaxSchedSeqs = 1024;
 
 enum Bar {
     kKFull = 0,
@@ -86,8 +92,10 @@ struct Layout5 {
     static constexpr int kK = kQ + kTiles * kQBytes;
     static constexpr int kV = kK + kRing * kTileBytes;
     static constexpr int kBars = kV + kRing * kTileBytes;
-    static constexpr int kPrefix = kBars + kNumBars * 8 + 16;   // int [kMaxSchedSeqs + 1]
-    static constexpr int kEnd = kPrefix + (kMaxSchedSeqs + 1) * 4 + kThreads * 4;
+    // int prefix[kMaxSchedSeqs + 1], q_starts[kMaxSchedSeqs + 1], lens[kMaxSchedSeqs],
+    // partial[kThreads]
+    static constexpr int kSched = kBars + kNumBars * 8 + 16;
+    static constexpr int kEnd = kSched + (3 * kMaxSchedSeqs + 2 + kThreads) * 4;
     // at least 116 KB, so that a second CTA never shares an SM (each CTA
     // takes all 512 tensor-memory columns)
     static constexpr int kSmem = (1024 + kEnd) > 118784 ? (1024 + kEnd) : 118784;
@@ -102,29 +110,34 @@ struct Item {
     bool valid;
 };
 
-// Work items of sequence s: H_kv groups of ceil(n_s G / 256) items.
-__device__ __forceinline__ int items_of(const PrefillParams& p, int s) {
-    const int n = p.q_starts[s + 1] - p.q_starts[s];
+// The work order and the sequences' row offsets and lengths: shared-memory
+// copies when the batch has at most kMaxSchedSeqs sequences, else global.
+struct Sched {
+    const int* prefix;               // items of the sequences before s; null: rank-major
+    const int* q_starts;
+    const int* lens;
+    long long max_tiles;
+};
+
+__device__ __forceinline__ int items_of(int n, int G, int H_kv) {
     if (n <= 0) return 0;
-    const long long rows = (long long)n * p.G;
-    return (int)((rows + kRows - 1) / kRows) * p.H_kv;
+    const long long rows = (long long)n * G;
+    return (int)((rows + kRows - 1) / kRows) * H_kv;
 }
 
 // Item `it` -> (sequence, g, tile), the tile counted from the last rows.
-// With `prefix` (items of the sequences before s, shared memory): group-major
-// order; without: rank-major over max_tiles per (sequence, g).
-__device__ __forceinline__ bool load_item(const PrefillParams& p, long long it, const int* prefix,
-                                          long long max_tiles, Item& x) {
+__device__ __forceinline__ bool load_item(const PrefillParams& p, long long it, const Sched& sc,
+                                          Item& x) {
     int rank;
-    if (prefix) {
+    if (sc.prefix) {
         int lo = 0, hi = p.B - 1;          // the last s with prefix[s] <= it
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (prefix[mid] <= it) lo = mid; else hi = mid - 1;
+            if (sc.prefix[mid] <= it) lo = mid; else hi = mid - 1;
         }
         x.seq = lo;
-        const int local = (int)(it - prefix[lo]);
-        const int per_g = (prefix[lo + 1] - prefix[lo]) / p.H_kv;
+        const int local = (int)(it - sc.prefix[lo]);
+        const int per_g = (sc.prefix[lo + 1] - sc.prefix[lo]) / p.H_kv;
         if (per_g <= 0) return false;
         x.g = local / per_g;
         rank = local % per_g;
@@ -134,11 +147,11 @@ __device__ __forceinline__ bool load_item(const PrefillParams& p, long long it, 
         const int sg = (int)(it % per_rank);
         x.seq = sg / p.H_kv;
         x.g = sg % p.H_kv;
-        if (rank >= max_tiles) return false;
+        if (rank >= sc.max_tiles) return false;
     }
-    x.q0 = p.q_starts[x.seq];
-    x.n = p.q_starts[x.seq + 1] - x.q0;
-    x.c = p.lens[x.seq];
+    x.q0 = sc.q_starts[x.seq];
+    x.n = sc.q_starts[x.seq + 1] - x.q0;
+    x.c = sc.lens[x.seq];
     if (x.n <= 0) return false;
     const long long rows = (long long)x.n * p.G;
     const int n_tiles = (int)((rows + kRows - 1) / kRows);
@@ -183,8 +196,10 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* prefix = reinterpret_cast<int*>(sm + L::kPrefix);
-    int* partial = prefix + kMaxSchedSeqs + 1;
+    int* prefix = reinterpret_cast<int*>(sm + L::kSched);
+    int* qs_c = prefix + kMaxSchedSeqs + 1;
+    int* len_c = qs_c + kMaxSchedSeqs + 1;
+    int* partial = len_c + kMaxSchedSeqs;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -213,15 +228,20 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
     grid_dependency_wait();
     // the work order: items per sequence and their prefix sums (every CTA
-    // computes the same)
+    // computes the same), with the sequences' offsets and lengths copied
     const bool grouped = allow_grouped && p.B <= kMaxSchedSeqs;
     int s0 = 0, s1 = 0;
+    if (grouped) {
+        for (int s = tid; s <= p.B; s += kThreads) qs_c[s] = p.q_starts[s];
+        for (int s = tid; s < p.B; s += kThreads) len_c[s] = p.lens[s];
+    }
+    __syncthreads();
     if (grouped) {
         const int per = (p.B + kThreads - 1) / kThreads;
         s0 = min(p.B, tid * per);
         s1 = min(p.B, s0 + per);
         int sum = 0;
-        for (int s = s0; s < s1; ++s) sum += items_of(p, s);
+        for (int s = s0; s < s1; ++s) sum += items_of(qs_c[s + 1] - qs_c[s], p.G, p.H_kv);
         partial[tid] = sum;
     }
     __syncthreads();
@@ -239,14 +259,15 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         int run = partial[tid];
         for (int s = s0; s < s1; ++s) {
             prefix[s] = run;
-            run += items_of(p, s);
+            run += items_of(qs_c[s + 1] - qs_c[s], p.G, p.H_kv);
         }
     }
     tc05::fence_before();
     __syncthreads();
     tc05::fence_after();
     const long long n_items = grouped ? (long long)prefix[p.B] : max_tiles * p.B * p.H_kv;
-    const int* pre = grouped ? prefix : nullptr;
+    const Sched sc{grouped ? prefix : nullptr, grouped ? qs_c : p.q_starts,
+                   grouped ? len_c : p.lens, max_tiles};
     const uint32_t tmem = *tmem_slot;
     // snake order over the persistent CTAs
     const long long G0 = gridDim.x;
@@ -256,20 +277,42 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
-        const uint64_t policy = l2_evict_first_policy();
+        // the other work items of the same (sequence, KV head), running on
+        // other SMs at about the same time, read the same K/V tiles: keep them
+        // in L2
+        const uint64_t policy = tc05::l2_evict_last_policy();
         const int bs = p.block_size;
         const int rpb = bs < 16 ? bs : 16;          // rows per TMA box
-        const int boxes = kN / rpb;                  // boxes per half-tile
+        const int boxes = kN / rpb;                  // boxes per half-tile (<= 128)
         long long armed_k = 0, armed_v = 0;          // K, V tiles whose barrier was armed
         bool ok = true;
         for (long long rd = 0; ok; ++rd) {
             const long long it = item_at(rd);
             if (it >= n_items) break;
             Item x;
-            if (!load_item(p, it, pre, max_tiles, x) || !x.valid) continue;
+            if (!load_item(p, it, sc, x) || !x.valid) continue;
             const int32_t* table = p.tables + (long long)x.seq * p.max_blocks;
             for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
                 const int a0 = kt * kN;
+                // the block ids of this lane's boxes (l, l + 32, ...), read once
+                // for K and V, before waiting for the slots; -1: past the end
+                // or out of range (skipped; the softmax warps zero such an
+                // item's output)
+                int ids[4];
+                uint32_t good = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int b = lane + 32 * i;
+                    const int t0 = a0 + b * rpb;
+                    int id = -1;
+                    if (b < boxes && t0 < x.kv_end) {
+                        id = table[t0 / bs];
+                        if (id < 0 || id >= p.num_blocks) id = -1;
+                    }
+                    ids[i] = id;
+                    good += id >= 0 ? 1u : 0u;
+                }
+                good = __reduce_add_sync(kFull, good);
                 for (int kv = 0; kv < 2; ++kv) {
                     const long long j = kv ? armed_v : armed_k;
                     const int st = (int)(j % kRing);
@@ -283,29 +326,21 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                             break;
                         }
                     }
-                    // lane l handles boxes l, l + 32, ...; ids out of range are
-                    // skipped (the softmax warps zero such an item's output)
-                    uint32_t good = 0;
-                    for (int b = lane; b < boxes; b += 32) {
-                        const int t0 = a0 + b * rpb;
-                        if (t0 >= x.kv_end) break;
-                        const int id = table[t0 / bs];
-                        good += (id >= 0 && id < p.num_blocks) ? 1u : 0u;
-                    }
-                    good = __reduce_add_sync(kFull, good);
                     uint64_t* full = &bar[(kv ? kVFull : kKFull) + st];
-                    if (lane == 0)
+                    if (tc05::elect_one())
                         mbar_arrive_expect_tx(full, good * (uint32_t)(rpb * 128 * HALVES));
                     __syncwarp();
                     (kv ? armed_v : armed_k) = j + 1;
                     uint8_t* dst = (kv ? sV : sK) + st * L::kTileBytes;
                     const CUtensorMap* map = kv ? &tmap_v : &tmap_k;
-                    for (int b = lane; b < boxes; b += 32) {
+                    // every lane issues its own boxes: the copies' issue
+                    // latencies overlap instead of adding up
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (ids[i] < 0) continue;
+                        const int b = lane + 32 * i;
                         const int t0 = a0 + b * rpb;
-                        if (t0 >= x.kv_end) break;
-                        const int id = table[t0 / bs];
-                        if (id < 0 || id >= p.num_blocks) continue;
-                        const int y = (id * p.H_kv + x.g) * bs + (t0 % bs);
+                        const int y = (ids[i] * p.H_kv + x.g) * bs + (t0 % bs);
 #pragma unroll
                         for (int hf = 0; hf < HALVES; ++hf)
                             tc::tma_load_2d(dst + hf * (kN * 128) + b * rpb * 128, map, hf * 64, y,
@@ -329,8 +364,12 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
         constexpr uint32_t idS = tc05::idesc_f16(kBf16, false, kM, kN);
         constexpr uint32_t idPV = tc05::idesc_f16(kBf16, true, kM, D);
-        const uint32_t aQ = smem_addr(sQ);
-        const uint32_t aK = smem_addr(sK), aV = smem_addr(sV);
+        // descriptors of the operands' first 16-element K step; later steps add
+        // their byte offset / 16 to the start-address field (the addresses
+        // stay below 256 KB, so the field never carries over)
+        const uint64_t dQ = tc05::sdesc_sw128(smem_addr(sQ), 16, 1024);
+        const uint64_t dK = tc05::sdesc_sw128(smem_addr(sK), 16, 1024);
+        const uint64_t dV = tc05::sdesc_sw128(smem_addr(sV), kN * 128, 1024);
         long long kc = 0;                  // K/V tiles consumed
         long long cnt0 = 0, cnt1 = 0;      // P.V issued per query tile
         long long qc0 = 0, qc1 = 0;        // items started per query tile
@@ -344,22 +383,21 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             return ok;
         };
-        // S_x of a key tile whose K sits in ring slot st (issued after this
-        // tile's P.V of the previous key tile)
+        // S_x of a key tile whose K sits in ring slot st
         auto issue_s = [&](int x, int st, bool first) {
             // this tile's previous P.V is done: its P (in S_x's columns) was read
             const long long c = x ? cnt1 : cnt0;
             if (!first && !wait_ok(&bar[kPvDone + x], (uint32_t)((c - 1) & 1))) return;
             tc05::fence_after();
-            if (lane == 0) {
+            const uint64_t a0 = dQ + (uint64_t)((x * L::kQBytes) >> 4);
+            const uint64_t b0 = dK + (uint64_t)((st * L::kTileBytes) >> 4);
+            const uint32_t d = tmem + x * kTileCols;
+            if (tc05::elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * (kM * 128) + (kk & 3) * 32);
-                    const uint64_t a = tc05::sdesc_sw128(aQ + x * L::kQBytes + off, 16, 1024);
-                    const uint64_t b = tc05::sdesc_sw128(
-                        aK + st * L::kTileBytes + (uint32_t)((kk >> 2) * (kN * 128) + (kk & 3) * 32),
-                        16, 1024);
-                    tc05::mma_ss(tmem + x * kTileCols, a, b, idS, kk > 0 ? 1u : 0u);
+                    const uint32_t q_off = ((kk >> 2) * (kM * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t k_off = ((kk >> 2) * (kN * 128) + (kk & 3) * 32) >> 4;
+                    tc05::mma_ss(d, a0 + q_off, b0 + k_off, idS, kk > 0 ? 1u : 0u);
                 }
                 tc05::commit(&bar[kSFull + x]);
             }
@@ -370,12 +408,19 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             long long& c = x ? cnt1 : cnt0;
             if (!wait_ok(&bar[kPFull + x], (uint32_t)(c & 1))) return;
             tc05::fence_after();
-            if (lane == 0) {
-                for (int kk = 0; kk < ksteps; ++kk) {
-                    const uint64_t b = tc05::sdesc_sw128(
-                        aV + st * L::kTileBytes + (uint32_t)(kk * 16 * 128), kN * 128, 1024);
-                    tc05::mma_ts(tmem + x * kTileCols + kM, tmem + x * kTileCols + kk * 8, b, idPV,
-                                 (!first || kk > 0) ? 1u : 0u);
+            const uint64_t b0 = dV + (uint64_t)((st * L::kTileBytes) >> 4);
+            const uint32_t a = tmem + x * kTileCols;
+            const uint32_t d = a + kM;
+            if (tc05::elect_one()) {
+                if (ksteps == kN / 16) {
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk)
+                        tc05::mma_ts(d, a + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), idPV,
+                                     (!first || kk > 0) ? 1u : 0u);
+                } else {
+                    for (int kk = 0; kk < ksteps; ++kk)
+                        tc05::mma_ts(d, a + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), idPV,
+                                     (!first || kk > 0) ? 1u : 0u);
                 }
                 tc05::commit(&bar[kPvDone + x]);
             }
@@ -386,7 +431,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const long long it = item_at(rd);
             if (it >= n_items) break;
             Item x;
-            if (!load_item(p, it, pre, max_tiles, x) || !x.valid) continue;
+            if (!load_item(p, it, sc, x) || !x.valid) continue;
             if (x.n_kt[0] > 0 && wait_ok(&bar[kQFull + 0], (uint32_t)(qc0 & 1))) ++qc0;
             if (ok && x.n_kt[1] > 0 && wait_ok(&bar[kQFull + 1], (uint32_t)(qc1 & 1))) ++qc1;
             if (!ok) break;
@@ -397,7 +442,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (x.n_kt[0] > 0) issue_s(0, st, true);
                 if (ok && x.n_kt[1] > 0) issue_s(1, st, true);
                 if (!ok) break;
-                if (lane == 0) tc05::commit(&bar[kKEmpty + st]);
+                if (tc05::elect_one()) tc05::commit(&bar[kKEmpty + st]);
                 __syncwarp();
             }
             for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
@@ -425,22 +470,20 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                // per tile: P.V of this key tile, then S of the next one
                 // both tiles' P.V of this key tile first, then (each once its
                 // own P.V has completed, so that its P is read before S
                 // overwrites it) both tiles' S of the next one: the second P.V
-                // and the first S queue behind running work, so the tensor pipe
-                // does not wait for the issuing thread
+                // and the first S queue behind running work
                 if (kt < x.n_kt[0]) issue_pv(0, st, ksteps, kt == 0);
                 if (ok && kt < x.n_kt[1]) issue_pv(1, st, ksteps, kt == 0);
                 if (!ok) break;
-                if (lane == 0) tc05::commit(&bar[kVEmpty + st]);
+                if (tc05::elect_one()) tc05::commit(&bar[kVEmpty + st]);
                 __syncwarp();
                 if (more) {
                     if (kt + 1 < x.n_kt[0]) issue_s(0, st1, false);
                     if (ok && kt + 1 < x.n_kt[1]) issue_s(1, st1, false);
                     if (!ok) break;
-                    if (lane == 0) tc05::commit(&bar[kKEmpty + st1]);
+                    if (tc05::elect_one()) tc05::commit(&bar[kKEmpty + st1]);
                     __syncwarp();
                 }
                 ++kc;
@@ -448,7 +491,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         // every tensor-core operation issued has completed before the CTA
         // frees tensor memory and exits
-        if (lane == 0) tc05::commit(&bar[kDrain]);
+        if (tc05::elect_one()) tc05::commit(&bar[kDrain]);
         __syncwarp();
         (void)mbar_wait(&bar[kDrain], 0);
     } else {
@@ -470,67 +513,114 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         T* out = reinterpret_cast<T*>(p.out);
         const T* qg = reinterpret_cast<const T*>(p.q);
-        for (long long rd = 0; ok; ++rd) {
-            const long long it = item_at(rd);
-            if (it >= n_items) break;
-            Item x;
-            if (!load_item(p, it, pre, max_tiles, x)) continue;
-            // this warp's tile (plain values: no run-time index into x)
-            const int my_n_kt = t ? x.n_kt[1] : x.n_kt[0];
-            const int my_row_end = t ? x.row_end[1] : x.row_end[0];
-            if (my_n_kt == 0) continue;                    // this tile is past the rows
-            const int row0 = x.row0 + t * kM;
-            const int gr = row0 + r;                       // this thread's row of (seq, g)
-            const bool row_ok = gr < my_row_end;
-            const int last = row_ok ? gr : my_row_end - 1;
-            const int tok = last / p.G;
-            const int head = x.g * p.G + last % p.G;
-            T* orow = out + ((size_t)(x.q0 + tok) * p.H_q + head) * D;
-            if (!x.valid) {
-                if (r == 0 && t == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
-                if (x.n <= p.max_q_len && row_ok)
-                    for (int i = 0; i < D; i += 8)
-                        *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-                continue;
-            }
-            // block ids of the item in range? (the producer skipped bad ones;
-            // each warp checks on its own: no CTA-wide barrier inside the
-            // roles, which a warp that gave up could leave unreached)
-            bool bad = false;
-            const int n_blk = (x.kv_end + p.block_size - 1) / p.block_size;
-            const int32_t* table = p.tables + (long long)x.seq * p.max_blocks;
-            for (int j = lane; j < n_blk; j += 32) {
-                const int id = table[j];
-                bad |= id < 0 || id >= p.num_blocks;
-            }
-            bad = __any_sync(kFull, bad);
-            if (bad && r == 0 && t == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
-            // Q row -> shared memory, 128-byte swizzle
-            {
-                const T* qrow = qg + ((size_t)(x.q0 + tok) * p.H_q + head) * D;
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + c * 8)
-                                     : make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(sQt + (c >> 3) * (kM * 128) + (r >> 3) * 1024 +
-                                              (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+        // this thread's row of an item: position in the (sequence, g) rows,
+        // whether it exists, and its token and query head
+        struct Row {
+            int row0, row_end, n_kt, tok, head;
+            bool ok;
+        };
+        auto row_of = [&](const Item& x) {
+            Row w;
+            w.row0 = x.row0 + t * kM;
+            w.row_end = t ? x.row_end[1] : x.row_end[0];
+            w.n_kt = t ? x.n_kt[1] : x.n_kt[0];
+            const int gr = w.row0 + r;
+            w.ok = gr < w.row_end;
+            const int last = w.ok ? gr : w.row_end - 1;
+            w.tok = last / p.G;
+            w.head = x.g * p.G + last % p.G;
+            return w;
+        };
+        // the next item this tile takes part in; items with a bad length have
+        // their rows zeroed on the way
+        long long rd = 0;
+        auto next_item = [&](Item& x) -> bool {
+            for (;; ++rd) {
+                const long long it = item_at(rd);
+                if (it >= n_items) return false;
+                if (!load_item(p, it, sc, x)) continue;
+                const Row w = row_of(x);
+                if (w.n_kt == 0) continue;                 // this tile is past the rows
+                if (!x.valid) {
+                    if (r == 0 && t == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
+                    if (x.n <= p.max_q_len && w.ok) {
+                        T* orow = out + ((size_t)(x.q0 + w.tok) * p.H_q + w.head) * D;
+                        for (int i = 0; i < D; i += 8)
+                            *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
+                    }
+                    continue;
                 }
+                ++rd;
+                return true;
             }
+        };
+        // this thread's Q row of item x -> shared memory (128-byte swizzle),
+        // without passing through registers; rows past the end are zero
+        auto fetch_q = [&](const Item& x) {
+            const Row w = row_of(x);
+            const T* qrow = qg + ((size_t)(x.q0 + w.tok) * p.H_q + w.head) * D;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                uint8_t* dst = sQt + (c >> 3) * (kM * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                               (((c & 7) ^ (r & 7)) << 4);
+                if (w.ok)
+                    tc05::cp_async16(dst, qrow + c * 8);
+                else
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+            }
+            tc05::cp_async_commit();
+        };
+        // hand the fetched Q rows to the tensor cores
+        auto publish_q = [&]() {
+            tc05::cp_async_wait_all();
             fence_proxy_async_smem();
             tc05::fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bar[kQFull + t]);
+        };
 
-            const int lim = x.base + tok;                  // last visible key of this row
-            const int min_lim = x.base + row0 / p.G;
+        Item nxt;
+        bool have = next_item(nxt);
+        if (have) {
+            fetch_q(nxt);
+            publish_q();
+        }
+        while (have && ok) {
+            const Item x = nxt;
+            const Row w = row_of(x);
+            T* orow = out + ((size_t)(x.q0 + w.tok) * p.H_q + w.head) * D;
+            // block ids of the item in range? (the producer skipped bad ones;
+            // checked here, while the tensor cores compute the first S, each
+            // warp on its own: no CTA-wide barrier inside the roles, which a
+            // warp that gave up could leave unreached)
+            bool bad = false;
+            {
+                const int n_blk = (x.kv_end + p.block_size - 1) / p.block_size;
+                const int32_t* table = p.tables + (long long)x.seq * p.max_blocks;
+                for (int j = lane; j < n_blk; j += 32) {
+                    const int id = table[j];
+                    bad |= id < 0 || id >= p.num_blocks;
+                }
+                bad = __any_sync(kFull, bad);
+                if (bad && r == 0 && t == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
+            }
+            const int lim = x.base + w.tok;                // last visible key of this row
+            const int min_lim = x.base + w.row0 / p.G;
             float m_run = -INFINITY, l_run = 0.f;
-            for (int kt = 0; kt < my_n_kt; ++kt) {
+            bool have_next = false;
+            for (int kt = 0; kt < w.n_kt; ++kt) {
                 if (!wait_ok(&bar[kSFull + t], (uint32_t)(cnt & 1))) break;
                 tc05::fence_after();
-                // pass 1 over S: the largest scaled score of each row (32 columns
-                // at a time: few live registers).  Keys past the row's position
-                // are masked, which only the tile on the diagonal needs; the
-                // scale may be negative, then the smallest raw score counts.
+                if (kt == w.n_kt - 1) {
+                    // the item's last S of this tile is done: its Q rows are no
+                    // longer read, so the next item's can come in
+                    have_next = next_item(nxt);
+                    if (have_next) fetch_q(nxt);
+                }
+                // pass 1 over S: the largest scaled score of each row.  Keys
+                // past the row's position are masked, which only the tile on
+                // the diagonal needs; the scale may be negative, then the
+                // smallest raw score counts.
                 const int k0 = kt * kN;
                 const bool full_tile = k0 + kN - 1 <= min_lim;
                 const bool up = p.q_scale >= 0.f;
@@ -541,13 +631,26 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     tc05::tmem_ld64(t_lane + c * 64, u);
                     const int vis = lim - k0 - c * 64;     // columns j <= vis are visible
                     if (full_tile) {
+                        // eight independent chains, then a tree
+                        float e8[8];
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) e8[a] = ext;
                         if (up) {
 #pragma unroll
-                            for (int j = 0; j < 64; ++j) ext = fmaxf(ext, __uint_as_float(u[j]));
+                            for (int j = 0; j < 64; ++j) e8[j & 7] = fmaxf(e8[j & 7], __uint_as_float(u[j]));
+#pragma unroll
+                            for (int a = 4; a > 0; a >>= 1)
+#pragma unroll
+                                for (int b = 0; b < a; ++b) e8[b] = fmaxf(e8[b], e8[b + a]);
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 64; ++j) ext = fminf(ext, __uint_as_float(u[j]));
+                            for (int j = 0; j < 64; ++j) e8[j & 7] = fminf(e8[j & 7], __uint_as_float(u[j]));
+#pragma unroll
+                            for (int a = 4; a > 0; a >>= 1)
+#pragma unroll
+                                for (int b = 0; b < a; ++b) e8[b] = fminf(e8[b], e8[b + a]);
                         }
+                        ext = e8[0];
                     } else {
 #pragma unroll
                         for (int j = 0; j < 64; ++j) {
@@ -577,7 +680,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 // columns; chunk c's P lands in columns 32 c .. 32 c + 31, all
                 // of them S values already read
                 const float neg_m = -m_new;
-                float rs = 0.f;
+                float rs4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll 1
                 for (int c = 0; c < kN / 64; ++c) {
                     uint32_t u[64];
@@ -588,15 +691,16 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                             uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 32; j += 2) {
-                                const float a = tc05::ex2(fmaf(__uint_as_float(u[h * 32 + j]), p.q_scale, neg_m));
-                                const float b = tc05::ex2(fmaf(__uint_as_float(u[h * 32 + j + 1]), p.q_scale, neg_m));
-                                rs += a + b;
+                                const int jj = h * 32 + j;
+                                const float a = tc05::ex2(fmaf(__uint_as_float(u[jj]), p.q_scale, neg_m));
+                                const float b = tc05::ex2(fmaf(__uint_as_float(u[jj + 1]), p.q_scale, neg_m));
+                                rs4[(j >> 1) & 3] += a + b;
                                 pk[j / 2] = tc::MmaType<T>::pack(a, b);
                             }
                             tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
                         }
                     } else {
-                        const int vis = lim - k0 - c * 64;
+                        const int vis = lim - k0 - c * 64;   // columns j <= vis are visible
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             uint32_t pk[16];
@@ -607,7 +711,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                     ? tc05::ex2(fmaf(__uint_as_float(u[jj]), p.q_scale, neg_m)) : 0.f;
                                 const float b = jj + 1 <= vis
                                     ? tc05::ex2(fmaf(__uint_as_float(u[jj + 1]), p.q_scale, neg_m)) : 0.f;
-                                rs += a + b;
+                                rs4[(j >> 1) & 3] += a + b;
                                 pk[j / 2] = tc::MmaType<T>::pack(a, b);
                             }
                             tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
@@ -615,13 +719,16 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
                 tc05::tmem_st_wait();
-                l_run = l_run * alpha + rs;
+                l_run = l_run * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
                 tc05::fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bar[kPFull + t]);
                 ++cnt;
             }
             if (!ok) break;
+            // the next item's Q goes to the tensor cores before this item's
+            // epilogue, which its first S can then overlap
+            if (have_next) publish_q();
             // epilogue: O / l of the item's last P.V
             if (!wait_ok(&bar[kPvDone + t], (uint32_t)((cnt - 1) & 1))) break;
             tc05::fence_after();
@@ -634,7 +741,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                     for (int j = 0; j < 32; ++j) o[j] = 0u;   // the item's keys were not read
                 }
-                if (row_ok) {
+                if (w.ok) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         uint4 v;
@@ -647,7 +754,10 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
             tc05::fence_before();
+            have = have_next;
         }
+        // a fetch still in flight (after giving up) must land before the CTA exits
+        tc05::cp_async_wait_all();
     }
 
     // every role is done: free tensor memory

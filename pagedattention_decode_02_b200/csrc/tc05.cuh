@@ -194,6 +194,40 @@ __device__ __forceinline__ void commit(uint64_t* bar) {
         : "memory");
 }
 
+// True in exactly one lane of the (converged) warp.  Tensor-core and bulk
+// copy instructions issued under it take operands the whole warp computed,
+// which stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// L2 policy for data that other CTAs read again soon: kept in L2 in
+// preference to other lines.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// 16 bytes global -> shared without passing through registers (both
+// addresses 16-byte aligned); completion by cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 // 2^x on the special-function unit (approximate, subnormal results flushed to
 // zero; 2^-inf = +0).
 __device__ __forceinline__ float ex2(float x) {
