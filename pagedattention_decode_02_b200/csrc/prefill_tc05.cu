@@ -26,9 +26,10 @@
 //              current item is done, and handed to the tensor cores before
 //              the current item's output is written, so that the next S runs
 //              under that epilogue;
-//   warp 8     producer: 128-key K and V tiles through two-deep rings, each
-//              tile 16-key stages of 2-D TMA boxes (128-byte swizzle) read
-//              through the block table from this GPU's own pool;
+//   warps 8, 10  producers of the 128-key K tiles and V tiles, each through
+//              a two-deep ring: 16-key stages of 2-D TMA boxes (128-byte
+//              swizzle) read through the block table from this GPU's own
+//              pool, every lane issuing its own boxes;
 //   warp 9     MMA: one thread issues, per tile x, S_x = Q_x K^T (M 128,
 //              N 128, K = d; both operands in shared memory) and O_x += P_x V
 //              (M 128, N = d, K 128; P from tensor memory, V from shared memory
@@ -59,9 +60,10 @@ constexpr int kTiles = 2;            // query tiles per work item
 constexpr int kRows = kTiles * kM;   // rows per work item
 constexpr int kN = 128;              // keys per K/V tile
 constexpr int kRing = 2;             // K ring and V ring depth
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;     // K tiles
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 10 * 32;
+constexpr int kProducerVWarp = 10;   // V tiles
+constexpr int kThreads = 11 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTileCols = 256;  // per query tile: S (P) then O
 constexpr float kRescaleLog2 = 8.f;  // keep a stale maximum while the new one is within 2^8
@@ -275,8 +277,8 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         return round * G0 + ((round & 1) ? (G0 - 1 - blockIdx.x) : blockIdx.x);
     };
 
-    if (warp == kProducerWarp) {
-        // ------------------------------------------------------------ producer
+    if (warp == kProducerWarp || warp == kProducerVWarp) {
+        // ----------------------------------------------------------- producers
         // the other work items of the same (sequence, KV head), running on
         // other SMs at about the same time, read the same K/V tiles: keep them
         // in L2
@@ -284,7 +286,8 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int bs = p.block_size;
         const int rpb = bs < 16 ? bs : 16;          // rows per TMA box
         const int boxes = kN / rpb;                  // boxes per half-tile (<= 128)
-        long long armed_k = 0, armed_v = 0;          // K, V tiles whose barrier was armed
+        const int kv = warp == kProducerVWarp ? 1 : 0;   // this warp's tiles: K or V
+        long long armed = 0;                         // tiles whose barrier was armed
         bool ok = true;
         for (long long rd = 0; ok; ++rd) {
             const long long it = item_at(rd);
@@ -294,10 +297,9 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int32_t* table = p.tables + (long long)x.seq * p.max_blocks;
             for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
                 const int a0 = kt * kN;
-                // the block ids of this lane's boxes (l, l + 32, ...), read once
-                // for K and V, before waiting for the slots; -1: past the end
-                // or out of range (skipped; the softmax warps zero such an
-                // item's output)
+                // the block ids of this lane's boxes (l, l + 32, ...), read
+                // before waiting for the slot; -1: past the end or out of range
+                // (skipped; the softmax warps zero such an item's output)
                 int ids[4];
                 uint32_t good = 0;
 #pragma unroll
@@ -313,8 +315,8 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     good += id >= 0 ? 1u : 0u;
                 }
                 good = __reduce_add_sync(kFull, good);
-                for (int kv = 0; kv < 2; ++kv) {
-                    const long long j = kv ? armed_v : armed_k;
+                {
+                    const long long j = armed;
                     const int st = (int)(j % kRing);
                     if (j >= kRing) {
                         const bool w = mbar_wait(&bar[(kv ? kVEmpty : kKEmpty) + st],
@@ -330,7 +332,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     if (tc05::elect_one())
                         mbar_arrive_expect_tx(full, good * (uint32_t)(rpb * 128 * HALVES));
                     __syncwarp();
-                    (kv ? armed_v : armed_k) = j + 1;
+                    armed = j + 1;
                     uint8_t* dst = (kv ? sV : sK) + st * L::kTileBytes;
                     const CUtensorMap* map = kv ? &tmap_v : &tmap_k;
                     // every lane issues its own boxes: the copies' issue
@@ -350,15 +352,12 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
         }
-        // no copy may outlive the CTA: the last armed tiles of each ring may
+        // no copy may outlive the CTA: the last armed tiles of this ring may
         // still be in flight (an earlier tile's slot was reused only after the
         // MMA warp had waited for it to land)
-        for (int kv = 0; kv < 2; ++kv) {
-            const long long n = kv ? armed_v : armed_k;
-            for (long long j = n - kRing < 0 ? 0 : n - kRing; j < n; ++j)
-                (void)mbar_wait(&bar[(kv ? kVFull : kKFull) + (int)(j % kRing)],
-                                (uint32_t)((j / kRing) & 1));
-        }
+        for (long long j = armed - kRing < 0 ? 0 : armed - kRing; j < armed; ++j)
+            (void)mbar_wait(&bar[(kv ? kVFull : kKFull) + (int)(j % kRing)],
+                            (uint32_t)((j / kRing) & 1));
     } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------------- MMA
         constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
