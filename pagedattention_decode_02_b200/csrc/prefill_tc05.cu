@@ -27,15 +27,16 @@
 //              the current item's output is written, so that the next S runs
 //              under that epilogue;
 //   warps 8, 10  producers of the 128-key K tiles and V tiles, each through
-//              a two-deep ring: 16-key stages of 2-D TMA boxes (128-byte
-//              swizzle) read through the block table from this GPU's own
-//              pool, every lane issuing its own boxes;
+//              a two-deep ring: 2-D TMA boxes (128-byte swizzle) of up to 16
+//              rows of one block and one 64-column half, read through the
+//              block table from this GPU's own pool, every lane issuing its
+//              own boxes;
 //   warp 9     MMA: one thread issues, per tile x, S_x = Q_x K^T (M 128,
 //              N 128, K = d; both operands in shared memory) and O_x += P_x V
 //              (M 128, N = d, K 128; P from tensor memory, V from shared memory
 //              as an MN-major operand), completion by tcgen05.commit.  Per key
-//              tile: P_0 V, P_1 V, then S_0 and S_1 of the next key tile (each
-//              after its tile's P.V completed: S overwrites P).
+//              tile: P_0 V, S_0 of the next key tile, P_1 V, S_1 of the next
+//              (each S after its tile's P.V completed: S overwrites P).
 // Tensor memory: tile x owns columns [256 x, 256 x + 128) for S (P packed
 // into the first 64 of them) and [256 x + 128, 256 x + 128 + d) for O.
 // Every wait is bounded; a wait that gives up sets PKV_DEVERR_TIMEOUT, the CTA
@@ -59,7 +60,8 @@ constexpr int kM = 128;              // rows per query tile (tensor-memory lanes
 constexpr int kTiles = 2;            // query tiles per work item
 constexpr int kRows = kTiles * kM;   // rows per work item
 constexpr int kN = 128;              // keys per K/V tile
-constexpr int kRing = 2;             // K ring and V ring depth
+constexpr int kRingK = 2;            // K ring depth
+constexpr int kRingV = 2;            // V ring depth
 constexpr int kProducerWarp = 8;     // K tiles
 constexpr int kMmaWarp = 9;
 constexpr int kProducerVWarp = 10;   // V tiles
@@ -74,10 +76,10 @@ constexpr int kMaxSchedSeqs = 1024;
 
 enum Bar {
     kKFull = 0,
-    kKEmpty = kKFull + kRing,
-    kVFull = kKEmpty + kRing,
-    kVEmpty = kVFull + kRing,
-    kSFull = kVEmpty + kRing,        // per tile: S_x computed
+    kKEmpty = kKFull + kRingK,
+    kVFull = kKEmpty + kRingK,
+    kVEmpty = kVFull + kRingV,
+    kSFull = kVEmpty + kRingV,        // per tile: S_x computed
     kPFull = kSFull + kTiles,        // per tile: P_x written, O_x rescaled (4 warps)
     kPvDone = kPFull + kTiles,       // per tile: O_x += P_x V done
     kQFull = kPvDone + kTiles,       // per tile: Q_x rows written (4 warps)
@@ -92,8 +94,8 @@ struct Layout5 {
     static constexpr int kTileBytes = kHalves * kN * 128;// K or V tile [half][key][128 B]
     static constexpr int kQ = 0;                          // [kTiles][kQBytes]
     static constexpr int kK = kQ + kTiles * kQBytes;
-    static constexpr int kV = kK + kRing * kTileBytes;
-    static constexpr int kBars = kV + kRing * kTileBytes;
+    static constexpr int kV = kK + kRingK * kTileBytes;
+    static constexpr int kBars = kV + kRingV * kTileBytes;
     // int prefix[kMaxSchedSeqs + 1], q_starts[kMaxSchedSeqs + 1], lens[kMaxSchedSeqs],
     // partial[kThreads]
     static constexpr int kSched = kBars + kNumBars * 8 + 16;
@@ -208,9 +210,11 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int lane = tid & 31;
 
     if (tid == 0) {
-        for (int i = 0; i < kRing; ++i) {
+        for (int i = 0; i < kRingK; ++i) {
             mbar_init(&bar[kKFull + i], 1);
             mbar_init(&bar[kKEmpty + i], 1);
+        }
+        for (int i = 0; i < kRingV; ++i) {
             mbar_init(&bar[kVFull + i], 1);
             mbar_init(&bar[kVEmpty + i], 1);
         }
@@ -287,6 +291,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int rpb = bs < 16 ? bs : 16;          // rows per TMA box
         const int boxes = kN / rpb;                  // boxes per half-tile (<= 128)
         const int kv = warp == kProducerVWarp ? 1 : 0;   // this warp's tiles: K or V
+        const int ring = kv ? kRingV : kRingK;
         long long armed = 0;                         // tiles whose barrier was armed
         bool ok = true;
         for (long long rd = 0; ok; ++rd) {
@@ -317,10 +322,10 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 good = __reduce_add_sync(kFull, good);
                 {
                     const long long j = armed;
-                    const int st = (int)(j % kRing);
-                    if (j >= kRing) {
+                    const int st = (int)(j % ring);
+                    if (j >= ring) {
                         const bool w = mbar_wait(&bar[(kv ? kVEmpty : kKEmpty) + st],
-                                                 (uint32_t)(((j / kRing) - 1) & 1), p.wait_ns);
+                                                 (uint32_t)(((j / ring) - 1) & 1), p.wait_ns);
                         if (!__all_sync(kFull, w) || *abort_flag) {
                             if (lane == 0 && !w) report_error(p.err, PKV_DEVERR_TIMEOUT);
                             if (lane == 0) *abort_flag = 1;
@@ -355,9 +360,9 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // no copy may outlive the CTA: the last armed tiles of this ring may
         // still be in flight (an earlier tile's slot was reused only after the
         // MMA warp had waited for it to land)
-        for (long long j = armed - kRing < 0 ? 0 : armed - kRing; j < armed; ++j)
-            (void)mbar_wait(&bar[(kv ? kVFull : kKFull) + (int)(j % kRing)],
-                            (uint32_t)((j / kRing) & 1));
+        for (long long j = armed - ring < 0 ? 0 : armed - ring; j < armed; ++j)
+            (void)mbar_wait(&bar[(kv ? kVFull : kKFull) + (int)(j % ring)],
+                            (uint32_t)((j / ring) & 1));
     } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------------- MMA
         constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -383,10 +388,14 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             return ok;
         };
         // S_x of a key tile whose K sits in ring slot st
-        auto issue_s = [&](int x, int st, bool first) {
-            // this tile's previous P.V is done: its P (in S_x's columns) was read
+        auto issue_s = [&](int x, int st) {
+            // this tile's last P.V (of this item or, at its first key tile, of
+            // the previous one) is done: its P, in S_x's columns, was read.
+            // Tensor-core operations on different accumulators are not
+            // ordered among themselves, so issue order alone does not keep S
+            // from overwriting P early.
             const long long c = x ? cnt1 : cnt0;
-            if (!first && !wait_ok(&bar[kPvDone + x], (uint32_t)((c - 1) & 1))) return;
+            if (c > 0 && !wait_ok(&bar[kPvDone + x], (uint32_t)((c - 1) & 1))) return;
             tc05::fence_after();
             const uint64_t a0 = dQ + (uint64_t)((x * L::kQBytes) >> 4);
             const uint64_t b0 = dK + (uint64_t)((st * L::kTileBytes) >> 4);
@@ -436,20 +445,20 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (!ok) break;
             // key tile 0: S_0, S_1
             {
-                const int st = (int)(kc % kRing);
-                if (!wait_ok(&bar[kKFull + st], (uint32_t)((kc / kRing) & 1))) break;
-                if (x.n_kt[0] > 0) issue_s(0, st, true);
-                if (ok && x.n_kt[1] > 0) issue_s(1, st, true);
+                const int st = (int)(kc % kRingK);
+                if (!wait_ok(&bar[kKFull + st], (uint32_t)((kc / kRingK) & 1))) break;
+                if (x.n_kt[0] > 0) issue_s(0, st);
+                if (ok && x.n_kt[1] > 0) issue_s(1, st);
                 if (!ok) break;
                 if (tc05::elect_one()) tc05::commit(&bar[kKEmpty + st]);
                 __syncwarp();
             }
             for (int kt = 0; kt < x.n_kt_all && ok; ++kt) {
-                const int st = (int)(kc % kRing);
-                const int st1 = (int)((kc + 1) % kRing);
+                const int st = (int)(kc % kRingV);          // V of this key tile
+                const int st1 = (int)((kc + 1) % kRingK);   // K of the next
                 const bool more = kt + 1 < x.n_kt_all;
-                if (!wait_ok(&bar[kVFull + st], (uint32_t)((kc / kRing) & 1))) break;
-                if (more && !wait_ok(&bar[kKFull + st1], (uint32_t)(((kc + 1) / kRing) & 1))) break;
+                if (!wait_ok(&bar[kVFull + st], (uint32_t)((kc / kRingV) & 1))) break;
+                if (more && !wait_ok(&bar[kKFull + st1], (uint32_t)(((kc + 1) / kRingK) & 1))) break;
                 tc05::fence_after();
                 const int keys = min(kN, x.kv_end - kt * kN);
                 const int ksteps = (keys + 15) >> 4;
@@ -469,18 +478,18 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                // both tiles' P.V of this key tile first, then (each once its
-                // own P.V has completed, so that its P is read before S
-                // overwrites it) both tiles' S of the next one: the second P.V
-                // and the first S queue behind running work
+                // per tile, P.V of this key tile and then S of the next: tile
+                // 0's S does not wait for tile 1's P, so the two softmax
+                // groups fall half a step apart and take turns on the
+                // exponential units while the tensor cores serve the other
                 if (kt < x.n_kt[0]) issue_pv(0, st, ksteps, kt == 0);
+                if (ok && more && kt + 1 < x.n_kt[0]) issue_s(0, st1);
                 if (ok && kt < x.n_kt[1]) issue_pv(1, st, ksteps, kt == 0);
                 if (!ok) break;
                 if (tc05::elect_one()) tc05::commit(&bar[kVEmpty + st]);
                 __syncwarp();
                 if (more) {
-                    if (kt + 1 < x.n_kt[0]) issue_s(0, st1, false);
-                    if (ok && kt + 1 < x.n_kt[1]) issue_s(1, st1, false);
+                    if (kt + 1 < x.n_kt[1]) issue_s(1, st1);
                     if (!ok) break;
                     if (tc05::elect_one()) tc05::commit(&bar[kKEmpty + st1]);
                     __syncwarp();
@@ -680,6 +689,11 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 // of them S values already read
                 const float neg_m = -m_new;
                 float rs4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+                // the full tile's scaling and sums two lanes at a time (packed
+                // f32x2 FMA and add: half the issue slots)
+                const float2 sc2 = make_float2(p.q_scale, p.q_scale);
+                const float2 nm2 = make_float2(neg_m, neg_m);
+                float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 1
                 for (int c = 0; c < kN / 64; ++c) {
                     uint32_t u[64];
@@ -691,10 +705,12 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                             for (int j = 0; j < 32; j += 2) {
                                 const int jj = h * 32 + j;
-                                const float a = tc05::ex2(fmaf(__uint_as_float(u[jj]), p.q_scale, neg_m));
-                                const float b = tc05::ex2(fmaf(__uint_as_float(u[jj + 1]), p.q_scale, neg_m));
-                                rs4[(j >> 1) & 3] += a + b;
-                                pk[j / 2] = tc::MmaType<T>::pack(a, b);
+                                const float2 x2 = __ffma2_rn(
+                                    make_float2(__uint_as_float(u[jj]), __uint_as_float(u[jj + 1])),
+                                    sc2, nm2);
+                                const float2 e = make_float2(tc05::ex2(x2.x), tc05::ex2(x2.y));
+                                rs2[(j >> 1) & 1] = __fadd2_rn(rs2[(j >> 1) & 1], e);
+                                pk[j / 2] = tc::MmaType<T>::pack(e.x, e.y);
                             }
                             tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
                         }
@@ -718,7 +734,8 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                 }
                 tc05::tmem_st_wait();
-                l_run = l_run * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+                l_run = l_run * alpha + (((rs4[0] + rs4[1]) + (rs4[2] + rs4[3])) +
+                                         ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)));
                 tc05::fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&bar[kPFull + t]);

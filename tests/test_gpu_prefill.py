@@ -76,6 +76,22 @@ def test_prefill_small(dt, d, bs, hq, hkv, kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("bs", [8, 64, 128, 256])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_block_sizes(bs, d, kernel):
+    # one TMA box per block of up to 128 rows (a 256-token block takes two),
+    # over histories of several 128-key tiles with ragged ends
+    cfg = small("llama2_70b", n_q_heads=8, n_kv_heads=2, head_dim=d, kv_dtype="bf16",
+                q_dtype="bf16", block_size=bs, batch=3, lengths=("uniform", 100, 700))
+    side = setup_config(cfg, seed=bs + d)
+    hist = [side.orc.bm.lengths[s] for s in side.seqs]
+    n = [int(h) if i == 0 else max(1, int(h) // 3) for i, h in enumerate(hist)]
+    gpu, ref = run_prefill(side, n, kernel=kernel)
+    for g, r in zip(gpu, ref):
+        compare_out(g, r, "bf16")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("hq,hkv,d", [(64, 8, 128), (71, 1, 64), (40, 40, 128), (8, 2, 64)])
 def test_prefill_long_prompts(hq, hkv, d, kernel):
     # several row tiles per (sequence, KV head) and several key tiles
