@@ -496,8 +496,11 @@ pkv_status paged_decode_attention_static(pkv_pool* pool, const void* d_q, pkv_dt
  *   n_i > c_i or n_i > max_q_len sets PKV_DEVERR_CONTEXT_LEN (that sequence's
  *   rows are zero where the grid covers them); a block id outside
  *   [0, num_blocks) sets PKV_DEVERR_BLOCK_ID and zeroes the affected work
- *   item's rows (128 rows with the tcgen05 kernel, 64 with mma.sync).  No
- *   workspace.  Runs the tcgen05 kernel (see paged_prefill_attention_ex).
+ *   item's rows (256 rows with the tcgen05 kernel, 64 with mma.sync).  No
+ *   workspace: the tcgen05 kernel's work counters live in the pool (one pair
+ *   per launch in flight, taken in turn from 64), so at most 64 prompt
+ *   launches on one pool may run at the same time.  Runs the tcgen05 kernel
+ *   (see paged_prefill_attention_ex).
  *   Errors: INVALID_ARG, CUDA. */
 pkv_status paged_prefill_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_dtype,
                                    const int32_t* d_q_starts, int max_q_len,
@@ -507,9 +510,10 @@ pkv_status paged_prefill_attention(pkv_pool* pool, const void* d_q, pkv_dtype q_
 
 /* Kernel selection for paged_prefill_attention_ex. */
 #define PKV_PREFILL_AUTO 0         /* PKV_PREFILL_TCGEN05 */
-#define PKV_PREFILL_TCGEN05 1      /* fifth-generation tensor cores: 128 query rows per work item,
-                                      S = Q K^T and O += P V by tcgen05.mma into tensor memory, one
-                                      persistent CTA per SM taking the heaviest items first */
+#define PKV_PREFILL_TCGEN05 1      /* fifth-generation tensor cores: 256 query rows (two 128-row
+                                      tiles) per work item, S = Q K^T and O += P V by tcgen05.mma
+                                      into tensor memory, one persistent CTA per SM claiming items
+                                      from a global counter (each sequence's heaviest first) */
 #define PKV_PREFILL_MMA_SYNC 2     /* warp-level mma.sync m16n8k16, register accumulators, one CTA
                                       per 64 query rows */
 

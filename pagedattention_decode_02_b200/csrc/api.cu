@@ -181,8 +181,11 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
             }
             p->owns_buffers = true;
         }
-        if (cudaMalloc(&p->d_err, sizeof(uint32_t)) != cudaSuccess ||
-            cudaMemset(p->d_err, 0, sizeof(uint32_t)) != cudaSuccess) {
+        // the error word, then (256 bytes in) the prompt kernel's counters
+        constexpr size_t kSchedOff = 256;
+        const size_t err_bytes = kSchedOff + 2 * sizeof(unsigned long long) * pkv_pool::kPrefillSlots;
+        if (cudaMalloc(&p->d_err, err_bytes) != cudaSuccess ||
+            cudaMemset(p->d_err, 0, err_bytes) != cudaSuccess) {
             if (p->owns_buffers) {
                 cudaFree(p->k);
                 cudaFree(p->v);
@@ -191,6 +194,8 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
             delete p;
             return PKV_ERR_CUDA;
         }
+        p->d_sched = reinterpret_cast<unsigned long long*>(reinterpret_cast<uint8_t*>(p->d_err) +
+                                                           kSchedOff);
         pkv::pool_init_device_extras(p);
         // the no-allocation decode call's scratch array: placed on this device
         // now, while allocating is allowed (a failure here is not fatal; that
@@ -525,6 +530,7 @@ pkv_status paged_prefill_attention_ex(pkv_pool* p, const void* q, pkv_dtype q_dt
     pp.max_q_len = max_q_len;
     pp.q_scale = scale * 1.4426950408889634f;
     pp.wait_ns = p->wait_ns;
+    pp.sched = p->d_sched + 2 * (p->prefill_seq.fetch_add(1) % pkv_pool::kPrefillSlots);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const cudaError_t e = kernel == PKV_PREFILL_MMA_SYNC ? pkv::launch_prefill(pp, p, st)
                                                          : pkv::launch_prefill_tc05(pp, p, st);

@@ -63,6 +63,9 @@ struct PrefillParams {
     int max_q_len;             // >= every n_i (sizes the grid)
     float q_scale;             // scale * log2(e)
     unsigned long long wait_ns;// budget of the main loops' waits (the pool's)
+    // the tcgen05 kernel's work counters {next item, CTAs done}: zero at the
+    // launch, zero again after it (its last CTA resets them)
+    unsigned long long* sched;
 };
 bool prefill_supported(const pkv_pool* pool, int q_dtype);
 // the mma.sync kernel (m16n8k16, register accumulators)

@@ -1,6 +1,7 @@
 // The pool object behind the opaque pkv_pool handle.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -25,6 +26,12 @@ struct pkv_pool {
     uint8_t* v = nullptr;
     size_t bytes = 0;       // bytes of one of the two buffers
     uint32_t* d_err = nullptr;
+    // work counters of the prompt kernel's dynamic schedule: kPrefillSlots
+    // pairs {next item, CTAs done}, one pair per launch in flight (launch i
+    // takes pair i % kPrefillSlots); each launch's last CTA zeroes its pair
+    static constexpr int kPrefillSlots = 64;
+    unsigned long long* d_sched = nullptr;
+    std::atomic<unsigned> prefill_seq{0};
     // budget of the kernels' main-loop waits on a copy (pkv_set_wait_budget)
     unsigned long long wait_ns = 2000000000ull;
     pkv::BlockManager bm;

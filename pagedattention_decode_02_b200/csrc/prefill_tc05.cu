@@ -13,9 +13,9 @@
 // (token, query head of the group) pairs in token-major order.  Items are
 // ordered group by group - all items of one (sequence, g) next to each other,
 // its last rows (the most keys) first - so that the CTAs working at the same
-// time re-read the same K/V from L2; one persistent CTA per SM takes them in a
-// snake order (forward in even rounds, backward in odd ones), which evens out
-// the decreasing item sizes.  Per CTA:
+// time re-read the same K/V from L2; one persistent CTA per SM claims them in
+// that order from a global counter, one at a time, so that every CTA finishes
+// within about one item of the others.  Per CTA:
 //   warps 0-3, 4-7  softmax of tile 0 and tile 1: read each score tile
 //              S = Q K^T from tensor memory (one row per thread), mask
 //              causally, online softmax in base 2, write P (f16/bf16) back
@@ -26,7 +26,9 @@
 //              current item is done, and handed to the tensor cores before
 //              the current item's output is written, so that the next S runs
 //              under that epilogue;
-//   warps 8, 10  producers of the 128-key K tiles and V tiles, each through
+//   warps 8, 10  producers of the 128-key K tiles and V tiles (warp 8 also
+//              claims the items and hands their indices to every role through
+//              a small shared-memory ring), each through
 //              a two-deep ring: 2-D TMA boxes (128-byte swizzle) of up to 16
 //              rows of one block and one 64-column half, read through the
 //              block table from this GPU's own pool, every lane issuing its
@@ -73,6 +75,12 @@ constexpr unsigned kFull = 0xffffffffu;
 // sequences for which the group-major order and shared copies of q_starts
 // and context lengths are kept in shared memory
 constexpr int kMaxSchedSeqs = 1024;
+// Work items are claimed at run time from a global counter (one claim per
+// item, in the group-major order): the K producer claims and publishes each
+// item index through a ring of kItemRing shared-memory slots, which the V
+// producer, the MMA warp and the eight softmax warps each read.
+constexpr int kItemRing = 4;
+constexpr int kItemReaders = 10;
 
 enum Bar {
     kKFull = 0,
@@ -83,7 +91,9 @@ enum Bar {
     kPFull = kSFull + kTiles,        // per tile: P_x written, O_x rescaled (4 warps)
     kPvDone = kPFull + kTiles,       // per tile: O_x += P_x V done
     kQFull = kPvDone + kTiles,       // per tile: Q_x rows written (4 warps)
-    kDrain = kQFull + kTiles,
+    kItemFull = kQFull + kTiles,     // per ring slot: item index written
+    kItemEmpty = kItemFull + kItemRing,   // per ring slot: read by every reader
+    kDrain = kItemEmpty + kItemRing,
     kNumBars = kDrain + 1
 };
 
@@ -98,7 +108,8 @@ struct Layout5 {
     static constexpr int kBars = kV + kRingV * kTileBytes;
     // int prefix[kMaxSchedSeqs + 1], q_starts[kMaxSchedSeqs + 1], lens[kMaxSchedSeqs],
     // partial[kThreads]
-    static constexpr int kSched = kBars + kNumBars * 8 + 16;
+    static constexpr int kItems = kBars + kNumBars * 8 + 16;   // long long [kItemRing]
+    static constexpr int kSched = kItems + kItemRing * 8;
     static constexpr int kEnd = kSched + (3 * kMaxSchedSeqs + 2 + kThreads) * 4;
     // at least 116 KB, so that a second CTA never shares an SM (each CTA
     // takes all 512 tensor-memory columns)
@@ -200,6 +211,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile long long* items = reinterpret_cast<volatile long long*>(sm + L::kItems);
     int* prefix = reinterpret_cast<int*>(sm + L::kSched);
     int* qs_c = prefix + kMaxSchedSeqs + 1;
     int* len_c = qs_c + kMaxSchedSeqs + 1;
@@ -223,6 +235,10 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mbar_init(&bar[kPFull + t], 4);
             mbar_init(&bar[kPvDone + t], 1);
             mbar_init(&bar[kQFull + t], 4);
+        }
+        for (int i = 0; i < kItemRing; ++i) {
+            mbar_init(&bar[kItemFull + i], 1);
+            mbar_init(&bar[kItemEmpty + i], kItemReaders);
         }
         mbar_init(&bar[kDrain], 1);
         *abort_flag = 0;
@@ -275,11 +291,6 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const Sched sc{grouped ? prefix : nullptr, grouped ? qs_c : p.q_starts,
                    grouped ? len_c : p.lens, max_tiles};
     const uint32_t tmem = *tmem_slot;
-    // snake order over the persistent CTAs
-    const long long G0 = gridDim.x;
-    auto item_at = [&](long long round) -> long long {
-        return round * G0 + ((round & 1) ? (G0 - 1 - blockIdx.x) : blockIdx.x);
-    };
 
     if (warp == kProducerWarp || warp == kProducerVWarp) {
         // ----------------------------------------------------------- producers
@@ -294,8 +305,43 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int ring = kv ? kRingV : kRingK;
         long long armed = 0;                         // tiles whose barrier was armed
         bool ok = true;
-        for (long long rd = 0; ok; ++rd) {
-            const long long it = item_at(rd);
+        auto wait_ok = [&](uint64_t* b, uint32_t ph) {
+            const bool w = mbar_wait(b, ph, p.wait_ns);
+            if (!__all_sync(kFull, w) || *abort_flag) {
+                if (lane == 0 && !w) report_error(p.err, PKV_DEVERR_TIMEOUT);
+                if (lane == 0) *abort_flag = 1;
+                ok = false;
+            }
+            return ok;
+        };
+        // the K producer's claim of the item after the one it publishes next:
+        // the atomic's round trip overlaps a whole item's loads
+        unsigned long long ahead = 0;
+        if (kv == 0 && lane == 0) ahead = atomicAdd(p.sched, 1ull);
+        for (long long kn = 0; ok; ++kn) {
+            const int s_it = (int)(kn % kItemRing);
+            long long it;
+            if (kv == 0) {
+                // publish this CTA's next item (n_items: no more), claim the
+                // one after it
+                if (kn >= kItemRing &&
+                    !wait_ok(&bar[kItemEmpty + s_it], (uint32_t)(((kn / kItemRing) - 1) & 1)))
+                    break;
+                unsigned long long c = 0;
+                if (lane == 0) {
+                    c = ahead;
+                    if (c < (unsigned long long)n_items) ahead = atomicAdd(p.sched, 1ull);
+                    else c = (unsigned long long)n_items;
+                    items[s_it] = (long long)c;
+                    tc::mbar_arrive(&bar[kItemFull + s_it]);
+                }
+                it = (long long)__shfl_sync(kFull, c, 0);
+            } else {
+                if (!wait_ok(&bar[kItemFull + s_it], (uint32_t)((kn / kItemRing) & 1))) break;
+                it = items[s_it];
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bar[kItemEmpty + s_it]);
+            }
             if (it >= n_items) break;
             Item x;
             if (!load_item(p, it, sc, x) || !x.valid) continue;
@@ -323,16 +369,9 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 {
                     const long long j = armed;
                     const int st = (int)(j % ring);
-                    if (j >= ring) {
-                        const bool w = mbar_wait(&bar[(kv ? kVEmpty : kKEmpty) + st],
-                                                 (uint32_t)(((j / ring) - 1) & 1), p.wait_ns);
-                        if (!__all_sync(kFull, w) || *abort_flag) {
-                            if (lane == 0 && !w) report_error(p.err, PKV_DEVERR_TIMEOUT);
-                            if (lane == 0) *abort_flag = 1;
-                            ok = false;
-                            break;
-                        }
-                    }
+                    if (j >= ring && !wait_ok(&bar[(kv ? kVEmpty : kKEmpty) + st],
+                                              (uint32_t)(((j / ring) - 1) & 1)))
+                        break;
                     uint64_t* full = &bar[(kv ? kVFull : kKFull) + st];
                     if (tc05::elect_one())
                         mbar_arrive_expect_tx(full, good * (uint32_t)(rpb * 128 * HALVES));
@@ -435,8 +474,12 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             __syncwarp();
             ++c;
         };
-        for (long long rd = 0; ok; ++rd) {
-            const long long it = item_at(rd);
+        for (long long kn = 0; ok; ++kn) {
+            const int s_it = (int)(kn % kItemRing);
+            if (!wait_ok(&bar[kItemFull + s_it], (uint32_t)((kn / kItemRing) & 1))) break;
+            const long long it = items[s_it];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bar[kItemEmpty + s_it]);
             if (it >= n_items) break;
             Item x;
             if (!load_item(p, it, sc, x) || !x.valid) continue;
@@ -541,11 +584,24 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
         // the next item this tile takes part in; items with a bad length have
         // their rows zeroed on the way
-        long long rd = 0;
-        auto next_item = [&](Item& x) -> bool {
-            for (;; ++rd) {
-                const long long it = item_at(rd);
-                if (it >= n_items) return false;
+        // 1: the next item, 0: no more (or gave up), -1: not published yet
+        // (only without blocking).  Inside a key step this never blocks: the
+        // K producer publishes the next item only after the MMA warp issued
+        // this item's S tiles, which may wait for this step's P.
+        long long kn = 0;
+        auto next_item = [&](Item& x, bool block) -> int {
+            for (;; ++kn) {
+                const int s_it = (int)(kn % kItemRing);
+                const uint32_t ph = (uint32_t)((kn / kItemRing) & 1);
+                if (!block) {
+                    if (!__all_sync(kFull, mbar_test_wait(&bar[kItemFull + s_it], ph))) return -1;
+                } else if (!wait_ok(&bar[kItemFull + s_it], ph)) {
+                    return 0;
+                }
+                const long long it = items[s_it];
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&bar[kItemEmpty + s_it]);
+                if (it >= n_items) return 0;
                 if (!load_item(p, it, sc, x)) continue;
                 const Row w = row_of(x);
                 if (w.n_kt == 0) continue;                 // this tile is past the rows
@@ -558,8 +614,8 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     }
                     continue;
                 }
-                ++rd;
-                return true;
+                ++kn;
+                return 1;
             }
         };
         // this thread's Q row of item x -> shared memory (128-byte swizzle),
@@ -588,7 +644,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
         };
 
         Item nxt;
-        bool have = next_item(nxt);
+        bool have = next_item(nxt, true) == 1;
         if (have) {
             fetch_q(nxt);
             publish_q();
@@ -615,15 +671,15 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int lim = x.base + w.tok;                // last visible key of this row
             const int min_lim = x.base + w.row0 / p.G;
             float m_run = -INFINITY, l_run = 0.f;
-            bool have_next = false;
+            int nx = 0;
             for (int kt = 0; kt < w.n_kt; ++kt) {
                 if (!wait_ok(&bar[kSFull + t], (uint32_t)(cnt & 1))) break;
                 tc05::fence_after();
                 if (kt == w.n_kt - 1) {
                     // the item's last S of this tile is done: its Q rows are no
                     // longer read, so the next item's can come in
-                    have_next = next_item(nxt);
-                    if (have_next) fetch_q(nxt);
+                    nx = next_item(nxt, false);
+                    if (nx == 1) fetch_q(nxt);
                 }
                 // pass 1 over S: the largest scaled score of each row.  Keys
                 // past the row's position are masked, which only the tile on
@@ -633,7 +689,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const bool full_tile = k0 + kN - 1 <= min_lim;
                 const bool up = p.q_scale >= 0.f;
                 float ext = up ? -INFINITY : INFINITY;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < kN / 64; ++c) {
                     uint32_t u[64];
                     tc05::tmem_ld64(t_lane + c * 64, u);
@@ -673,7 +729,7 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 // O of this tile is idle: the MMA warp issued this S only after
                 // the previous P.V had completed
                 if (kt > 0 && __any_sync(kFull, m_new != m_run)) {
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
                         tc05::tmem_ld32(t_lane + kM + c * 32, o);
@@ -695,43 +751,32 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const float2 nm2 = make_float2(neg_m, neg_m);
                 float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 1
-                for (int c = 0; c < kN / 64; ++c) {
-                    uint32_t u[64];
-                    tc05::tmem_ld64(t_lane + c * 64, u);
+                for (int c = 0; c < kN / 32; ++c) {
+                    uint32_t u[32];
+                    tc05::tmem_ld32(t_lane + c * 32, u);
+                    uint32_t pk[16];
                     if (full_tile) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t pk[16];
-#pragma unroll
-                            for (int j = 0; j < 32; j += 2) {
-                                const int jj = h * 32 + j;
-                                const float2 x2 = __ffma2_rn(
-                                    make_float2(__uint_as_float(u[jj]), __uint_as_float(u[jj + 1])),
-                                    sc2, nm2);
-                                const float2 e = make_float2(tc05::ex2(x2.x), tc05::ex2(x2.y));
-                                rs2[(j >> 1) & 1] = __fadd2_rn(rs2[(j >> 1) & 1], e);
-                                pk[j / 2] = tc::MmaType<T>::pack(e.x, e.y);
-                            }
-                            tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
+                        for (int j = 0; j < 32; j += 2) {
+                            const float2 x2 = __ffma2_rn(
+                                make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])), sc2, nm2);
+                            const float2 e = make_float2(tc05::ex2(x2.x), tc05::ex2(x2.y));
+                            rs2[(j >> 1) & 1] = __fadd2_rn(rs2[(j >> 1) & 1], e);
+                            pk[j / 2] = tc::MmaType<T>::pack(e.x, e.y);
                         }
                     } else {
-                        const int vis = lim - k0 - c * 64;   // columns j <= vis are visible
+                        const int vis = lim - k0 - c * 32;   // columns j <= vis are visible
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t pk[16];
-#pragma unroll
-                            for (int j = 0; j < 32; j += 2) {
-                                const int jj = h * 32 + j;
-                                const float a = jj <= vis
-                                    ? tc05::ex2(fmaf(__uint_as_float(u[jj]), p.q_scale, neg_m)) : 0.f;
-                                const float b = jj + 1 <= vis
-                                    ? tc05::ex2(fmaf(__uint_as_float(u[jj + 1]), p.q_scale, neg_m)) : 0.f;
-                                rs4[(j >> 1) & 3] += a + b;
-                                pk[j / 2] = tc::MmaType<T>::pack(a, b);
-                            }
-                            tc05::tmem_st16(t_lane + c * 32 + h * 16, pk);
+                        for (int j = 0; j < 32; j += 2) {
+                            const float a = j <= vis
+                                ? tc05::ex2(fmaf(__uint_as_float(u[j]), p.q_scale, neg_m)) : 0.f;
+                            const float b = j + 1 <= vis
+                                ? tc05::ex2(fmaf(__uint_as_float(u[j + 1]), p.q_scale, neg_m)) : 0.f;
+                            rs4[(j >> 1) & 3] += a + b;
+                            pk[j / 2] = tc::MmaType<T>::pack(a, b);
                         }
                     }
+                    tc05::tmem_st16(t_lane + c * 16, pk);
                 }
                 tc05::tmem_st_wait();
                 l_run = l_run * alpha + (((rs4[0] + rs4[1]) + (rs4[2] + rs4[3])) +
@@ -744,12 +789,20 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (!ok) break;
             // the next item's Q goes to the tensor cores before this item's
             // epilogue, which its first S can then overlap
+            if (nx == -1) {
+                // not published during the last step: wait for it now that
+                // this tile's P has been handed over
+                nx = next_item(nxt, true);
+                if (nx == 1) fetch_q(nxt);
+            }
+            if (!ok) break;
+            const bool have_next = nx == 1;
             if (have_next) publish_q();
             // epilogue: O / l of the item's last P.V
             if (!wait_ok(&bar[kPvDone + t], (uint32_t)((cnt - 1) & 1))) break;
             tc05::fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tc05::tmem_ld32(t_lane + kM + c * 32, o);
@@ -782,6 +835,16 @@ prefill_tc05_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (warp == 0) {
         tc05::fence_after();
         tc05::tmem_dealloc(tmem, kTmemCols);
+    }
+    // this CTA claims no more items: the last CTA to get here zeroes the
+    // launch's counters for the launch that next takes them
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1ull) == gridDim.x - 1) {
+            __threadfence();
+            p.sched[0] = 0;
+            p.sched[1] = 0;
+        }
     }
 }
 
