@@ -24,6 +24,7 @@ scaling, no collective on the data path); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -53,6 +54,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="opt13b", choices=sorted(wl.CONFIGS))
     ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per batch (0: the workload's own); for small profiling runs")
     ap.add_argument("--variant", default="b", choices=["a", "b"])
     ap.add_argument("--replicas", type=int, default=0,
                     help="replica batches in the pool (0: enough that the cycled distinct KV "
@@ -76,6 +79,8 @@ def config_of(args) -> wl.Config:
     cfg = wl.CONFIGS[args.config]
     if args.block_size:
         cfg = cfg.with_block_size(args.block_size)
+    if args.batch:
+        cfg = dataclasses.replace(cfg, batch=args.batch)
     return cfg
 
 
