@@ -169,19 +169,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int n_boxes = (n + rows_per_box - 1) / rows_per_box;   // boxes per half
         uint8_t* kd = ring + slot * SLOT;
         uint8_t* vd = kd + TILE;
-        if (lane == 0) {
+        if (lane == 0)
             mbar_arrive_expect_tx(&my_full[slot], (uint32_t)(2 * HALVES * n_boxes * rows_per_box * 128));
-            for (int bx = 0; bx < n_boxes; ++bx) {
-                const int t0 = a + bx * rows_per_box;
-                const int lb = t0 / bs;
-                const int y = (blk[lb - lb0] * p.H_kv + g) * bs + (t0 - lb * bs);
-#pragma unroll
-                for (int hf = 0; hf < HALVES; ++hf) {
-                    const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
-                    tma_load_2d(kd + off, &tmap_k, hf * (128 / EB), y, &my_full[slot], policy);
-                    tma_load_2d(vd + off, &tmap_v, hf * (128 / EB), y, &my_full[slot], policy);
-                }
-            }
+        __syncwarp();
+        // one (box, half, K or V) copy per lane: the copies' issue latencies
+        // overlap instead of adding up
+        for (int i = lane; i < 2 * HALVES * n_boxes; i += 32) {
+            const int bx = i / (2 * HALVES), hf = (i >> 1) % HALVES, kv = i & 1;
+            const int t0 = a + bx * rows_per_box;
+            const int lb = t0 / bs;
+            const int y = (blk[lb - lb0] * p.H_kv + g) * bs + (t0 - lb * bs);
+            const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
+            tma_load_2d((kv ? vd : kd) + off, kv ? &tmap_v : &tmap_k, hf * (128 / EB), y,
+                        &my_full[slot], policy);
         }
         __syncwarp();
     };
