@@ -66,8 +66,8 @@ def parse():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-records", action="store_true",
-                    help="skip the Llama-2-70B GQA and FP8 records measured after the "
-                         "OPT-13B headline")
+                    help="skip the Llama-2-70B GQA and FP8 (MHA bs 16 and 4, GQA) records "
+                         "measured after the OPT-13B headline")
     ap.add_argument("--mode", choices=["decode", "prefill", "swap"], default="decode",
                     help="prefill: the prompt phase of the workload's batch (every history "
                          "attended causally as one prompt); swap: one sequence's blocks out to "
@@ -601,7 +601,8 @@ def e2e_of(m: dict) -> dict:
 # (record name, config, block size or 0 for the config's own)
 SUB_RECORDS = (("llama2_70b_gqa_bf16", "llama2_70b", 0),
                ("fp8_bs16", "fp8", 16),
-               ("fp8_bs4", "fp8", 4))
+               ("fp8_bs4", "fp8", 4),
+               ("fp8_gqa", "fp8_gqa", 0))
 
 
 def run_ours(args) -> None:
