@@ -90,26 +90,26 @@ def config_of(args) -> wl.Config:
 # only while the kernel's sources hash to the recorded value, else the bench
 # reports null.
 TRAFFIC = {
-    # (config, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
-    # 293.1 MB for 286.5 MB algorithmic
-    ("llama2_70b", "decode_tc_kernel"):
-        (1.0231, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # 149.0 MB for 143.3 MB
-    ("fp8_gqa", "decode_tc_kernel"):
-        (1.0397, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # 1,358.7 MB for 1,343.5 MB
-    ("fp8", "decode_tc_kernel"):
-        (1.0113, "784c175f582bb3671b2975428abdda67e757d18291b899c93fe572d44b160942"),
-    # 612.2 MB for 604.1 MB
-    ("opt13b", "decode_simt2_kernel"):
-        (1.0134, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
-    # 1,358.7 MB for 1,343.5 MB
-    ("fp8", "decode_simt2_kernel"):
-        (1.0113, "8b4328b47a577eecb8abeaa5559f64cccb7673d30d07124b4261770ada891d5f"),
-    # 2.98 MB for 8.31 MB (the samples of one prompt share its blocks; the
-    # re-reads within a launch hit L2)
-    ("falcon7b", "decode_lean_kernel"):
-        (0.3579, "b86acad210bccc586492a5dc87259763a1a6bc49bd327097f9d1f6005d917aba"),
+    # (config, block size, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
+    # 605.0 MB algorithmic, 612.8 MB read + written
+    ("opt13b", 16, "decode_simt2_kernel"):
+        (1.0128, "c72f458d1d6d9d8001854c60104969a0e3bab8b36cb1e0619e829c897f7c2082"),
+    # 287.0 MB, 292.9 MB
+    ("llama2_70b", 16, "decode_tc_kernel"):
+        (1.0207, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+    # 1,346.0 MB, 1,359.7 MB
+    ("fp8", 16, "decode_tc_kernel"):
+        (1.0101, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+    # 1,346.0 MB, 1,351.6 MB
+    ("fp8", 4, "decode_tc_kernel"):
+        (1.0042, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+    # 144.0 MB, 148.6 MB
+    ("fp8_gqa", 16, "decode_tc_kernel"):
+        (1.0323, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+    # 8.0 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
+    # within a launch hit L2)
+    ("falcon7b", 16, "decode_lean_kernel"):
+        (0.3748, "dd9310a17ee0059cda002e40a956fb4a1a811872f7db738e4f8f3a67c860b7de"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
@@ -129,10 +129,7 @@ def kernel_sources_sha(kernel: str) -> str:
 
 
 def traffic_per_launch(cfg: wl.Config, kernel: str, algorithmic_bytes: float):
-    # captured at each workload's own block size
-    if cfg.block_size != wl.CONFIGS[cfg.name].block_size:
-        return None
-    entry = TRAFFIC.get((cfg.name, kernel))
+    entry = TRAFFIC.get((cfg.name, cfg.block_size, kernel))
     if entry is None or entry[1] != kernel_sources_sha(kernel):
         return None
     return int(entry[0] * algorithmic_bytes)
@@ -576,7 +573,7 @@ def roofline_of(cfg: wl.Config, m: dict, peak: float, peak_kind: str) -> dict:
         "decode_ms_mean": round(dec_total / max(n, 1), 6),
         "merge_ms_mean": round(float(np.mean(m["merge_ms"])), 6),
         "prologue_ms_mean": round(float(np.mean(m["pro_ms"])), 6),
-        "profile_note": f"every {m['prof_every']}th timed round (a stride coprime with the "
+        "profile_note": f"one timed round in {m['prof_every']} (a stride coprime with the "
                         f"{m['R']} replica batches) records CUDA events on the launch stream "
                         "around its kernels, which run without programmatic dependent launch "
                         "in those rounds; achieved = profiled_bytes / profiled_launches / "
