@@ -96,16 +96,16 @@ TRAFFIC = {
         (1.0128, "c72f458d1d6d9d8001854c60104969a0e3bab8b36cb1e0619e829c897f7c2082"),
     # 287.0 MB, 292.9 MB
     ("llama2_70b", 16, "decode_tc_kernel"):
-        (1.0207, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+        (1.0207, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
     # 1,346.0 MB, 1,359.7 MB
     ("fp8", 16, "decode_tc_kernel"):
-        (1.0101, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+        (1.0101, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
     # 1,346.0 MB, 1,351.6 MB
     ("fp8", 4, "decode_tc_kernel"):
-        (1.0042, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+        (1.0042, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
     # 144.0 MB, 148.6 MB
     ("fp8_gqa", 16, "decode_tc_kernel"):
-        (1.0323, "94062cc9649d6568976b0c10f655c151ade795f71a742a572379f8b2c2080537"),
+        (1.0323, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
     # 8.0 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
     # within a launch hit L2)
     ("falcon7b", 16, "decode_lean_kernel"):

@@ -18,7 +18,7 @@
 //
 // CTA = (partition, KV head, sequence).  Warps: MT warps of 8 query heads
 // (MT = ceil(G / 8)) x TS token groups.  Each token group owns a ring of
-// kStages slots; lane 0 of its first warp issues the copies, every warp of the
+// kStages slots; its first warp issues the copies (one box per lane), every warp of the
 // group consumes every stage, and with MT > 1 an "empty" mbarrier per slot
 // (MT arrivals) tells the producer when all of them are done with it.
 // A warp computes S^T = K Q^T and O^T += V^T P^T (16 tokens or 16 d-rows by
