@@ -198,3 +198,36 @@ def test_prefill_negative_scale(kernel):
     for i, (s, q) in enumerate(zip(seqs, qs)):
         ref = side.orc.prefill(s, q, "bf16", -cfg.scale)
         compare_out(got[starts[i]:starts[i + 1]], ref, "bf16")
+
+
+@pytest.mark.slow
+def test_prefill_full_size_sampled_rows():
+    # the prompt-phase workload bench.py --mode prefill times, at full size
+    # (64 sequences of the Llama-2-70B-shaped layer, every history one
+    # prompt, the tcgen05 kernel): three rows per sequence - its first,
+    # middle and last token - every query head, against the oracle's
+    # attention of that row over its causal prefix
+    from oracle.attention import decode_attention
+
+    cfg = wl.CONFIGS["llama2_70b"]
+    side = setup_config(cfg, seed=11)
+    seqs = side.seqs
+    n = [int(side.orc.bm.lengths[s]) for s in seqs]
+    qs = [wl.round_to(wl.prompt_queries(cfg, 11, s, k), cfg.q_dtype) for s, k in zip(seqs, n)]
+    starts = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    max_blocks = max(pk.bt_num_blocks(side.pool, s) for s in seqs)
+    tables, lens, _ = pk.bt_export(side.pool, seqs, max_blocks)
+    out = pk.paged_prefill_attention(side.pool, to_torch(np.concatenate(qs), cfg.q_dtype),
+                                     torch.from_numpy(starts).cuda(),
+                                     torch.from_numpy(tables).cuda(),
+                                     torch.from_numpy(lens).cuda(), cfg.scale,
+                                     kernel=pk.PKV_PREFILL_TCGEN05)
+    torch.cuda.synchronize()
+    assert pk.pkv_device_error(side.pool) == 0
+    got = to_f64(from_torch(out, cfg.q_dtype), cfg.q_dtype)
+    for i, s in enumerate(seqs):
+        kh, vh = side.orc.history(int(s))
+        kd, vd = side.orc.dequant(kh, "k"), side.orc.dequant(vh, "v")
+        for t in sorted({0, n[i] // 2, n[i] - 1}):
+            ref = decode_attention(to_f64(qs[i][t], cfg.q_dtype), kd[:t + 1], vd[:t + 1], cfg.scale)
+            compare_out(got[starts[i] + t][None], ref[None], cfg.q_dtype)
