@@ -292,7 +292,7 @@ def test_fp8_gqa_full(kernel):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("bs", [1, 16])
+@pytest.mark.parametrize("bs", [1, 4, 16])   # 4 and 16: the bench's FP8 sub-records
 def test_fp8_full(bs):
     cfg = wl.CONFIGS["fp8"].with_block_size(bs)
     side = setup_config(cfg)
