@@ -351,7 +351,13 @@ void pkv_step_destroy(pkv_step* step);
  *   a round sends only what changed (slots, lengths, rows, copy pairs, new
  *   table entries) as the parameters of one prologue kernel, falling back to
  *   a packed host-to-device copy of the batch's full tables when that does not
- *   fit (first sight of many long sequences).  With split contexts the
+ *   fit (first sight of many long sequences).  On the parameter path (up to
+ *   128 sequences) the decode kernel also receives each launch slot's length,
+ *   row, sequence index and the count of leading table entries the prologue
+ *   leaves unchanged, and starts loading those blocks and its queries while
+ *   the prologue still runs (programmatic dependent launch); the block that
+ *   takes the new token, and any copy-on-write target, are read only after
+ *   the prologue has finished.  With split contexts the
  *   decode kernel merges the partitions itself (counters in the runtime's
  *   workspace, zero between calls) when the tensor-core or swizzled-TMA
  *   kernel runs.

@@ -363,7 +363,8 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
                                  int* counters = nullptr, bool pdl = false,
                                  const int32_t* table_rows = nullptr, int n_table_rows = 0,
                                  int* n_launches = nullptr, int* kernel_used = nullptr,
-                                 const int32_t* order = nullptr) {
+                                 const int32_t* order = nullptr,
+                                 const pkv::StepPrefetch* pre = nullptr) {
     if (n_launches) *n_launches = 0;
     if (kernel_used) *kernel_used = 0;
     if (!p || p->host_only || B < 0) return PKV_ERR_INVALID_ARG;
@@ -444,6 +445,7 @@ pkv_status decode_attention_impl(pkv_pool* p, const void* q, pkv_dtype q_dtype,
     dp.table_rows = table_rows;
     dp.n_table_rows = n_table_rows;
     dp.order = order;
+    dp.pre = pre;
     const float log2e = 1.4426950408889634f;
     dp.q_scale = scale * log2e * p->k_scale;
     dp.v_scale = p->v_scale;
@@ -608,7 +610,9 @@ struct pkv_step {
     // one round's host scratch
     std::vector<int32_t> h_slots, h_src, h_dst, h_rows, h_cow_rows, h_upd_idx, h_upd_val;
     std::vector<int32_t> h_lens, h_order, h_key;   // fast path: lengths, launch order, sort key
+    std::vector<int32_t> h_stable;    // fast path: leading row entries the prologue keeps
     pkv::StepArgs args;
+    pkv::StepPrefetch pre{};          // fast path: per launch slot, for the decode kernel
     long long fast_rounds = 0, slow_rounds = 0;
     // profiling: every prof_every-th round records four events (before the
     // prologue, before the decode kernel, between it and the merge, after the
@@ -855,6 +859,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
     s->h_rows.resize(B);
     s->h_upd_idx.clear();
     s->h_upd_val.clear();
+    s->h_stable.resize(B);
     for (int i = 0; i < B; ++i) {
         const int r = row_for(s, seq_ids[i]);
         if (r < 0) return PKV_ERR_INVALID_ARG;   // cannot happen: max_seqs >= max_batch
@@ -869,6 +874,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         const int nb = (int)sq->blocks.size();
         const bool same = s->row_epoch[r] == sq->epoch;
         const int from = same ? (s->row_nb[r] > 0 ? s->row_nb[r] - 1 : 0) : 0;
+        s->h_stable[i] = from;   // entries below `from` stay as the device holds them
         const int32_t* m = s->mirror.data() + (size_t)r * s->max_blocks;
         for (int e = from; e < nb; ++e) {
             if (same && e < s->row_nb[r] && m[e] == sq->blocks[e]) continue;
@@ -934,6 +940,15 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
         for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_idx[u];
         d += a.n_upd;
         for (int32_t u = 0; u < a.n_upd; ++u) d[u] = s->h_upd_val[u];
+        // what the prologue will leave in the launch slots' lengths, rows and
+        // leading table entries, for the decode kernel to start from
+        s->pre.n = B <= pkv::kPreSlots ? B : 0;
+        for (int z = 0; z < s->pre.n; ++z) {
+            s->pre.lens[z] = s->h_lens[s->h_order[z]];
+            s->pre.rows[z] = s->h_rows[s->h_order[z]];
+            s->pre.order[z] = s->h_order[z];
+            s->pre.stable[z] = s->h_stable[s->h_order[z]];
+        }
         cudaError_t e = pkv::launch_step_prologue(
             a, pool->k, pool->v, k_new, v_new, s->q_dtype, pool->dtype, s->d_tables, d_lens,
             d_rows, d_order, pool->n_kv_heads, pool->head_dim, bs, pool->num_blocks, pool->k_scale,
@@ -996,7 +1011,7 @@ pkv_status pkv_decode_step(pkv_step* s, const int64_t* seq_ids, int B, const voi
                                s->n_q_heads, scale, out, s->d_ws, s->ws_bytes, s->partition_tokens,
                                s->kernel, stream, e0, e1, e2, s->d_counters, fits && !profiled,
                                d_rows, s->max_seqs, &decode_launches, &s->last_kernel,
-                               fits ? d_order : nullptr);
+                               fits ? d_order : nullptr, fits ? &s->pre : nullptr);
     if (ps != PKV_OK) return ps;
     if (profiled) ++s->prof_count;
     launches += decode_launches;

@@ -112,7 +112,7 @@ template <typename KV, typename QT, int D, int W, int S>
 __global__ void __launch_bounds__(W * 32)
 decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p,
-                    int table_entries, int bs_shift) {
+                    const __grid_constant__ StepPrefetch pf, int table_entries, int bs_shift) {
     using L = Simt2Smem<KV, D, W, S>;
     constexpr int NT = W * 32;
     constexpr int PARTS = L::kParts;                 // 1, 2 or 4
@@ -144,11 +144,27 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int P = p.part_tokens;
 
     __shared__ int last_flag;
-    grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
-    const long long trow = table_row(p, slot);   // issued together with the length load
-    const int c = p.lens[slot];
-    const int seq = seq_of(p, slot);             // the caller's sequence: q, out, partials
+    // Lengths, tables, rows and the launch order come from the preceding
+    // kernel.  A launch slot that the host's prefetch block covers takes its
+    // length, row and sequence from there, and loads the table entries below
+    // its stable count, the stages they cover and its query before waiting
+    // for that kernel.
+    const bool pre = slot < pf.n;
+    long long trow;
+    int c, seq;   // seq: the caller's sequence (q, out, partials)
+    if (pre) {
+        const int r = pf.rows[slot];
+        trow = (r >= 0 && r < p.n_table_rows) ? r : -1;
+        c = pf.lens[slot];
+        seq = pf.order[slot];
+    } else {
+        grid_dependency_wait();
+        trow = table_row(p, slot);   // issued together with the length load
+        c = p.lens[slot];
+        seq = seq_of(p, slot);
+    }
     if (c < 1 || c > p.max_blocks * bs) {
+        if (pre) grid_dependency_wait();
         if (part == 0) {
             if (tid == 0 && h == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
             QT* out = reinterpret_cast<QT*>(p.out);
@@ -164,9 +180,11 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int t_end = min(c, t_begin + Ps);
     const int lb0 = t_begin >> bs_shift;
     const int n_lb = ((t_end - 1) >> bs_shift) - lb0 + 1;
+    // table entries final before the preceding kernel ends
+    const int n_pre = pre ? max(0, min(n_lb, pf.stable[slot] - lb0)) : n_lb;
 
     bool bad = trow < 0;
-    for (int i = tid; i < n_lb && trow >= 0; i += NT) {
+    for (int i = tid; i < n_pre && trow >= 0; i += NT) {
         const int32_t b = p.tables[trow * p.max_blocks + lb0 + i];
         bad |= (b < 0 || b >= p.num_blocks);
         blk[i] = b;
@@ -175,24 +193,7 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int i = 0; i < W * S; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
-    const bool split = nparts > 1;
-    if (__syncthreads_or(bad)) {
-        if (tid == 0 && h == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
-        for (int d = tid; d < D; d += NT) {
-            const size_t row = ((size_t)seq * p.H_q + h) * p.max_parts + part;
-            if (split) {
-                p.ws_acc[row * D + d] = 0.f;
-                if (d == 0) { p.ws_ml[row * 2] = -INFINITY; p.ws_ml[row * 2 + 1] = 0.f; }
-            } else {
-                reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<QT>::from_f(0.f);
-            }
-        }
-        if (split && p.counters &&
-            finish_partition(&p.counters[(size_t)seq * p.H_q + h], nparts, &last_flag))
-            merge_group_in_cta<QT, D>(p, seq, h, 1, nparts, reinterpret_cast<float*>(smem),
-                                      L::kTiles / 4);
-        return;
-    }
+    bad = __syncthreads_or(bad);
 
     const int n_stages = (t_end - t_begin + kTok - 1) / kTok;
     const int my_n = n_stages > warp ? (n_stages - warp + W - 1) / W : 0;
@@ -224,20 +225,62 @@ decode_simt2_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
     };
 
-    const int pro = min(S, my_n);
-    for (int k = 0; k < pro; ++k) issue(k, k);
-
     // this lane's half of q (score chunks), pre-scaled; loaded while the first
     // stages are in flight
     const int tok = lane & 15;
     const int side = lane >> 4;
     float qk[CPL * EPC];
-    {
+    auto load_q = [&]() {
         const QT* qp = reinterpret_cast<const QT*>(p.q) + ((size_t)seq * p.H_q + h) * D;
 #pragma unroll
         for (int j = 0; j < CPL * EPC; ++j)
             qk[j] = Elem<QT>::to_f(qp[side * (D / 2) + j]) * p.q_scale;
+    };
+
+    const int pro = min(S, my_n);
+    int issued = 0;   // first stages in flight before the wait
+    if (pre) {
+        if (!bad)
+            for (; issued < pro; ++issued) {
+                const int a = t_begin + (warp + issued * W) * kTok;
+                if (((min(a + kTok, t_end) - 1) >> bs_shift) - lb0 >= n_pre) break;
+                issue(issued, issued);
+            }
+        load_q();
+        grid_dependency_wait();
+        if (n_pre < n_lb) {
+            bool bad2 = false;
+            for (int i = n_pre + tid; i < n_lb && trow >= 0; i += NT) {
+                const int32_t b = p.tables[trow * p.max_blocks + lb0 + i];
+                bad2 |= (b < 0 || b >= p.num_blocks);
+                blk[i] = b;
+            }
+            bad = __syncthreads_or(bad2) || bad;
+        }
     }
+    const bool split = nparts > 1;
+    if (bad) {
+        // copies issued before the wait land before the CTA leaves
+        for (int j = 0; j < issued; ++j) (void)mbar_wait(&my_bars[j], 0u);
+        if (tid == 0 && h == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
+        for (int d = tid; d < D; d += NT) {
+            const size_t row = ((size_t)seq * p.H_q + h) * p.max_parts + part;
+            if (split) {
+                p.ws_acc[row * D + d] = 0.f;
+                if (d == 0) { p.ws_ml[row * 2] = -INFINITY; p.ws_ml[row * 2 + 1] = 0.f; }
+            } else {
+                reinterpret_cast<QT*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<QT>::from_f(0.f);
+            }
+        }
+        if (split && p.counters &&
+            finish_partition(&p.counters[(size_t)seq * p.H_q + h], nparts, &last_flag))
+            merge_group_in_cta<QT, D>(p, seq, h, 1, nparts, reinterpret_cast<float*>(smem),
+                                      L::kTiles / 4);
+        return;
+    }
+
+    for (int k = issued; k < pro; ++k) issue(k, k);
+    if (!pre) load_q();
 
     float m_run = -INFINITY, l_run = 0.f;
     float acc[VEC];
@@ -390,7 +433,7 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap* tk, const CUtenso
     cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
     e = launch_kernel(kern, dim3(p.max_parts, p.H_q, p.B), dim3(W * 32), smem, st, p.pdl != 0,
-                      *tk, *tv, p, te, bs_shift);
+                      *tk, *tv, p, prefetch_of(p), te, bs_shift);
     if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
     if (e != cudaSuccess || p.max_parts <= 1 || p.counters) return e;
     return launch_merge(p, q_dtype, D, st);

@@ -60,7 +60,8 @@ __host__ __device__ constexpr int tc_union_bytes() {
 template <typename T, int D, int MT, int TS, int S, int EB>
 __global__ void __launch_bounds__(MT * TS * 32)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                 const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+                 const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p,
+                 const __grid_constant__ StepPrefetch pf) {
     constexpr int kStages = S;
     constexpr int NW = MT * TS;
     constexpr int NT = NW * 32;
@@ -98,11 +99,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int h_base = g * G;       // first query head of the group
 
     __shared__ int last_flag;
-    grid_dependency_wait();   // lengths, tables and rows come from the preceding kernel
-    const long long trow = table_row(p, slot);   // issued together with the length load
-    const int c = p.lens[slot];
-    const int seq = seq_of(p, slot);             // the caller's sequence: q, out, partials
+    // Lengths, tables, rows and the launch order come from the preceding
+    // kernel.  A launch slot that the host's prefetch block covers takes its
+    // length, row and sequence from there, and loads the table entries below
+    // its stable count, the stages they cover and its query before waiting
+    // for that kernel.
+    const bool pre = slot < pf.n;
+    long long trow;
+    int c, seq;   // seq: the caller's sequence (q, out, partials)
+    if (pre) {
+        const int r = pf.rows[slot];
+        trow = (r >= 0 && r < p.n_table_rows) ? r : -1;
+        c = pf.lens[slot];
+        seq = pf.order[slot];
+    } else {
+        grid_dependency_wait();
+        trow = table_row(p, slot);   // issued together with the length load
+        c = p.lens[slot];
+        seq = seq_of(p, slot);
+    }
     if (c < 1 || c > p.max_blocks * bs) {
+        if (pre) grid_dependency_wait();
         if (part == 0) {
             if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_CONTEXT_LEN);
             T* out = reinterpret_cast<T*>(p.out);
@@ -119,11 +136,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int32_t* table = p.tables + (trow < 0 ? 0 : trow) * p.max_blocks;
 
     const int lb0 = t_begin / bs;
+    const int n_lb = (t_end - 1) / bs - lb0 + 1;
+    // table entries final before the preceding kernel ends
+    const int n_pre = pre ? max(0, min(n_lb, pf.stable[slot] - lb0)) : n_lb;
     bool bad = trow < 0;
-    for (int lb = lb0 + tid; lb <= (t_end - 1) / bs && trow >= 0; lb += NT) {
-        const int32_t b = table[lb];
+    for (int i = tid; i < n_pre && trow >= 0; i += NT) {
+        const int32_t b = table[lb0 + i];
         bad |= (b < 0 || b >= p.num_blocks);
-        blk[lb - lb0] = b;
+        blk[i] = b;
     }
     if (tid == 0) {
         for (int i = 0; i < TS * kStages; ++i) {
@@ -132,25 +152,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         fence_mbar_init();
     }
-    const bool split = nparts > 1;
-    if (__syncthreads_or(bad)) {
-        if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
-        for (int i = tid; i < G * D; i += NT) {
-            const int h = h_base + i / D, d = i % D;
-            const size_t row = ((size_t)seq * p.H_q + h) * p.max_parts + part;
-            if (split) {
-                p.ws_acc[row * D + d] = 0.f;
-                if (d == 0) { p.ws_ml[row * 2] = -INFINITY; p.ws_ml[row * 2 + 1] = 0.f; }
-            } else {
-                reinterpret_cast<T*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<T>::from_f(0.f);
-            }
-        }
-        if (split && p.counters &&
-            finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
-            merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
-                                     tc_union_bytes<D, MT, TS, S, EB>() / 4);
-        return;
-    }
+    bad = __syncthreads_or(bad);
 
     const int n_stages = (t_end - t_begin + kStageTokens - 1) / kStageTokens;
     const int my_n = n_stages > ts ? (n_stages - ts + TS - 1) / TS : 0;
@@ -190,12 +192,60 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int gq = lane >> 2;       // fragment row: d (and d + 8) of O^T
     const int tq = lane & 3;        // this lane's heads: 2 tq, 2 tq + 1 of the warp's 8
     uint32_t qb[KSTEPS][2];
-    if constexpr (EB == 1)
-        tc::load_qT_frags_fp8(qb, reinterpret_cast<const __half*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
-                              mt * 8, G, lane);
-    else
-        tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
-                                mt * 8, G, lane);
+    auto load_q = [&]() {
+        if constexpr (EB == 1)
+            tc::load_qT_frags_fp8(qb, reinterpret_cast<const __half*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
+                                  mt * 8, G, lane);
+        else
+            tc::load_qT_frags<T, D>(qb, reinterpret_cast<const T*>(p.q) + ((size_t)seq * p.H_q + h_base) * D,
+                                    mt * 8, G, lane);
+    };
+
+    const int pro = min(kStages, my_n);
+    int issued = 0;   // first stages in flight before the wait (producer warps)
+    if (pre) {
+        if (!bad && producer)
+            for (; issued < pro; ++issued) {
+                const int a = t_begin + (ts + issued * TS) * kStageTokens;
+                if ((min(a + kStageTokens, t_end) - 1) / bs - lb0 >= n_pre) break;
+                issue(issued, issued);
+            }
+        load_q();
+        grid_dependency_wait();
+        if (n_pre < n_lb) {
+            bool bad2 = false;
+            for (int i = n_pre + tid; i < n_lb && trow >= 0; i += NT) {
+                const int32_t b = table[lb0 + i];
+                bad2 |= (b < 0 || b >= p.num_blocks);
+                blk[i] = b;
+            }
+            bad = __syncthreads_or(bad2) || bad;
+        }
+    }
+    const bool split = nparts > 1;
+    if (bad) {
+        // copies issued before the wait land before the CTA leaves
+        for (int j = 0; j < issued; ++j) (void)mbar_wait(&my_full[j], 0u);
+        __syncthreads();
+        if (tid == 0 && g == 0) report_error(p.err, PKV_DEVERR_BLOCK_ID);
+        for (int i = tid; i < G * D; i += NT) {
+            const int h = h_base + i / D, d = i % D;
+            const size_t row = ((size_t)seq * p.H_q + h) * p.max_parts + part;
+            if (split) {
+                p.ws_acc[row * D + d] = 0.f;
+                if (d == 0) { p.ws_ml[row * 2] = -INFINITY; p.ws_ml[row * 2 + 1] = 0.f; }
+            } else {
+                reinterpret_cast<T*>(p.out)[((size_t)seq * p.H_q + h) * D + d] = Elem<T>::from_f(0.f);
+            }
+        }
+        if (split && p.counters &&
+            finish_partition(&p.counters[(size_t)seq * p.H_kv + g], nparts, &last_flag))
+            merge_group_in_cta<T, D>(p, seq, h_base, G, nparts, reinterpret_cast<float*>(smem),
+                                     tc_union_bytes<D, MT, TS, S, EB>() / 4);
+        return;
+    }
+
+    if (!pre) load_q();
 
     float o[D / 16][4];
 #pragma unroll
@@ -203,10 +253,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
 
-    if (producer) {
-        const int pro = min(kStages, my_n);
-        for (int k = 0; k < pro; ++k) issue(k, k);
-    }
+    if (producer)
+        for (int k = issued; k < pro; ++k) issue(k, k);
 
     int k = 0;
     bool timed_out = false;
@@ -370,7 +418,8 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap* tk, const CUte
     cudaError_t e = allow_large_smem(kern, &attr_done);
     if (e != cudaSuccess) return e;
     const dim3 grid(p.max_parts, p.H_kv, p.B);
-    e = launch_kernel(kern, grid, dim3(MT * TS * 32), smem, st, p.pdl != 0, *tk, *tv, p);
+    e = launch_kernel(kern, grid, dim3(MT * TS * 32), smem, st, p.pdl != 0, *tk, *tv, p,
+                      prefetch_of(p));
     if (e == cudaSuccess && mid) e = cudaEventRecord(mid, st);
     if (e != cudaSuccess || p.max_parts <= 1 || p.counters) return e;
     return launch_merge(p, q_dtype, D, st);

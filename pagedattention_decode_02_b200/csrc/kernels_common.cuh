@@ -295,7 +295,32 @@ struct DecodeParams {
     long long head_stride;   // bytes of one (block, kv head) tile: bs * D * elem
     long long block_stride;  // bytes of one block: H_kv * head_stride
     unsigned long long wait_ns;  // budget of the main loops' waits (the pool's)
+    const struct StepPrefetch* pre;   // host side only: see StepPrefetch (null: none)
 };
+
+// What the decode-step runtime knows on the host about each launch slot
+// before the round's prologue kernel runs: the context length, the table row,
+// the caller's sequence index, and how many leading entries of the row the
+// prologue leaves unchanged (their blocks hold no token it writes and no
+// copy-on-write target).  Passed to the decode kernel by value, so that a CTA
+// can read those entries, start loading their blocks and load its query
+// before the prologue has finished (the query is not the prologue's output:
+// it was written before the prologue, which starts only once all preceding
+// work on the stream has completed).
+constexpr int kPreSlots = 128;
+struct StepPrefetch {
+    int n;                        // launch slots covered: 0 .. n - 1 (0: none)
+    int32_t lens[kPreSlots];
+    int32_t rows[kPreSlots];
+    int32_t order[kPreSlots];
+    int32_t stable[kPreSlots];
+};
+
+// The launch's prefetch block, or an empty one.
+inline const StepPrefetch& prefetch_of(const DecodeParams& p) {
+    static const StepPrefetch none{};
+    return p.pre ? *p.pre : none;
+}
 
 }  // namespace pkv
 
