@@ -94,7 +94,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int mt = warp % MT;       // m-tile of this warp
     const int ts = warp / MT;       // token group of this warp
     const int G = p.G;
-    const int bs = p.block_size;
+    const int bs = p.block_size;   // a power of two (row tensor maps)
+    const int bs_shift = __ffs(bs) - 1;
     const int P = p.part_tokens;
     const int h_base = g * G;       // first query head of the group
 
@@ -135,8 +136,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int t_end = min(c, t_begin + Ps);
     const int32_t* table = p.tables + (trow < 0 ? 0 : trow) * p.max_blocks;
 
-    const int lb0 = t_begin / bs;
-    const int n_lb = (t_end - 1) / bs - lb0 + 1;
+    const int lb0 = t_begin >> bs_shift;
+    const int n_lb = ((t_end - 1) >> bs_shift) - lb0 + 1;
     // table entries final before the preceding kernel ends
     const int n_pre = pre ? max(0, min(n_lb, pf.stable[slot] - lb0)) : n_lb;
     bool bad = trow < 0;
@@ -179,8 +180,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int i = lane; i < 2 * HALVES * n_boxes; i += 32) {
             const int bx = i / (2 * HALVES), hf = (i >> 1) % HALVES, kv = i & 1;
             const int t0 = a + bx * rows_per_box;
-            const int lb = t0 / bs;
-            const int y = (blk[lb - lb0] * p.H_kv + g) * bs + (t0 - lb * bs);
+            const int lb = t0 >> bs_shift;
+            const int y = ((blk[lb - lb0] * p.H_kv + g) << bs_shift) + (t0 & (bs - 1));
             const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
             tma_load_2d((kv ? vd : kd) + off, kv ? &tmap_v : &tmap_k, hf * (128 / EB), y,
                         &my_full[slot], policy);
@@ -207,7 +208,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (!bad && producer)
             for (; issued < pro; ++issued) {
                 const int a = t_begin + (ts + issued * TS) * kStageTokens;
-                if ((min(a + kStageTokens, t_end) - 1) / bs - lb0 >= n_pre) break;
+                if (((min(a + kStageTokens, t_end) - 1) >> bs_shift) - lb0 >= n_pre) break;
                 issue(issued, issued);
             }
         load_q();

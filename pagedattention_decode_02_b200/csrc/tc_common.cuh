@@ -168,7 +168,8 @@ __device__ __forceinline__ float ex2_fast(float x) {
 
 // Online-softmax update of one stage for this lane's two heads; returns P^T
 // as the B operand of the P.V product (pb0 = tokens 0-7, pb1 = tokens 8-15)
-// and rescales o when a running maximum moved.
+// and rescales o and l when the running maxima move (lazily: only when a
+// score exceeds its head's maximum by more than 2^8).
 template <typename T, int MTILES>
 __device__ __forceinline__ void softmax_step(const float (&s)[4], float (&o)[MTILES][4],
                                              float (&m_run)[2], float (&l_run)[2], uint32_t& pb0,
@@ -180,22 +181,18 @@ __device__ __forceinline__ void softmax_step(const float (&s)[4], float (&o)[MTI
         mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
         mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
     }
-    float alpha[2];
+    // lazy rescaling: the running maximum moves only when a new score
+    // exceeds it by more than 2^8 (probabilities stay below 256, exact to the
+    // f16/bf16 rounding of P); the whole warp moves together
+    if (__any_sync(0xffffffffu, mx[0] > m_run[0] + 8.f || mx[1] > m_run[1] + 8.f)) {
+        float alpha[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float m_new = fmaxf(m_run[h], mx[h]);
-        alpha[h] = ex2_fast(m_run[h] - m_new);
-        m_run[h] = m_new;
-    }
-    const float p0 = ex2_fast(s[0] - m_run[0]);
-    const float p1 = ex2_fast(s[1] - m_run[1]);
-    const float p2 = ex2_fast(s[2] - m_run[0]);
-    const float p3 = ex2_fast(s[3] - m_run[1]);
-    l_run[0] = l_run[0] * alpha[0] + (p0 + p2);
-    l_run[1] = l_run[1] * alpha[1] + (p1 + p3);
-    pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
-    pb1 = movmatrix_trans(MmaType<T>::pack(p2, p3));
-    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+        for (int h = 0; h < 2; ++h) {
+            const float m_new = fmaxf(m_run[h], mx[h]);
+            alpha[h] = ex2_fast(m_run[h] - m_new);
+            m_run[h] = m_new;
+            l_run[h] *= alpha[h];
+        }
 #pragma unroll
         for (int mt = 0; mt < MTILES; ++mt) {
             o[mt][0] *= alpha[0];
@@ -204,6 +201,14 @@ __device__ __forceinline__ void softmax_step(const float (&s)[4], float (&o)[MTI
             o[mt][3] *= alpha[1];
         }
     }
+    const float p0 = ex2_fast(s[0] - m_run[0]);
+    const float p1 = ex2_fast(s[1] - m_run[1]);
+    const float p2 = ex2_fast(s[2] - m_run[0]);
+    const float p3 = ex2_fast(s[3] - m_run[1]);
+    l_run[0] += p0 + p2;
+    l_run[1] += p1 + p3;
+    pb0 = movmatrix_trans(MmaType<T>::pack(p0, p1));
+    pb1 = movmatrix_trans(MmaType<T>::pack(p2, p3));
 }
 
 // One 16-token stage for one warp's 8 query heads, in transposed form (no
@@ -229,7 +234,7 @@ __device__ __forceinline__ void stage_math_t(const uint32_t (&qb)[D / 16][2],
     float s[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
-    mask_scores(s, n, lane);
+    if (n < 16) mask_scores(s, n, lane);
     uint32_t pb0, pb1;
     softmax_step<T, D / 16>(s, o, m_run, l_run, pb0, pb1);
 #pragma unroll
@@ -258,7 +263,7 @@ __device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], co
     float s[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
-    mask_scores(s, n, lane);
+    if (n < 16) mask_scores(s, n, lane);
     uint32_t pb0, pb1;
     softmax_step<T, D / 16>(s, o, m_run, l_run, pb0, pb1);
     if (n == kStageTokens) {
@@ -382,7 +387,7 @@ __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const
     float s[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
-    mask_scores(s, n, lane);
+    if (n < 16) mask_scores(s, n, lane);
     uint32_t pb0, pb1;
     softmax_step<__half, 8>(s, o, m_run, l_run, pb0, pb1);
     // V^T fragments: a token pair's codes of one d interleaved byte by byte
