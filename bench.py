@@ -91,25 +91,25 @@ def config_of(args) -> wl.Config:
 # reports null.
 TRAFFIC = {
     # (config, block size, kernel): (dram bytes / algorithmic bytes, sha256 of its sources)
-    # 605.0 MB algorithmic, 612.8 MB read + written
+    # 605.3 MB algorithmic, 612.7 MB read + written
     ("opt13b", 16, "decode_simt2_kernel"):
-        (1.0128, "c72f458d1d6d9d8001854c60104969a0e3bab8b36cb1e0619e829c897f7c2082"),
-    # 287.0 MB, 292.9 MB
+        (1.0123, "3d500856b22f29f4b5587277bc162b747071c43be02490f014a82dffad3bbe4e"),
+    # 287.0 MB, 293.3 MB
     ("llama2_70b", 16, "decode_tc_kernel"):
-        (1.0207, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
-    # 1,346.0 MB, 1,359.7 MB
+        (1.0217, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
+    # 1,346.1 MB, 1,359.6 MB
     ("fp8", 16, "decode_tc_kernel"):
-        (1.0101, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
-    # 1,346.0 MB, 1,351.6 MB
+        (1.0100, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
+    # 1,346.1 MB, 1,352.1 MB
     ("fp8", 4, "decode_tc_kernel"):
-        (1.0042, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
-    # 144.0 MB, 148.6 MB
+        (1.0044, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
+    # 143.5 MB, 149.4 MB
     ("fp8_gqa", 16, "decode_tc_kernel"):
-        (1.0323, "4687a032144946de838cb90e45ecfa775463e1691ff8012f9e5f44b5ffba5aec"),
-    # 8.0 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
+        (1.0412, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
+    # 8.3 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
     # within a launch hit L2)
     ("falcon7b", 16, "decode_lean_kernel"):
-        (0.3748, "dd9310a17ee0059cda002e40a956fb4a1a811872f7db738e4f8f3a67c860b7de"),
+        (0.3593, "e2a75488c288e0bd0a4722ca2df2516788ab74b71ed6900530846a5d6a95cde7"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
