@@ -162,14 +162,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     uint64_t* my_empty = empty + ts * kStages;
     const bool producer = (mt == 0);
     const uint64_t policy = l2_evict_first_policy();
-    const int rows_per_box = bs < kStageTokens ? bs : kStageTokens;   // 8 or 16
+    const int rpb_shift = bs_shift < 4 ? bs_shift : 4;   // rows per box: min(bs, 16)
+    const int rows_per_box = 1 << rpb_shift;
 
     // issue stage k_local (this group's k-th) into `slot`; called by the
     // producer warp (all lanes)
     auto issue = [&](int k_local, int slot) {
         const int a = t_begin + (ts + k_local * TS) * kStageTokens;
         const int n = min(kStageTokens, t_end - a);
-        const int n_boxes = (n + rows_per_box - 1) / rows_per_box;   // boxes per half
+        const int n_boxes = (n + rows_per_box - 1) >> rpb_shift;   // boxes per half
         uint8_t* kd = ring + slot * SLOT;
         uint8_t* vd = kd + TILE;
         if (lane == 0)
@@ -179,10 +180,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // overlap instead of adding up
         for (int i = lane; i < 2 * HALVES * n_boxes; i += 32) {
             const int bx = i / (2 * HALVES), hf = (i >> 1) % HALVES, kv = i & 1;
-            const int t0 = a + bx * rows_per_box;
+            const int t0 = a + (bx << rpb_shift);
             const int lb = t0 >> bs_shift;
             const int y = ((blk[lb - lb0] * p.H_kv + g) << bs_shift) + (t0 & (bs - 1));
-            const int off = hf * (kStageTokens * 128) + bx * rows_per_box * 128;
+            const int off = hf * (kStageTokens * 128) + (bx << rpb_shift) * 128;
             tma_load_2d((kv ? vd : kd) + off, kv ? &tmap_v : &tmap_k, hf * (128 / EB), y,
                         &my_full[slot], policy);
         }
@@ -259,15 +260,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     int k = 0;
     bool timed_out = false;
+    int rslot = 0;         // ring slot: k % kStages
+    uint32_t phase = 0;    // its parity: (k / kStages) & 1
     for (; k < my_n; ++k) {
-        const int slot = k % kStages;
-        if (!mbar_wait(&my_full[slot], (uint32_t)((k / kStages) & 1), p.wait_ns)) {
+        if (k > 0 && ++rslot == kStages) {
+            rslot = 0;
+            phase ^= 1u;
+        }
+        if (!mbar_wait(&my_full[rslot], phase, p.wait_ns)) {
             timed_out = true;
             break;
         }
         const int a = t_begin + (ts + k * TS) * kStageTokens;
         const int n = min(kStageTokens, t_end - a);
-        const uint8_t* kt = ring + slot * SLOT;
+        const uint8_t* kt = ring + rslot * SLOT;
         const uint8_t* vt = kt + TILE;
         // hand the slot back for the next copy: the producer waits (MT > 1)
         // until every warp of the group has read it
@@ -275,18 +281,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
             fence_proxy_async_smem();   // these reads before the async proxy's refill
             __syncwarp();
             if constexpr (MT > 1) {
-                if (lane == 0) mbar_arrive(&my_empty[slot]);
+                if (lane == 0) mbar_arrive(&my_empty[rslot]);
             }
             if (producer && k + kStages < my_n) {
                 if constexpr (MT > 1) {
-                    if (!mbar_wait(&my_empty[slot], (uint32_t)((k / kStages) & 1), p.wait_ns)) return false;
+                    if (!mbar_wait(&my_empty[rslot], phase, p.wait_ns)) return false;
                 }
-                issue(k + kStages, slot);
+                issue(k + kStages, rslot);
             }
             return true;
         };
         if constexpr (kEarly) {
-            // the stage moves into registers, the slot is released, and the
+            // the stage moves into registers, the rslot is released, and the
             // math runs while the next copy is in flight
             using Frags = std::conditional_t<EB == 1, tc::Fp8Raw, tc::StageFrags<D>>;
             Frags f;
