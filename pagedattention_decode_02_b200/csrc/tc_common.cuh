@@ -337,6 +337,13 @@ __device__ __forceinline__ void stage_raw_fp8(const uint8_t* kt, const uint8_t* 
 #pragma unroll
         for (int j = 0; j < 2; ++j)
             r.k[i][j] = *reinterpret_cast<const uint4*>(kt + swz_chunk(gq + 8 * i, 2 * tq + j));
+    if (n == kStageTokens) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            r.v[i] = *reinterpret_cast<const uint4*>(
+                vt + swz_chunk(2 * tq + (i & 1) + 8 * (i >> 1), gq));
+        return;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int row = 2 * tq + (i & 1) + 8 * (i >> 1);
