@@ -378,9 +378,9 @@ __device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t y, uint32_t s
 __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const Fp8Raw& r, int n,
                                                float q_scale, float (&o)[8][4],
                                                float (&m_run)[2], float (&l_run)[2], int lane) {
-    float acc[4][4];
+    float acc[2][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
+    for (int a = 0; a < 2; ++a) acc[a][0] = acc[a][1] = acc[a][2] = acc[a][3] = 0.f;
     const uint32_t* k0 = reinterpret_cast<const uint32_t*>(&r.k[0][0]);   // row gq, 8 words
     const uint32_t* k1 = reinterpret_cast<const uint32_t*>(&r.k[1][0]);   // row gq + 8
 #pragma unroll
@@ -389,11 +389,11 @@ __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const
         uint32_t a[4];
         e4m3x4_to_f16x2(k0[kk], a[0], a[2]);
         e4m3x4_to_f16x2(k1[kk], a[1], a[3]);
-        MmaType<__half>::mma(acc[kk & 3], a, qb[kk][0], qb[kk][1]);
+        MmaType<__half>::mma(acc[kk & 1], a, qb[kk][0], qb[kk][1]);
     }
     float s[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) s[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) * q_scale;
+    for (int e = 0; e < 4; ++e) s[e] = (acc[0][e] + acc[1][e]) * q_scale;
     if (n < 16) mask_scores(s, n, lane);
     uint32_t pb0, pb1;
     softmax_step<__half, 8>(s, o, m_run, l_run, pb0, pb1);
