@@ -96,16 +96,16 @@ TRAFFIC = {
         (1.0123, "3d500856b22f29f4b5587277bc162b747071c43be02490f014a82dffad3bbe4e"),
     # 287.0 MB, 293.3 MB
     ("llama2_70b", 16, "decode_tc_kernel"):
-        (1.0217, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
-    # 1,346.1 MB, 1,359.6 MB
+        (1.0217, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
+    # 1,346.1 MB, 1,359.5 MB
     ("fp8", 16, "decode_tc_kernel"):
-        (1.0100, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
-    # 1,346.1 MB, 1,352.1 MB
+        (1.0099, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
+    # 1,346.1 MB, 1,351.6 MB
     ("fp8", 4, "decode_tc_kernel"):
-        (1.0044, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
-    # 143.5 MB, 149.4 MB
+        (1.0041, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
+    # 143.5 MB, 148.4 MB
     ("fp8_gqa", 16, "decode_tc_kernel"):
-        (1.0412, "100bf9931773bbf99838482997398d0d11f0206454e950d699c7d1916c96dd1f"),
+        (1.0340, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
     # 8.3 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
     # within a launch hit L2)
     ("falcon7b", 16, "decode_lean_kernel"):
