@@ -348,11 +348,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
     {
         float* cw = comb + warp * 8 * (D + 2);
         const int ra = 2 * tq, rb = ra + 1;
-        // o[j] rows: d = 16 j + gq and + 8 (FP8: d = 16 gq + 2 j and + 1)
+        // o[j] rows: d = 16 j + gq and + 8
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
-            const int d0 = EB == 1 ? 16 * gq + 2 * j : 16 * j + gq;
-            const int d1 = EB == 1 ? d0 + 1 : d0 + 8;
+            const int d0 = 16 * j + gq;
+            const int d1 = d0 + 8;
             cw[ra * (D + 2) + d0] = o[j][0];
             cw[rb * (D + 2) + d0] = o[j][1];
             cw[ra * (D + 2) + d1] = o[j][2];

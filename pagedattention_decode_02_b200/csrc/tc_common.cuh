@@ -58,6 +58,16 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+// Two 16 x 16 byte matrices, transposed: lanes 0-15 address the rows of the
+// first, lanes 16-31 those of the second; per matrix this lane receives rows
+// 4 (lane % 4) .. + 3 of column lane / 4 (one byte per row, in row order) in
+// the first register and of column lane / 4 + 8 in the second.
+__device__ __forceinline__ void ldsm_x2_t_b8(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                             uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
 
 // 2-D tiled TMA load of one box into shared memory, completion on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -293,13 +303,15 @@ __device__ __forceinline__ void stage_body_t(const uint32_t (&qb)[D / 16][2], co
 
 // ---------------------------------------------------------------------------
 // FP8-E4M3 pools (d = 128, f16 queries): the stage's K and V tiles hold codes
-// in 128-byte rows.  Each lane reads its codes with four 16-byte loads per
-// tile, contiguous and free of bank conflicts, and converts them to f16 in
-// registers.  To make that possible the d index is permuted, which leaves
-// both products unchanged (a sum over d in any order; O^T rows in any order):
+// in 128-byte rows, converted to f16 in registers.  K: each lane reads its
+// codes with four 16-byte loads, contiguous and free of bank conflicts, with
+// the d index of the score contraction permuted (a sum over d in any order):
 //   S^T k-step kk, fragment columns 2 tq + {0, 1} / 2 tq + {8, 9}
-//       <-> d = 32 tq + 4 kk + {0, 1} / + {2, 3};
-//   O^T m-tile mt, fragment row gq / gq + 8  <->  d = 16 gq + 2 mt / + 1.
+//       <-> d = 32 tq + 4 kk + {0, 1} / + {2, 3}.
+// V: four transposing byte-matrix loads give each lane, per 16-column
+// d-block, four consecutive tokens of one column, which are the A fragment's
+// contraction indices 2 tq, + 1, + 8, + 9 once the stage's tokens are taken
+// in that order on both products (fp8_token_of; K rows follow it too).
 // ---------------------------------------------------------------------------
 
 // Four FP8-E4M3 codes (one word, low byte first) -> two f16x2: lo = codes 0
@@ -320,10 +332,20 @@ __device__ __forceinline__ uint32_t swz_chunk(int r, int c) {
     return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
+// The contraction index r (0..15) of an FP8 stage and its token: the order
+// in which the transposed byte-matrix load hands a lane a column's tokens
+// (4 (lane % 4) .. + 3 = the indices 2 (lane % 4), + 1, + 8, + 9 of the
+// f16 A fragment).
+__device__ __forceinline__ int fp8_token_of(int r) {
+    return 4 * ((r >> 1) & 3) + 2 * (r >> 3) + (r & 1);
+}
+
 // This lane's codes of one stage:
-//   k[i][j]: K row gq + 8 i, bytes 32 tq + 16 j .. + 15;
-//   v[i]:    V row 2 tq + (i & 1) + 8 (i >> 1), bytes 16 gq .. 16 gq + 15
-//            (zero for rows at or past n).
+//   k[i][j]: K row fp8_token_of(gq + 8 i), bytes 32 tq + 16 j .. + 15;
+//   v[jj]:   V transposed, d-blocks 2 jj (.x, .y) and 2 jj + 1 (.z, .w) of 16
+//            columns: .x tokens 4 tq .. + 3 of column 16 (2 jj) + gq, .y the
+//            same tokens of that column + 8 (likewise .z, .w); codes of
+//            tokens at or past n are zero.
 struct Fp8Raw {
     uint4 k[2][2];
     uint4 v[4];
@@ -336,19 +358,23 @@ __device__ __forceinline__ void stage_raw_fp8(const uint8_t* kt, const uint8_t* 
     for (int i = 0; i < 2; ++i)
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-            r.k[i][j] = *reinterpret_cast<const uint4*>(kt + swz_chunk(gq + 8 * i, 2 * tq + j));
-    if (n == kStageTokens) {
+            r.k[i][j] = *reinterpret_cast<const uint4*>(
+                kt + swz_chunk(fp8_token_of(gq + 8 * i), 2 * tq + j));
+    const uint32_t vbase = smem_addr(vt);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            r.v[i] = *reinterpret_cast<const uint4*>(
-                vt + swz_chunk(2 * tq + (i & 1) + 8 * (i >> 1), gq));
-        return;
-    }
+    for (int jj = 0; jj < 4; ++jj)
+        ldsm_x2_t_b8(vbase + swz_chunk(lane & 15, 2 * jj + (lane >> 4)), r.v[jj].x, r.v[jj].y,
+                     r.v[jj].z, r.v[jj].w);
+    if (n < kStageTokens) {
+        const int valid = min(max(n - 4 * tq, 0), 4);   // of this lane's tokens 4 tq .. + 3
+        const uint32_t m = valid >= 4 ? 0xffffffffu : ((1u << (8 * valid)) - 1u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int row = 2 * tq + (i & 1) + 8 * (i >> 1);
-        r.v[i] = row < n ? *reinterpret_cast<const uint4*>(vt + swz_chunk(row, gq))
-                         : make_uint4(0u, 0u, 0u, 0u);
+        for (int jj = 0; jj < 4; ++jj) {
+            r.v[jj].x &= m;
+            r.v[jj].y &= m;
+            r.v[jj].z &= m;
+            r.v[jj].w &= m;
+        }
     }
 }
 
@@ -366,15 +392,10 @@ __device__ __forceinline__ void load_qT_frags_fp8(uint32_t (&qb)[8][2], const __
     }
 }
 
-__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t y, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(y), "r"(sel));
-    return d;
-}
-
 // The stage math of stage_math_t on an FP8 stage (scales folded by the
-// caller: q_scale includes k_scale, the output is multiplied by v_scale).
-// o[mt] = O^T rows d = 16 gq + 2 mt (o[mt][0..1]) and + 1 (o[mt][2..3]).
+// caller: q_scale includes k_scale, the output is multiplied by v_scale), the
+// stage's tokens taken in fp8_token_of order on both products.
+// o[mt] = O^T rows d = 16 mt + gq (o[mt][0..1]) and + 8 (o[mt][2..3]).
 __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const Fp8Raw& r, int n,
                                                float q_scale, float (&o)[8][4],
                                                float (&m_run)[2], float (&l_run)[2], int lane) {
@@ -394,28 +415,25 @@ __device__ __forceinline__ void stage_math_fp8(const uint32_t (&qb)[8][2], const
     float s[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) s[e] = (acc[0][e] + acc[1][e]) * q_scale;
-    if (n < 16) mask_scores(s, n, lane);
+    if (n < 16) {
+        // rows gq and gq + 8 of S^T are tokens fp8_token_of(gq) and that + 2
+        const int t0 = fp8_token_of(lane >> 2);
+        if (t0 >= n) s[0] = s[1] = -INFINITY;
+        if (t0 + 2 >= n) s[2] = s[3] = -INFINITY;
+    }
     uint32_t pb0, pb1;
     softmax_step<__half, 8>(s, o, m_run, l_run, pb0, pb1);
-    // V^T fragments: a token pair's codes of one d interleaved byte by byte
-    const uint32_t* x0 = reinterpret_cast<const uint32_t*>(&r.v[0]);   // token 2 tq
-    const uint32_t* y0 = reinterpret_cast<const uint32_t*>(&r.v[1]);   // token 2 tq + 1
-    const uint32_t* x1 = reinterpret_cast<const uint32_t*>(&r.v[2]);   // token 2 tq + 8
-    const uint32_t* y1 = reinterpret_cast<const uint32_t*>(&r.v[3]);   // token 2 tq + 9
+    // V^T fragments straight from the transposed codes: a word's low and high
+    // halves are a column's tokens at contraction indices 2 tq, + 1 and + 8, + 9
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        // word j: d = 16 gq + 4 j .. + 3 -> m-tiles 2 j (d + 0, + 1) and 2 j + 1 (d + 2, + 3)
-        const uint32_t lo01 = byte_perm(x0[j], y0[j], 0x5140u);
-        const uint32_t hi01 = byte_perm(x0[j], y0[j], 0x7362u);
-        const uint32_t lo23 = byte_perm(x1[j], y1[j], 0x5140u);
-        const uint32_t hi23 = byte_perm(x1[j], y1[j], 0x7362u);
-        uint32_t a0[4], a1[4];
-        e4m3x4_to_f16x2(lo01, a0[0], a0[1]);
-        e4m3x4_to_f16x2(lo23, a0[2], a0[3]);
-        MmaType<__half>::mma(o[2 * j], a0, pb0, pb1);
-        e4m3x4_to_f16x2(hi01, a1[0], a1[1]);
-        e4m3x4_to_f16x2(hi23, a1[2], a1[3]);
-        MmaType<__half>::mma(o[2 * j + 1], a1, pb0, pb1);
+    for (int jj = 0; jj < 4; ++jj) {
+        uint32_t a[4];
+        e4m3x4_to_f16x2(r.v[jj].x, a[0], a[2]);
+        e4m3x4_to_f16x2(r.v[jj].y, a[1], a[3]);
+        MmaType<__half>::mma(o[2 * jj], a, pb0, pb1);
+        e4m3x4_to_f16x2(r.v[jj].z, a[0], a[2]);
+        e4m3x4_to_f16x2(r.v[jj].w, a[1], a[3]);
+        MmaType<__half>::mma(o[2 * jj + 1], a, pb0, pb1);
     }
 }
 
