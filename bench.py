@@ -94,22 +94,22 @@ TRAFFIC = {
     # 605.3 MB algorithmic, 612.7 MB read + written
     ("opt13b", 16, "decode_simt2_kernel"):
         (1.0123, "3d500856b22f29f4b5587277bc162b747071c43be02490f014a82dffad3bbe4e"),
-    # 287.0 MB, 293.3 MB
+    # 287.0 MB, 293.0 MB
     ("llama2_70b", 16, "decode_tc_kernel"):
-        (1.0217, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
-    # 1,346.1 MB, 1,359.5 MB
+        (1.0206, "41088eff1f3e70d27c0838ec828e7bc4b6fb816a0c73fc2f08446899f6ee67fb"),
+    # 1,346.1 MB, 1,359.6 MB
     ("fp8", 16, "decode_tc_kernel"):
-        (1.0099, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
-    # 1,346.1 MB, 1,351.6 MB
+        (1.0100, "41088eff1f3e70d27c0838ec828e7bc4b6fb816a0c73fc2f08446899f6ee67fb"),
+    # 1,346.1 MB, 1,351.7 MB
     ("fp8", 4, "decode_tc_kernel"):
-        (1.0041, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
-    # 143.5 MB, 148.4 MB
+        (1.0041, "41088eff1f3e70d27c0838ec828e7bc4b6fb816a0c73fc2f08446899f6ee67fb"),
+    # 143.5 MB, 148.8 MB
     ("fp8_gqa", 16, "decode_tc_kernel"):
-        (1.0340, "e16d6927280b886ab8a80d2ec05591a1abd85cd223c89513c62eb143f15caa0a"),
+        (1.0370, "41088eff1f3e70d27c0838ec828e7bc4b6fb816a0c73fc2f08446899f6ee67fb"),
     # 8.3 MB, 3.0 MB (the samples of one prompt share its blocks; the re-reads
     # within a launch hit L2)
     ("falcon7b", 16, "decode_lean_kernel"):
-        (0.3593, "e2a75488c288e0bd0a4722ca2df2516788ab74b71ed6900530846a5d6a95cde7"),
+        (0.3593, "ce148d142c0abfb12978045714de63ba937c3f19448974ab10a4b1c96d8c6e00"),
 }
 KERNEL_SOURCES = {
     "decode_lean_kernel": ("decode_lean.cu", "tc_common.cuh", "kernels_common.cuh"),
