@@ -59,3 +59,21 @@ def test_bench_traffic_only_at_the_captured_block_size():
     cfg = wl.CONFIGS["fp8"]
     assert bench.traffic_per_launch(cfg.with_block_size(1), "decode_simt2_kernel", 1e9) is None
     assert bench.traffic_per_launch(cfg, "no_such_kernel", 1e9) is None
+
+
+def test_bench_roofline_recomputes_from_its_own_fields():
+    # achieved = profiled_bytes / (profiled_launches x decode_ms_mean), and
+    # frac = achieved / peak, from the printed fields alone
+    import bench
+    cfg = wl.CONFIGS["opt13b"]
+    m = {"kernel": "decode_simt2_kernel", "dec_ms": [0.110, 0.108, 0.112],
+         "prof_bytes": [605_000_000, 604_000_000, 606_000_000],
+         "step_bytes": [605_000_000] * 9, "merge_ms": [0.0, 0.0, 0.0],
+         "pro_ms": [0.007, 0.008, 0.0075], "prof_batches": [0, 1, 2], "prof_every": 3, "R": 8}
+    r = bench.roofline_of(cfg, m, 6650.0, "fallback")
+    n = r["profiled_launches"]
+    assert n == 3 and r["profiled_bytes"] == sum(m["prof_bytes"])
+    achieved = r["profiled_bytes"] / n / (r["decode_ms_mean"] / 1e3) / 1e9
+    assert abs(achieved - r["achieved"]) <= 0.01 * achieved
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-4
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
