@@ -139,6 +139,18 @@ void kv_pool_destroy(pkv_pool* pool);
 /* kv_pool_get_info - fills *info (device pointers, sizes, scales). */
 pkv_status kv_pool_get_info(const pkv_pool* pool, pkv_pool_info* info);
 
+/* kv_pool_check_guards - a debugging check of the pool's own buffers.  A pool
+ *   that allocated its K and V buffers keeps one guard block (the block size
+ *   rounded up to 256 bytes) of a fixed byte before and after each of them;
+ *   no call of the library writes there, so a changed byte means a write out
+ *   of the pool's bounds.  Waits for all work on the pool's device
+ *   (cudaDeviceSynchronize), copies the four guard regions to the host and
+ *   sets *intact to 1 if every byte still holds the guard value, else 0.
+ *   Pools on caller-owned buffers and host-only pools have no guards:
+ *   *intact = 1.  Errors: INVALID_ARG (NULL argument, another current
+ *   device), CUDA (the wait or a copy failed). */
+pkv_status kv_pool_check_guards(const pkv_pool* pool, int* intact);
+
 /* ---------------------------------------------------------------------------
  * Block tables (host; [F55] §块表, FAQ 08; [IPLEX] §分离逻辑顺序与实际存储位置,
  * §同一提示生成两个回答的假想例子).  Free-queue policy: FIFO; a block is taken from

@@ -97,6 +97,7 @@ _sig("kv_pool_create", _st, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_i
      ctypes.POINTER(_P))
 _sig("kv_pool_destroy", None, _P)
 _sig("kv_pool_get_info", _st, _P, ctypes.POINTER(pkv_pool_info))
+_sig("kv_pool_check_guards", _st, _P, ctypes.POINTER(ctypes.c_int))
 _sig("bt_reset", _st, _P, _I32P)
 _sig("bt_alloc", _st, _P, ctypes.c_int64, ctypes.c_int, _I32P)
 _sig("bt_append", _st, _P, ctypes.c_int64, _I32P, _I32P, _I32P)
@@ -146,7 +147,7 @@ _sig("pkv_step_profile_read", _st, _P, ctypes.POINTER(ctypes.c_float), ctypes.PO
      ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.POINTER(ctypes.c_int))
 
 EXPORTED = [
-    "kv_pool_create", "kv_pool_destroy", "kv_pool_get_info", "bt_reset", "bt_alloc", "bt_append",
+    "kv_pool_create", "kv_pool_destroy", "kv_pool_get_info", "kv_pool_check_guards", "bt_reset", "bt_alloc", "bt_append",
     "bt_append_batch", "bt_fork", "bt_free", "bt_export", "bt_num_blocks", "bt_refcount",
     "bt_free_queue", "bt_stats", "kv_append", "block_copy", "paged_decode_attention",
     "paged_decode_attention_ex", "paged_decode_workspace_bytes", "paged_decode_workspace_bytes_ex",
@@ -472,6 +473,14 @@ def pkv_set_wait_budget(pool: Pool, budget_ns: int) -> None:
 def pkv_wait_probe(pool: Pool, stream=None) -> None:
     """Queue the probe kernel: a wait that nothing completes, with the pool's budget."""
     _check(_lib.pkv_wait_probe(pool.handle, _stream_ptr(stream)), "pkv_wait_probe")
+
+
+def kv_pool_check_guards(pool: Pool) -> bool:
+    """Wait for the device; True when the guard blocks around the pool's own
+    K/V buffers still hold their fixed byte (always True without guards)."""
+    ok = ctypes.c_int(0)
+    _check(_lib.kv_pool_check_guards(pool.handle, ctypes.byref(ok)), "kv_pool_check_guards")
+    return bool(ok.value)
 
 
 def pkv_device_error(pool: Pool, stream=None) -> int:

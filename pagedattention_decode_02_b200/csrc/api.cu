@@ -170,16 +170,30 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
             p->v = static_cast<uint8_t*>(v_buf);
             p->owns_buffers = false;
         } else {
-            if (cudaMalloc(&p->k, bytes) != cudaSuccess) {
+            // each buffer between two guard blocks of a known byte
+            const size_t g = ((bytes / num_blocks) + 255) & ~(size_t)255;
+            if (cudaMalloc(&p->k_alloc, bytes + 2 * g) != cudaSuccess) {
                 delete p;
                 return PKV_ERR_CUDA;
             }
-            if (cudaMalloc(&p->v, bytes) != cudaSuccess) {
-                cudaFree(p->k);
+            if (cudaMalloc(&p->v_alloc, bytes + 2 * g) != cudaSuccess) {
+                cudaFree(p->k_alloc);
                 delete p;
                 return PKV_ERR_CUDA;
             }
+            p->guard = g;
+            p->k = p->k_alloc + g;
+            p->v = p->v_alloc + g;
             p->owns_buffers = true;
+            if (cudaMemset(p->k_alloc, pkv_pool::kGuardByte, g) != cudaSuccess ||
+                cudaMemset(p->k + bytes, pkv_pool::kGuardByte, g) != cudaSuccess ||
+                cudaMemset(p->v_alloc, pkv_pool::kGuardByte, g) != cudaSuccess ||
+                cudaMemset(p->v + bytes, pkv_pool::kGuardByte, g) != cudaSuccess) {
+                cudaFree(p->k_alloc);
+                cudaFree(p->v_alloc);
+                delete p;
+                return PKV_ERR_CUDA;
+            }
         }
         // the error word, then (256 bytes in) the prompt kernel's counters
         constexpr size_t kSchedOff = 256;
@@ -187,8 +201,8 @@ pkv_status kv_pool_create(int num_blocks, int block_size, int n_kv_heads, int he
         if (cudaMalloc(&p->d_err, err_bytes) != cudaSuccess ||
             cudaMemset(p->d_err, 0, err_bytes) != cudaSuccess) {
             if (p->owns_buffers) {
-                cudaFree(p->k);
-                cudaFree(p->v);
+                cudaFree(p->k_alloc);
+                cudaFree(p->v_alloc);
             }
             if (p->d_err) cudaFree(p->d_err);
             delete p;
@@ -210,12 +224,32 @@ void kv_pool_destroy(pkv_pool* p) {
     if (!p) return;
     if (!p->host_only) {
         if (p->owns_buffers) {
-            cudaFree(p->k);
-            cudaFree(p->v);
+            cudaFree(p->k_alloc);
+            cudaFree(p->v_alloc);
         }
         cudaFree(p->d_err);
     }
     delete p;
+}
+
+pkv_status kv_pool_check_guards(const pkv_pool* p, int* intact) {
+    if (!p || !intact) return PKV_ERR_INVALID_ARG;
+    *intact = 1;
+    if (p->host_only || !p->owns_buffers || p->guard == 0) return PKV_OK;
+    if (!same_device(p)) return PKV_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PKV_ERR_CUDA;
+    std::vector<uint8_t> h(p->guard);
+    const uint8_t* regions[4] = {p->k_alloc, p->k + p->bytes, p->v_alloc, p->v + p->bytes};
+    for (const uint8_t* r : regions) {
+        if (cudaMemcpy(h.data(), r, p->guard, cudaMemcpyDeviceToHost) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        for (uint8_t b : h)
+            if (b != pkv_pool::kGuardByte) {
+                *intact = 0;
+                return PKV_OK;
+            }
+    }
+    return PKV_OK;
 }
 
 pkv_status kv_pool_get_info(const pkv_pool* p, pkv_pool_info* info) {

@@ -25,6 +25,13 @@ struct pkv_pool {
     uint8_t* k = nullptr;   // device [num_blocks][n_kv_heads][block_size][head_dim]
     uint8_t* v = nullptr;
     size_t bytes = 0;       // bytes of one of the two buffers
+    // buffers the pool allocated itself: one guard block (rounded up to 256
+    // bytes) before and after each, filled with kGuardByte and never written
+    // by the library; k_alloc / v_alloc are the allocations (k = k_alloc + guard)
+    static constexpr unsigned char kGuardByte = 0xA5;
+    uint8_t* k_alloc = nullptr;
+    uint8_t* v_alloc = nullptr;
+    size_t guard = 0;
     uint32_t* d_err = nullptr;
     // work counters of the prompt kernel's dynamic schedule: kPrefillSlots
     // pairs {next item, CTAs done}, one pair per launch in flight (launch i
