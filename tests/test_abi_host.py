@@ -248,3 +248,12 @@ def test_utilisation_readout_fp8_sweep(bs):
         assert st["logical_tokens"] == st["table_slots"]
     # reserving the maximum length (2,048 + 1) up front stores about half as much
     assert float(max_reservation_utilisation(ctx, 2049)) < 0.55
+
+
+def test_guard_check_on_a_host_only_pool():
+    # no device buffers, no guards: reported intact without touching a device
+    pool = pk.kv_pool_create(16, 4, 2, 64, "f16", host_only=True)
+    assert pk.kv_pool_check_guards(pool)
+    pool.close()
+    st = pk._lib.kv_pool_check_guards(None, None)
+    assert st == pk.PKV_ERR_INVALID_ARG
